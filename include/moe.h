@@ -1,0 +1,159 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) quantized Mixture-of-Experts expert block.
+ *
+ * Per layer the library computes, for every token t of the hidden states x [T x H]:
+ *   logits l = W_r x (+ bias); the k experts with the largest logits (ties -> lower index);
+ *   routing weights = softmax over those k logits; for each selected expert e the FFN
+ *   y_e = Wd_e (silu(Wg_e x) * (Wu_e x)) with group-affine low-bit weights
+ *   W[r,c] = (q[r,c] - z[r,c/64]) * s[r,c/64]; and out[t] = sum_i w_i y_{e_i}.
+ * This is the MoE expert block that the pages "Krasis update" (HQQ 4/6/8-bit experts),
+ * "--moe-direct-io" / "Qwen-tin" (512 experts, top-10 routing) and "Raon-1-mini on an
+ * RTX 5070 Ti" (table rows "MoE megakernel" and "Pipelined megakernel": one persistent kernel
+ * per layer's expert block, next expert loaded while the current one computes) run in their
+ * decode and prefill loops; the pages print no formula, so the steps above are the plain
+ * reading of router top-k + softmax renormalisation, affine group dequantisation, gate/up,
+ * SiLU-GLU, down and a routing-weighted combine.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked (device) are CUDA device pointers owned by the caller; the library never
+ *    frees or retains them. Pointers marked (host) are read during the call only.
+ *  - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *  - All arguments are validated on the host before anything is launched; a bad argument
+ *    returns MOE_ERR_INVALID_ARG (or MOE_ERR_UNSUPPORTED for a valid but unsupported shape)
+ *    and launches nothing. A failed launch returns MOE_ERR_CUDA.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the call
+ *    returns without synchronising, except moe_get_device_status.
+ *  - No entry point allocates device memory: scratch space is the caller's workspace.
+ *  - Two calls that share a workspace must be ordered (same stream, or events); calls with
+ *    distinct workspaces may run concurrently.
+ *  - The library supports sm_100a (B200) only; on any other device calls return
+ *    MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a pointer to the runtime's opaque stream struct). */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, workspace too small */
+    MOE_ERR_UNSUPPORTED = 2,   /* shape or device outside what the kernels implement */
+    MOE_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    MOE_ERR_TIMEOUT = 4,       /* a bounded device-side wait expired (see moe_get_device_status) */
+    MOE_ERR_DEVICE_CHECK = 5   /* a device-side consistency check failed */
+} moe_status_t;
+
+/* Human-readable name of a status (static string, never NULL). */
+const char *moe_status_str(moe_status_t s);
+
+/* ABI version of this header: 1. */
+int moe_abi_version(void);
+
+/* ---------------------------------------------------------------------------------------
+ * Expert weights.
+ *
+ * Canonical (input) format of one expert, the format a quantiser hands over. Matrix m is
+ * 0 = gate [I x H], 1 = up [I x H], 2 = down [H x I] (rows x cols; the input dimension is
+ * the column dimension). For each matrix (all pointers device, 16-byte aligned):
+ *   codes[m]: rows x (cols*bits/8) bytes, row-major. Group g of a row (columns 64g..64g+63)
+ *             is a block of 8*bits bytes; code j of the group occupies bits
+ *             [j*bits, (j+1)*bits) of that block read as one little-endian bit string.
+ *   scale[m], zero[m]: fp16 [rows x cols/64], row-major; W[r,c] = (q - zero) * scale.
+ * bits is 4, 6 or 8 and may differ between the experts of one layer.
+ * ------------------------------------------------------------------------------------- */
+typedef struct moe_expert_src {
+    const void *codes[3];
+    const uint16_t *scale[3];
+    const uint16_t *zero[3];
+    int32_t bits;
+} moe_expert_src_t;
+
+/* Bytes of the packed form of one layer of E experts with per-expert widths bits[E] (host).
+ * Returns 0 if an argument is invalid (H or I not a multiple of 64, E < 1, bits not in
+ * {4,6,8}). */
+size_t moe_packed_layer_bytes(int E, int H, int I, const int32_t *bits);
+
+/* Converts one layer's experts from the canonical format (src: host array of E descriptors
+ * whose pointers are device pointers) into the packed form the forward kernels read, written
+ * to `packed` (device, 256-byte aligned, packed_bytes >= moe_packed_layer_bytes). The packed
+ * form is self-describing (it records E, H, I and each expert's width). The conversion is a
+ * byte permutation: no value is rounded. Asynchronous on `stream`; the canonical buffers
+ * must stay valid until it completes. */
+moe_status_t moe_pack_layer(const moe_expert_src_t *src, int E, int H, int I, void *packed,
+                            size_t packed_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Routing alone.
+ *
+ * x (device) bf16 [T x H]; w_router (device) fp32 [E x H]; bias (device) fp32 [E] or NULL.
+ * Writes idx_out (device) int32 [T x k], experts in descending logit order (ties -> lower
+ * index), and w_out (device) fp32 [T x k], the softmax of those k logits. Logits are fp32
+ * dot products of the bf16 x with the fp32 router rows.
+ * Limits: 1 <= T, H % 64 == 0, 1 <= k <= min(E, 32), E <= 1024. No workspace.
+ * ------------------------------------------------------------------------------------- */
+moe_status_t moe_route_topk(const uint16_t *x, const float *w_router, const float *bias, int T,
+                            int H, int E, int k, int32_t *idx_out, float *w_out,
+                            moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Whole expert block.
+ * ------------------------------------------------------------------------------------- */
+enum { MOE_MODE_DECODE = 0, MOE_MODE_PREFILL = 1 };
+
+/* Workspace bytes needed by a forward call of the given mode and shape (0 if invalid). */
+size_t moe_workspace_bytes(int T, int H, int I, int E, int k, int mode);
+
+/* Prepares a workspace (device, 256-byte aligned) for first use: clears its control words.
+ * Needed once after allocation; the forward calls keep it consistent afterwards. */
+moe_status_t moe_workspace_init(void *workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* Decode path, 1 <= T <= 32: one persistent kernel per call (routing, gate/up, SiLU-GLU,
+ * down and combine fused; intermediates stay on chip or in L2). Launched with programmatic
+ * dependent launch so that consecutive layer calls overlap their start-up.
+ *   x (device) bf16 [T x H]; w_router (device) fp32 [E x H]; bias (device) fp32 [E] or NULL;
+ *   packed (device) one layer in moe_pack_layer form with the same E, H, I;
+ *   out (device) bf16 [T x H]; idx_out (device) int32 [T x k] or NULL; w_out (device) fp32
+ *   [T x k] or NULL; workspace (device) of ws_bytes >= moe_workspace_bytes(..., DECODE),
+ *   prepared by moe_workspace_init.
+ * Limits: H % 64 == 0, I % 64 == 0, 1 <= k <= min(E, 32), E <= 1024.
+ * A bounded device-side wait that expires leaves `out` undefined and sets the workspace's
+ * status word (read it with moe_get_device_status). */
+moe_status_t moe_expert_forward_decode(const uint16_t *x, const float *w_router,
+                                       const float *bias, const void *packed, int T, int H,
+                                       int I, int E, int k, uint16_t *out, int32_t *idx_out,
+                                       float *w_out, void *workspace, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/* Prefill path, any T >= 1: routing, bucketing of the T*k (token, expert) pairs per expert
+ * (stable: ascending token within an expert), a grouped gate/up GEMM with a SiLU-GLU
+ * epilogue and a grouped down GEMM whose epilogue adds the routing-weighted rows into the
+ * output. Arguments as for moe_expert_forward_decode, with the PREFILL workspace size. */
+moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router,
+                                        const float *bias, const void *packed, int T, int H,
+                                        int I, int E, int k, uint16_t *out, int32_t *idx_out,
+                                        float *w_out, void *workspace, size_t ws_bytes,
+                                        moe_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace's device status word and maps it to a status:
+ * MOE_OK, MOE_ERR_TIMEOUT (a bounded wait expired) or MOE_ERR_DEVICE_CHECK. A non-zero word
+ * is cleared together with the workspace's other control words, so the workspace is ready for
+ * the next call. */
+moe_status_t moe_get_device_status(void *workspace, moe_stream_t stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait (grid barriers, copy completion).
+ * Default 2e9 (2 s). Values are clamped to [0, 6e10]; 0 makes every wait that is not
+ * already satisfied expire at once, which tests use to exercise the timeout path. */
+void moe_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

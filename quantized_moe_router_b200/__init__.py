@@ -1,0 +1,178 @@
+"""Python binding of the quantized MoE expert block's C ABI (include/moe.h).
+
+Argument marshalling only: every step of the block runs in the CUDA library
+``libmoe_b200.so`` built in-tree by ``quantized_moe_router_b200/build.py``. PyTorch provides
+device memory and streams. There is no fallback: if the library is missing or the device is
+not an sm_100a GPU, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_CHECK = range(6)
+MODE_DECODE, MODE_PREFILL = 0, 1
+
+# every C entry point of include/moe.h with its ctypes signature
+_vp, _i, _sz, _u64 = C.c_void_p, C.c_int, C.c_size_t, C.c_uint64
+SIGNATURES = {
+    "moe_status_str": (C.c_char_p, [_i]),
+    "moe_abi_version": (_i, []),
+    "moe_packed_layer_bytes": (_sz, [_i, _i, _i, _vp]),
+    "moe_pack_layer": (_i, [_vp, _i, _i, _i, _vp, _sz, _vp]),
+    "moe_route_topk": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "moe_workspace_init": (_i, [_vp, _sz, _vp]),
+    "moe_expert_forward_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_forward_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_get_device_status": (_i, [_vp, _vp]),
+    "moe_set_wait_limit_ns": (None, [_u64]),
+}
+
+
+class ExpertSrc(C.Structure):
+    """moe_expert_src_t"""
+    _fields_ = [("codes", C.c_void_p * 3), ("scale", C.c_void_p * 3), ("zero", C.c_void_p * 3),
+                ("bits", C.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what} failed: {status_name(status)}")
+        self.status = status
+
+
+_lib: Optional[C.CDLL] = None
+
+
+def lib() -> C.CDLL:
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; run quantized_moe_router_b200/build.py "
+                               "(or __graft_entry__.build())")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_name(status: int) -> str:
+    return lib().moe_status_str(status).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(what, status)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _p(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+# ------------------------------------------------------------------------------ weights
+
+def packed_layer_bytes(E: int, H: int, I: int, bits: Sequence[int]) -> int:
+    arr = (C.c_int32 * E)(*[int(b) for b in bits])
+    n = lib().moe_packed_layer_bytes(E, H, I, C.cast(arr, C.c_void_p))
+    if n == 0:
+        raise MoeError("moe_packed_layer_bytes", MOE_ERR_INVALID_ARG)
+    return n
+
+
+def pack_layer(experts: Sequence[dict], H: int, I: int, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """experts[e] = {"bits": b, "codes": [3 uint8 tensors], "scale": [3 fp16/int16 tensors],
+    "zero": [...]} on the GPU, canonical layout. Returns the packed layer (uint8 tensor)."""
+    E = len(experts)
+    bits = [int(ex["bits"]) for ex in experts]
+    nbytes = packed_layer_bytes(E, H, I, bits)
+    dev = experts[0]["codes"][0].device
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    src = (ExpertSrc * E)()
+    for e, ex in enumerate(experts):
+        for m in range(3):
+            src[e].codes[m] = ex["codes"][m].data_ptr()
+            src[e].scale[m] = ex["scale"][m].data_ptr()
+            src[e].zero[m] = ex["zero"][m].data_ptr()
+        src[e].bits = bits[e]
+    _check(lib().moe_pack_layer(C.cast(src, C.c_void_p), E, H, I, out.data_ptr(), out.numel(), _stream(stream)),
+           "moe_pack_layer")
+    return out
+
+
+# ------------------------------------------------------------------------------ routing
+
+def route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Tensor], k: int,
+               idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None, stream=None):
+    T, H = x.shape
+    E = w_router.shape[0]
+    if idx_out is None:
+        idx_out = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    if w_out is None:
+        w_out = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib().moe_route_topk(_p(x), _p(w_router), _p(bias), T, H, E, k, _p(idx_out), _p(w_out),
+                                _stream(stream)), "moe_route_topk")
+    return idx_out, w_out
+
+
+# ------------------------------------------------------------------------------ expert block
+
+def workspace_bytes(T: int, H: int, I: int, E: int, k: int, mode: int) -> int:
+    n = lib().moe_workspace_bytes(T, H, I, E, k, mode)
+    if n == 0:
+        raise MoeError("moe_workspace_bytes", MOE_ERR_INVALID_ARG)
+    return n
+
+
+def workspace(T: int, H: int, I: int, E: int, k: int, mode: int, device="cuda", stream=None) -> torch.Tensor:
+    ws = torch.empty(workspace_bytes(T, H, I, E, k, mode), dtype=torch.uint8, device=device)
+    _check(lib().moe_workspace_init(ws.data_ptr(), ws.numel(), _stream(stream)), "moe_workspace_init")
+    return ws
+
+
+def _forward(fn, what, x, w_router, bias, packed, I, E, k, ws, out, idx_out, w_out, stream):
+    T, H = x.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(fn(_p(x), _p(w_router), _p(bias), _p(packed), T, H, I, E, k, _p(out), _p(idx_out), _p(w_out),
+              _p(ws), ws.numel(), _stream(stream)), what)
+    return out
+
+
+def forward_decode(x, w_router, bias, packed, I, E, k, ws, out=None, idx_out=None, w_out=None, stream=None):
+    """Decode-path expert block (T <= 32): returns out [T x H] bf16."""
+    return _forward(lib().moe_expert_forward_decode, "moe_expert_forward_decode", x, w_router, bias, packed,
+                    I, E, k, ws, out, idx_out, w_out, stream)
+
+
+def forward_prefill(x, w_router, bias, packed, I, E, k, ws, out=None, idx_out=None, w_out=None, stream=None):
+    """Prefill-path expert block (any T): returns out [T x H] bf16."""
+    return _forward(lib().moe_expert_forward_prefill, "moe_expert_forward_prefill", x, w_router, bias, packed,
+                    I, E, k, ws, out, idx_out, w_out, stream)
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the workspace's device status."""
+    return lib().moe_get_device_status(ws.data_ptr(), _stream(stream))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().moe_set_wait_limit_ns(int(ns))

@@ -1,0 +1,80 @@
+"""Launch sequencing for a stack of decode layers: one CUDA graph per step.
+
+Plumbing only: the graph holds one moe_expert_forward_decode launch per layer (each a
+programmatic-dependent launch, so layer l+1's CTAs are scheduled while layer l finishes) and
+nothing else; all arithmetic is in the CUDA library.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import MODE_DECODE, MODE_PREFILL, forward_decode, forward_prefill, workspace
+
+
+class LayerWeights:
+    """Device tensors of one layer: router [E x H] fp32, optional bias [E], packed experts."""
+
+    def __init__(self, wr: torch.Tensor, bias: Optional[torch.Tensor], packed: torch.Tensor):
+        self.wr, self.bias, self.packed = wr, bias, packed
+
+
+class DecodeStack:
+    """L decode layers of the same shape sharing one workspace, replayed as one CUDA graph.
+
+    x_in[l] / out[l] are fixed device buffers (T x H bf16) that the graph reads and writes.
+    """
+
+    def __init__(self, layers: Sequence[LayerWeights], T: int, H: int, I: int, E: int, k: int,
+                 device="cuda", with_routing_outputs: bool = True):
+        self.layers = list(layers)
+        self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        L = len(self.layers)
+        self.ws = workspace(T, H, I, E, k, MODE_DECODE, device)
+        self.x_in = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
+        self.out = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
+        self.idx = torch.zeros((L, T, k), dtype=torch.int32, device=device) if with_routing_outputs else None
+        self.wts = torch.zeros((L, T, k), dtype=torch.float32, device=device) if with_routing_outputs else None
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+
+    def launch(self, stream=None):
+        for l, lw in enumerate(self.layers):
+            forward_decode(self.x_in[l], lw.wr, lw.bias, lw.packed, self.I, self.E, self.k, self.ws,
+                           out=self.out[l], idx_out=None if self.idx is None else self.idx[l],
+                           w_out=None if self.wts is None else self.wts[l], stream=stream)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.launch()          # warm-up outside the graph (also sets kernel attributes)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.launch()
+        self.graph = g
+        return g
+
+    def replay(self):
+        if self.graph is None:
+            self.capture()
+        self.graph.replay()
+
+
+class PrefillStack:
+    """L prefill layers of the same shape sharing one workspace, launched back to back."""
+
+    def __init__(self, layers: Sequence[LayerWeights], T: int, H: int, I: int, E: int, k: int, device="cuda"):
+        self.layers = list(layers)
+        self.T, self.H, self.I, self.E, self.k = T, H, I, E, k
+        L = len(self.layers)
+        self.ws = workspace(T, H, I, E, k, MODE_PREFILL, device)
+        self.x_in = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
+        self.out = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
+
+    def launch(self, stream=None):
+        for l, lw in enumerate(self.layers):
+            forward_prefill(self.x_in[l], lw.wr, lw.bias, lw.packed, self.I, self.E, self.k, self.ws,
+                            out=self.out[l], stream=stream)

@@ -1,0 +1,98 @@
+"""The C-ABI library: builds for sm_100a, loads, exports every entry point declared in
+include/moe.h, and rejects bad arguments on the host before touching the GPU (CPU only)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from tests_support import ROOT
+import quantized_moe_router_b200 as qm
+from quantized_moe_router_b200 import build as qbuild
+
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if qbuild.stale():
+        qbuild.build()
+    return qm.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("moe_route_topk", "moe_expert_forward_decode", "moe_expert_forward_prefill", "moe_pack_layer"):
+        assert n in names
+    assert set(names) == set(qm.SIGNATURES), set(names) ^ set(qm.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    assert L.moe_abi_version() == 1
+    names = [qm.status_name(s) for s in range(6)]
+    assert names == ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
+                     "MOE_ERR_DEVICE_CHECK"]
+
+
+def test_packed_layer_bytes(L):
+    # 4-bit tile = 512 B codes + 64 B scale/zero; an expert has 3*I*H/1024 tiles; experts are
+    # 256-byte aligned after a 32-byte header and 16 bytes per expert entry.
+    E, H, I = 256, 2048, 512
+    per_expert = 3 * I * H // 1024 * 576
+    assert per_expert == 1769472  # = the canonical bytes: I*H*3/2 codes + 4 bytes per group
+    head = (32 + 16 * E + 255) // 256 * 256
+    assert qm.packed_layer_bytes(E, H, I, [4] * E) == head + E * per_expert
+    mixed = [4, 6, 8]
+    per = {4: 576, 6: 832, 8: 1088}
+    want = (32 + 16 * 3 + 255) // 256 * 256
+    for b in mixed:
+        want += (3 * 64 * 128 // 1024 * per[b] + 255) // 256 * 256
+    assert qm.packed_layer_bytes(3, 128, 64, mixed) == want
+    arr = (C.c_int32 * 2)(4, 5)
+    assert L.moe_packed_layer_bytes(2, 128, 64, C.cast(arr, C.c_void_p)) == 0
+    arr = (C.c_int32 * 1)(4)
+    assert L.moe_packed_layer_bytes(1, 100, 64, C.cast(arr, C.c_void_p)) == 0
+
+
+def test_workspace_bytes_validation(L):
+    assert L.moe_workspace_bytes(1, 2048, 512, 256, 8, 0) > 0
+    assert L.moe_workspace_bytes(4096, 2048, 512, 256, 8, 1) > L.moe_workspace_bytes(1, 2048, 512, 256, 8, 1)
+    for bad in [(0, 2048, 512, 256, 8, 0), (1, 2000, 512, 256, 8, 0), (1, 2048, 500, 256, 8, 0),
+                (1, 2048, 512, 256, 0, 0), (1, 2048, 512, 4, 8, 0), (1, 2048, 512, 2048, 8, 0),
+                (1, 2048, 512, 256, 33, 0), (1, 2048, 512, 256, 8, 7)]:
+        assert L.moe_workspace_bytes(*bad) == 0, bad
+
+
+def test_host_validation_before_any_launch(L):
+    fake = 1 << 20  # aligned non-null address; never dereferenced because validation fails first
+    ws_small = 16
+    rc = L.moe_expert_forward_decode(fake, fake, None, fake, 1, 2048, 512, 256, 8, fake, None, None, fake, ws_small, None)
+    assert rc == qm.MOE_ERR_INVALID_ARG
+    rc = L.moe_expert_forward_prefill(fake, fake, None, fake, 4, 2048, 512, 256, 8, fake, None, None, fake, ws_small, None)
+    assert rc == qm.MOE_ERR_INVALID_ARG
+    rc = L.moe_expert_forward_decode(None, fake, None, fake, 1, 2048, 512, 256, 8, fake, None, None, fake, 1 << 30, None)
+    assert rc == qm.MOE_ERR_INVALID_ARG
+    rc = L.moe_expert_forward_decode(fake + 2, fake, None, fake, 1, 2048, 512, 256, 8, fake, None, None, fake, 1 << 30, None)
+    assert rc == qm.MOE_ERR_INVALID_ARG  # x not 16-byte aligned
+    rc = L.moe_expert_forward_decode(fake, fake, None, fake + 16, 1, 2048, 512, 256, 8, fake, None, None, fake, 1 << 30, None)
+    assert rc == qm.MOE_ERR_INVALID_ARG  # packed layer not 256-byte aligned
+    assert L.moe_route_topk(fake, fake, None, 1, 100, 8, 2, fake, fake, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_route_topk(fake, fake, None, 1, 128, 8, 9, fake, fake, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_route_topk(fake, None, None, 1, 128, 8, 2, fake, fake, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_layer(None, 1, 128, 64, fake, 1 << 20, None) == qm.MOE_ERR_INVALID_ARG
+    src = (qm.ExpertSrc * 1)()
+    src[0].bits = 5
+    assert L.moe_pack_layer(C.cast(src, C.c_void_p), 1, 128, 64, fake, 1 << 20, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_init(None, 1024, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_get_device_status(None, None) == qm.MOE_ERR_INVALID_ARG

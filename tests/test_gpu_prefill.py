@@ -1,0 +1,59 @@
+"""Prefill path (moe_expert_forward_prefill) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import quantized_moe_router_b200 as qm
+from gpu_support import HandLayer, SynthLayer, bf16_f64, to_dev_bf16
+from parity import check_block
+from tests_support import pins_module
+
+pytestmark = pytest.mark.gpu
+pins = pins_module()
+
+
+def prefill_call(layer, x_bits, I, E, k):
+    T, H = x_bits.shape
+    ws = qm.workspace(T, H, I, E, k, qm.MODE_PREFILL)
+    idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+    w = torch.zeros((T, k), dtype=torch.float32, device="cuda")
+    out = qm.forward_prefill(to_dev_bf16(x_bits), layer.wr, layer.bias, layer.packed, I, E, k, ws,
+                             idx_out=idx, w_out=w)
+    assert qm.device_status(ws) == qm.MOE_OK
+    return bf16_f64(out), idx.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,H,I,k,widths", [
+    (1, 8, 128, 64, 2, [4]), (7, 6, 192, 128, 2, [6]), (64, 5, 64, 64, 3, [8]), (300, 9, 256, 192, 4, [4, 6, 8]),
+    (129, 33, 128, 64, 8, [4, 8]), (40, 16, 320, 128, 16, [6, 4])])
+def test_prefill_hand_layers(T, E, H, I, k, widths):
+    rng = np.random.default_rng(T * 10 + E)
+    exs = [pins.make_expert(rng, H, I, widths[e % len(widths)])[0] for e in range(E)]
+    wr = (rng.normal(0, 1, (E, H)) / np.sqrt(H)).astype(np.float32)
+    b = rng.normal(0, 0.3, E).astype(np.float32)
+    layer = HandLayer(exs, wr, b, H, I)
+    x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
+    out, idx, w = prefill_call(layer, x, I, E, k)
+    check_block(oracle.get(), x, wr, b, layer.expert_fn, E, H, I, k, out, idx, w)
+
+
+def test_prefill_full_size_sampled_tokens():
+    w = synth.WORKLOADS["prefill_t4096_l8_h2048_e256_k8_i512_int4"]
+    layer = SynthLayer(w, 3)
+    x = synth.hidden(w, 0, 3)
+    out, idx, ww = prefill_call(layer, x, w.I, w.E, w.k)
+    rng = np.random.default_rng(0)
+    tokens = np.sort(np.concatenate([[0, 1, w.T - 1], rng.choice(w.T, 21, replace=False)]))
+    print(check_block(oracle.get(), x, layer.wr_np, None, layer.expert_fn, w.E, w.H, w.I, w.k, out, idx, ww,
+                      tokens=tokens))
+
+
+def test_prefill_agrees_with_decode_on_small_batch():
+    w = synth.WORKLOADS["decode_t16_l24_h2048_e256_k8_i768_mixed468_zipf1.1"]
+    layer = SynthLayer(w, 2)
+    x = synth.hidden(w, 1, 2)
+    o = oracle.get()
+    out_p, idx_p, w_p = prefill_call(layer, x, w.I, w.E, w.k)
+    check_block(o, x, layer.wr_np, layer.bias_np, layer.expert_fn, w.E, w.H, w.I, w.k, out_p, idx_p, w_p)
