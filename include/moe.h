@@ -118,9 +118,9 @@ moe_status_t moe_workspace_init(void *workspace, size_t ws_bytes, moe_stream_t s
 /* Decode path, 1 <= T <= 32: one persistent kernel per call (routing, gate/up, SiLU-GLU,
  * down and combine fused; intermediates stay on chip or in L2). Launched with programmatic
  * dependent launch so that consecutive layer calls overlap their start-up.
- *   x (device) bf16 [T x H]; w_router (device) fp32 [E x H]; bias (device) fp32 [E] or NULL;
- *   packed (device) one layer in moe_pack_layer form with the same E, H, I;
- *   out (device) bf16 [T x H]; idx_out (device) int32 [T x k] or NULL; w_out (device) fp32
+ *   x (device, 16-byte aligned) bf16 [T x H]; w_router (device, 16-byte aligned) fp32 [E x H];
+ *   bias (device) fp32 [E] or NULL; packed (device, 256-byte aligned) one layer in moe_pack_layer form with the same E, H, I;
+ *   out (device, 16-byte aligned) bf16 [T x H]; idx_out (device) int32 [T x k] or NULL; w_out (device) fp32
  *   [T x k] or NULL; workspace (device) of ws_bytes >= moe_workspace_bytes(..., DECODE),
  *   prepared by moe_workspace_init.
  * Limits: H % 64 == 0, I % 64 == 0, 1 <= k <= min(E, 32), E <= 1024.

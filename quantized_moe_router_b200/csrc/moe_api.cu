@@ -68,7 +68,7 @@ moe_status_t forward_common(const uint16_t *x, const float *w_router, const floa
                             size_t ws_bytes, int mode) {
     if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
     if (!x || !w_router || !out || !ws || !packed_ok(packed)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ws, 256) || !aligned(out, 4)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ws, 256) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
     if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
     if ((idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4))) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_workspace_bytes(T, H, I, E, k, mode)) return MOE_ERR_INVALID_ARG;

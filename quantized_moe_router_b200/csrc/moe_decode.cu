@@ -6,21 +6,31 @@
 // overlap (the next expert's tiles are in flight while the current one computes), designed
 // for sm_100a:
 //   * one CTA per SM, 8 consumer warps + 1 producer warp;
-//   * phase R: each CTA computes the fp32 router logits of E/nCTA experts, zeroes its share of
-//     the fp32 accumulators and the per-group sums of x, then a bounded grid barrier;
-//   * every CTA reads all logits from L2 and runs the same warp top-k + softmax, so all CTAs
-//     agree on the selected experts without a second exchange;
-//   * phase X: the selected experts' packed tiles are split into gate/up jobs (8 intermediate
-//     rows x all of H) and down jobs (16 output rows x all of I), statically balanced over CTAs
-//     by bytes; the producer streams each job's tiles with 1-D bulk copies (no multicast) into
-//     a 6-stage ring guarded by mbarriers, and each consumer warp multiplies one tile per stage
-//     with mma.sync on bf16 operands made from the 4-bit codes by one LOP3 per register (exact
-//     integers 128+q), applying the group's scale and zero to the fp32 partial sums;
-//   * gate/up jobs finish with SiLU-GLU and write h (split into bf16 hi + lo, exact to 2^-17)
-//     and its group sums; a second bounded grid barrier makes h visible; down jobs add
-//     w_i * y into an fp32 accumulator with red.add; the last CTA to finish converts it to
-//     bf16. The down tiles are already streaming while the barrier is pending.
-#include <cstdio>
+//   * prologue, before the programmatic-dependent-launch wait so that it overlaps the previous
+//     layer: barrier set-up, this CTA's router rows copied to shared memory, the packed layer's
+//     expert table read (both are weights, never produced by the previous launch);
+//   * phase R: x is copied to shared memory, each CTA computes the fp32 router logits of its
+//     E/nCTA experts, zeroes its share of the fp32 accumulators and the per-group sums of x,
+//     then a bounded grid barrier;
+//   * every CTA reads all logits from L2 and runs the same CTA-wide top-k + softmax (each warp
+//     selects within a slice of the experts, then every candidate's rank is counted in
+//     parallel), so all CTAs agree on the selected experts without a second exchange;
+//   * phase X: the selected experts' packed tiles form two job sequences, gate/up jobs
+//     (8 intermediate rows x all of H) and down jobs (16 output rows x all of I). Each CTA gets
+//     a contiguous range of each, cut so that every CTA streams the same number of bytes, so
+//     its data is a few long contiguous regions. The producer streams them in 24 KB bulk
+//     copies (on B200 one SM completes roughly one bulk copy per ~250 ns whatever its size,
+//     so copies must be large to reach HBM bandwidth) into a 4-stage ring. Tiles go
+//     round-robin to the 8 consumer warps, which multiply them with mma.sync on bf16
+//     operands made from the codes by one LOP3 per register (exact integers 128+q) and apply
+//     the group's scale and zero to fp32 partial sums;
+//   * gate/up partial sums are combined without CTA barriers: each warp flushes its partial of
+//     a job into a shared-memory slot and the last of the 8 warps to flush applies SiLU-GLU and
+//     writes h (bf16 hi + lo, exact to 2^-17) and its group sums;
+//   * a second bounded grid barrier makes h visible; each CTA loads h into shared memory; down
+//     jobs add w_i * y into an fp32 accumulator with red.add; the last CTA to finish converts
+//     it to bf16. The down tiles stream in while the barrier is pending.
+// The kernel is instantiated for 1, 2 and 4 MMA n-tiles (up to 8, 16 and 32 tokens per expert).
 #include "moe_internal.cuh"
 #include "moe_topk.cuh"
 
@@ -29,10 +39,13 @@ namespace {
 
 constexpr int kCW = 8;                      // consumer warps
 constexpr int kThreads = (kCW + 1) * 32;    // + one producer warp
-constexpr int kStageTiles = kCW;            // one tile per consumer warp per stage
-constexpr int kStageBytes = kStageTiles * tile_bytes(8);
-constexpr int kStages = 6;
+constexpr int kStageBytes = 24576;          // bytes per bulk copy / pipeline stage
+constexpr int kStages = 4;
+constexpr int kActBytes = 49152;            // smem for x (routing + gate/up), then h (down)
+constexpr int kRedBytes = 32768;            // gate/up partial-sum slots (top-k scratch before)
+constexpr int kHStageBytes = 16384;         // finished h of this CTA's gate/up jobs, written out in one burst
 constexpr int kMaxP = 256;                  // decode limit on T*k
+constexpr int kSlices = 8;                  // expert slices of the first top-k stage
 
 struct DecodeArgs {
     const uint16_t *x;
@@ -53,82 +66,135 @@ struct DecodeArgs {
 struct __align__(16) DecodeSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    int U, nGUc, nDc, d_start, d_stride, abort, is_last, uniform_bits;
+    uint64_t wbar, xbar;
+    int U, abort, is_last, nGUc;
+    int g0, g1, d0, d1;                 // this CTA's gate/up and down job ranges
+    int slot_cnt[8];
+    int slot_seq[8];
+    uint32_t eoff[kMaxE];               // packed offset / 256 of every expert
+    uint8_t ebits[kMaxE];               // code width of every expert
     uint32_t selmask[kMaxE / 32];
     int wordpre[kMaxE / 32];
-    int ue[kMaxP];
     int ubits[kMaxP];
-    unsigned long long uoff[kMaxP];
+    uint32_t uoff[kMaxP];
     int cnt[kMaxP];
     int pfirst[kMaxP + 1];
     int cursor[kMaxP];
+    uint32_t cgu[kMaxP + 1];            // 64-byte units of all gate/up jobs of expert slots < u
+    uint32_t cd[kMaxP + 1];             // 64-byte units of all down jobs of expert slots < u
     int ptok[kMaxP];
     int ppair[kMaxP];
     float pw[kMaxP];
     int sel_idx[kMaxP];
+    uint32_t sel_key[kMaxP];
     float sel_w[kMaxP];
 };
 
-__host__ __device__ inline int nt_max(int T) { return (T + 7) / 8; }
-
 size_t decode_smem_bytes(int T, int H) {
     size_t o = align_up(sizeof(DecodeSmem), 128);
-    o += (size_t)kStages * kStageBytes;
+    o += (size_t)kStages * kStageBytes + kActBytes + kRedBytes + kHStageBytes;
     o += align_up((size_t)T * (H / kGroup) * 4, 16);
-    o += (size_t)2 * kCW * nt_max(T) * 32 * 4 * 4;
     return o;
 }
 
+__host__ __device__ inline bool x_in_smem(int T, int H) { return (size_t)T * H * 2 <= (size_t)kActBytes; }
+__host__ __device__ inline size_t h_smem_bytes(int P, int I) {
+    return (size_t)2 * P * I * 2 + align_up((size_t)P * (I / kGroup) * 4, 16);
+}
+
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// CTA-scope acquire / release on shared-memory words (hand-off of partial sums between warps)
+__device__ __forceinline__ int ld_acquire_cta(const int *p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta(int *p, int v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_add_acq_rel_cta(int *p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
     const int w = e >> 5;
     return S.wordpre[w] + __popc(S.selmask[w] & ((1u << (e & 31)) - 1u));
 }
 
-struct Job {
+// ------------------------------------------------------------------------------ job layout
+// A run of consecutive jobs of one expert and one phase: contiguous in the packed layer.
+struct Region {
     const uint8_t *src;
-    int ntiles;  // tiles in this job
-    int tb;      // bytes per tile
-    int bits;
-    int u;       // unique-expert slot
-    int rb;      // row block
-    bool gu;
+    int tiles, tb, bits, u, rb0, job0, tpj;   // job0: CTA-local index of the first job
 };
 
-__device__ __forceinline__ Job job_at(const DecodeSmem &S, const DecodeArgs &a, int n, int c, int nC) {
-    Job j;
+__device__ __forceinline__ Region region_at(const DecodeSmem &S, const DecodeArgs &a, bool gu, int j) {
+    Region r;
     const int G = a.H / kGroup, GI = a.I / kGroup;
-    if (n < S.nGUc) {
-        const int gj = c + n * nC;
-        const int rbg = a.I / 8;
-        j.u = gj / rbg;
-        j.rb = gj % rbg;
-        j.gu = true;
-        j.ntiles = G;
-    } else {
-        const int d = S.d_start + (n - S.nGUc) * S.d_stride;
-        const int rbd = a.H / 16;
-        j.u = d / rbd;
-        j.rb = d % rbd;
-        j.gu = false;
-        j.ntiles = GI;
-    }
-    j.bits = S.ubits[j.u];
-    j.tb = tile_bytes(j.bits);
-    const uint8_t *base = a.packed + S.uoff[j.u];
-    if (j.gu)
-        j.src = base + (size_t)j.rb * G * j.tb;
-    else
-        j.src = base + gu_tiles(a.H, a.I) * j.tb + (size_t)j.rb * GI * j.tb;
-    return j;
+    const int per = gu ? a.I / 8 : a.H / 16;    // jobs per expert
+    const int end = gu ? S.g1 : S.d1;
+    r.u = j / per;
+    r.rb0 = j % per;
+    const int jend = min(end, (r.u + 1) * per);
+    r.tpj = gu ? G : GI;
+    r.tiles = (jend - j) * r.tpj;
+    r.bits = S.ubits[r.u];
+    r.tb = tile_bytes(r.bits);
+    r.job0 = gu ? (j - S.g0) : (S.nGUc + j - S.d0);
+    const uint8_t *base = a.packed + (size_t)S.uoff[r.u] * 256;
+    r.src = gu ? base + (size_t)r.rb0 * G * r.tb : base + gu_tiles(a.H, a.I) * r.tb + (size_t)r.rb0 * GI * r.tb;
+    return r;
+}
+__device__ __forceinline__ int region_chunks(const Region &r) {
+    const int cap = kStageBytes / r.tb;
+    return (r.tiles + cap - 1) / cap;
+}
+// tiles [c0, c0 + m) of chunk i of a region (balanced split)
+__device__ __forceinline__ void chunk_range(const Region &r, int n, int i, int &c0, int &m) {
+    const int base = r.tiles / n, rem = r.tiles % n;
+    m = base + (i < rem ? 1 : 0);
+    c0 = i * base + (i < rem ? i : rem);
 }
 
-// One tile (one quantisation group) of a job for every n-tile of the job's tokens.
-template <int BITS>
-__device__ __forceinline__ void consume_tile(const DecodeArgs &a, const DecodeSmem &S,
-                                             const uint8_t *tile, const Job &jb, int kg,
-                                             const float *Xs, int lane, float (&acc)[4][4]) {
+// First job (of the gate/up or down sequence) whose first 64-byte unit is at or after `pos`;
+// cum[u] = units of the jobs of expert slots < u, `per` jobs per expert.
+__device__ __forceinline__ int job_at_unit(const uint32_t *cum, int U, int per, uint32_t pos) {
+    if (pos == 0) return 0;
+    if (pos >= cum[U]) return U * per;
+    int lo = 0, hi = U;                 // largest u with cum[u] <= pos
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= pos) lo = mid; else hi = mid;
+    }
+    const uint32_t jb = (cum[lo + 1] - cum[lo]) / per;   // units per job of expert lo
+    return lo * per + (int)((pos - cum[lo] + jb - 1) / jb);
+}
+__device__ __forceinline__ uint32_t job_start_unit(const uint32_t *cum, int U, int per, int j) {
+    if (j >= U * per) return cum[U];
+    const int u = j / per;
+    return cum[u] + (cum[u + 1] - cum[u]) / per * (uint32_t)(j % per);
+}
+
+// ------------------------------------------------------------------------------ tile math
+// Operand sources of the current job for this lane: per n-tile, the row of x (gate/up) or of
+// h hi / lo (down) that the lane's B column reads, and the rows of group sums of its two
+// accumulator columns (null where the column has no token).
+template <int NT>
+struct JobCtx {
+    const uint16_t *b[NT];
+    const uint16_t *b2[NT];
+    const float *xs0[NT];
+    const float *xs1[NT];
+};
+
+template <int BITS, int NT, bool GU>
+__device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const JobCtx<NT> &jc, int lane,
+                                             float (&acc)[NT][4], float keep = 1.f) {
     const int g = lane >> 2, t = lane & 3;
     const uint4 lo = *reinterpret_cast<const uint4 *>(tile + 16 * lane);
     uint4 hi8 = make_uint4(0, 0, 0, 0);
@@ -136,137 +202,269 @@ __device__ __forceinline__ void consume_tile(const DecodeArgs &a, const DecodeSm
     if (BITS == 8) hi8 = *reinterpret_cast<const uint4 *>(tile + kLoBytes + 16 * lane);
     if (BITS == 6) hi6 = *reinterpret_cast<const uint2 *>(tile + kLoBytes + 8 * lane);
     const uint2 sz = *reinterpret_cast<const uint2 *>(tile + kLoBytes + hi_bytes(BITS) + 8 * g);
-    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
-    const int pf = S.pfirst[jb.u];
-    const int nu = S.pfirst[jb.u + 1] - pf;
-    const int G = a.H / kGroup, GI = a.I / kGroup;
-    const int ntn = (nu + 7) >> 3;
+    // keep = 0 turns the tile into a no-op (scales zeroed), so that pairs of tiles run without a
+    // branch and their MMA chains interleave
+    const float sA = keep * half_lo(sz.x), zA = half_hi(sz.x), sB = keep * half_lo(sz.y), zB = half_hi(sz.y);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        if (nt >= ntn) break;
-        const int q = nt * 8 + g, q0 = nt * 8 + 2 * t, q1 = q0 + 1;
+    for (int nt = 0; nt < NT; ++nt) {
         uint32_t b[8] = {0, 0, 0, 0, 0, 0, 0, 0}, b2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        float X0 = 0.f, X1 = 0.f;
-        if (jb.gu) {
-            if (q < nu) {
-                const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + (size_t)S.ptok[pf + q] * a.H +
-                                                                  kg * kGroup + 16 * t);
-                const uint4 xa = __ldg(xp), xb = __ldg(xp + 1);
-                b[0] = xa.x; b[1] = xa.y; b[2] = xa.z; b[3] = xa.w;
-                b[4] = xb.x; b[5] = xb.y; b[6] = xb.z; b[7] = xb.w;
+        if (jc.b[nt]) {
+            const uint16_t *p = jc.b[nt] + kg * kGroup + 16 * t;
+            const uint4 v0 = *reinterpret_cast<const uint4 *>(p), v1 = *reinterpret_cast<const uint4 *>(p + 8);
+            b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
+            b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
+            if (!GU) {
+                const uint16_t *p2 = jc.b2[nt] + kg * kGroup + 16 * t;
+                const uint4 w0 = *reinterpret_cast<const uint4 *>(p2), w1 = *reinterpret_cast<const uint4 *>(p2 + 8);
+                b2[0] = w0.x; b2[1] = w0.y; b2[2] = w0.z; b2[3] = w0.w;
+                b2[4] = w1.x; b2[5] = w1.y; b2[6] = w1.z; b2[7] = w1.w;
             }
-            if (q0 < nu) X0 = Xs[S.ptok[pf + q0] * G + kg];
-            if (q1 < nu) X1 = Xs[S.ptok[pf + q1] * G + kg];
-            tile_group_mma<BITS>(lo, hi8, hi6, b, nullptr, sA, zA, sB, zB, X0, X1, acc[nt]);
-        } else {
-            if (q < nu) {
-                const size_t off = (size_t)S.ppair[pf + q] * a.I + kg * kGroup + 16 * t;
-                const uint4 *hp = reinterpret_cast<const uint4 *>(a.h_hi + off);
-                const uint4 *lp = reinterpret_cast<const uint4 *>(a.h_lo + off);
-                const uint4 ha = __ldcg(hp), hb = __ldcg(hp + 1), la = __ldcg(lp), lb = __ldcg(lp + 1);
-                b[0] = ha.x; b[1] = ha.y; b[2] = ha.z; b[3] = ha.w;
-                b[4] = hb.x; b[5] = hb.y; b[6] = hb.z; b[7] = hb.w;
-                b2[0] = la.x; b2[1] = la.y; b2[2] = la.z; b2[3] = la.w;
-                b2[4] = lb.x; b2[5] = lb.y; b2[6] = lb.z; b2[7] = lb.w;
-            }
-            if (q0 < nu) X0 = __ldcg(a.hsum + (size_t)S.ppair[pf + q0] * GI + kg);
-            if (q1 < nu) X1 = __ldcg(a.hsum + (size_t)S.ppair[pf + q1] * GI + kg);
-            tile_group_mma<BITS>(lo, hi8, hi6, b, b2, sA, zA, sB, zB, X0, X1, acc[nt]);
         }
+        const float X0 = jc.xs0[nt] ? jc.xs0[nt][kg] : 0.f;
+        const float X1 = jc.xs1[nt] ? jc.xs1[nt][kg] : 0.f;
+        tile_group_mma<BITS>(lo, hi8, hi6, b, GU ? nullptr : b2, sA, zA, sB, zB, X0, X1, acc[nt]);
     }
 }
 
-__device__ void job_epilogue(const DecodeArgs &a, const DecodeSmem &S, const Job &jb, float *red,
-                             int NTM, int warp, int lane, float (&acc)[4][4]) {
-    const int pf = S.pfirst[jb.u];
-    const int nu = S.pfirst[jb.u + 1] - pf;
-    const int ntn = (nu + 7) >> 3;
-    for (int nt = 0; nt < ntn; ++nt)
-        *reinterpret_cast<float4 *>(red + ((warp * NTM + nt) * 32 + lane) * 4) =
-            make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-    consumer_sync();
-    if (warp != 0) return;
+// SiLU-GLU of a finished gate/up job from the 8 warps' partials in slot `red`. With `stage`
+// set, h (bf16 hi + lo of the lane's two columns) goes to shared memory and is written out
+// after the gate/up phase (a warp with global writes in flight makes every later CTA-scope
+// fence wait for them); otherwise h and its group sums go straight to global memory.
+template <int NT>
+__device__ void gu_finalize(const DecodeArgs &a, const DecodeSmem &S, int u, int rb, const float *red, int lane,
+                            uint2 *stage) {
+    const int pf = S.pfirst[u];
+    const int nu = S.pfirst[u + 1] - pf;
     const int g = lane >> 2, t = lane & 3;
     const int GI = a.I / kGroup;
-    for (int nt = 0; nt < ntn; ++nt) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
         float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
         for (int w = 0; w < kCW; ++w) {
-            const float4 p = *reinterpret_cast<const float4 *>(red + ((w * NTM + nt) * 32 + lane) * 4);
+            const float4 p = *reinterpret_cast<const float4 *>(red + ((w * NT + nt) * 32 + lane) * 4);
             v[0] += p.x; v[1] += p.y; v[2] += p.z; v[3] += p.w;
         }
+        uint32_t his = 0, los = 0;
+#pragma unroll
         for (int col = 0; col < 2; ++col) {
             const int q = nt * 8 + 2 * t + col;
             const bool valid = q < nu;
-            if (jb.gu) {
-                const float gate = v[col], up = v[2 + col];
-                const float h = gate / (1.f + expf(-gate)) * up;
-                const __nv_bfloat16 hi = __float2bfloat16_rn(h);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
-                float part = 0.f;
-                int pair = 0;
-                if (valid) {
-                    pair = S.ppair[pf + q];
-                    const size_t o = (size_t)pair * a.I + jb.rb * 8 + g;
-                    a.h_hi[o] = __bfloat16_as_ushort(hi);
-                    a.h_lo[o] = __bfloat16_as_ushort(lo);
-                    part = __bfloat162float(hi) + __bfloat162float(lo);
-                }
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                part += __shfl_xor_sync(0xffffffffu, part, 8);
-                part += __shfl_xor_sync(0xffffffffu, part, 16);
-                if (g == 0 && valid) red_add_f32(a.hsum + (size_t)pair * GI + (jb.rb >> 3), part);
-            } else if (valid) {
-                const int tok = S.ptok[pf + q];
-                const float wgt = S.pw[pf + q];
-                const int row = jb.rb * 16 + g;
-                red_add_f32(a.out_acc + (size_t)tok * a.H + row, wgt * v[col]);
-                red_add_f32(a.out_acc + (size_t)tok * a.H + row + 8, wgt * v[2 + col]);
+            const float gate = v[col], up = v[2 + col];
+            const float h = gate / (1.f + expf(-gate)) * up;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+            his |= (uint32_t)__bfloat16_as_ushort(hi) << (16 * col);
+            los |= (uint32_t)__bfloat16_as_ushort(lo) << (16 * col);
+            if (stage) continue;
+            float part = 0.f;
+            int pair = 0;
+            if (valid) {
+                pair = S.ppair[pf + q];
+                const size_t o = (size_t)pair * a.I + rb * 8 + g;
+                a.h_hi[o] = __bfloat16_as_ushort(hi);
+                a.h_lo[o] = __bfloat16_as_ushort(lo);
+                part = __bfloat162float(hi) + __bfloat162float(lo);
             }
+            part += __shfl_xor_sync(0xffffffffu, part, 4);
+            part += __shfl_xor_sync(0xffffffffu, part, 8);
+            part += __shfl_xor_sync(0xffffffffu, part, 16);
+            if (g == 0 && valid) red_add_f32(a.hsum + (size_t)pair * GI + (rb >> 3), part);
+        }
+        if (stage) stage[nt * 32 + lane] = make_uint2(his, los);
+    }
+}
+
+// Writes the staged h of the CTA's gate/up jobs [0, njobs) (global job index g0 + f) and adds
+// their group sums; run by all 256 consumer threads.
+template <int NT>
+__device__ void write_staged_h(const DecodeArgs &a, const DecodeSmem &S, const uint2 *stage, int njobs) {
+    const int GI = a.I / kGroup, pg = a.I / 8;
+    // one thread per (job, n-tile, t, col): the 8 rows g of that column
+    for (int i = threadIdx.x; i < njobs * NT * 8; i += kCW * 32) {
+        const int f = i / (NT * 8), nt = (i / 8) % NT, t = (i >> 1) & 3, col = i & 1;
+        const int gj = S.g0 + f, u = gj / pg, rb = gj % pg;
+        const int pf = S.pfirst[u], nu = S.pfirst[u + 1] - pf;
+        const int q = nt * 8 + 2 * t + col;
+        if (q >= nu) continue;
+        const int pair = S.ppair[pf + q];
+        float part = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const uint2 v = stage[(f * NT + nt) * 32 + g * 4 + t];
+            const uint16_t hi = (uint16_t)(v.x >> (16 * col)), lo = (uint16_t)(v.y >> (16 * col));
+            const size_t o = (size_t)pair * a.I + rb * 8 + g;
+            a.h_hi[o] = hi;
+            a.h_lo[o] = lo;
+            part += bf16_bits_to_float(hi) + bf16_bits_to_float(lo);
+        }
+        red_add_f32(a.hsum + (size_t)pair * GI + (rb >> 3), part);
+    }
+}
+
+// ------------------------------------------------------------------------------ top-k
+// Every CTA selects the top-k of each token from the logits in L2: stage 1, each (token,
+// slice) task keeps the k best of its E/8 experts (warp arg-max rounds); stage 2, each
+// candidate's rank among the token's 8k candidates is counted in parallel (larger logit first,
+// equal logits -> lower index); stage 3, softmax over the k selected.
+__device__ void cta_topk(const DecodeArgs &a, DecodeSmem &S, uint32_t *cand_key, int *cand_idx, int warp, int lane) {
+    const int T = a.T, E = a.E, K = a.k;
+    const int NC = kSlices * K;                 // candidates per token
+    const int slice = (E + kSlices - 1) / kSlices;
+    for (int task = warp; task < T * kSlices; task += kCW + 1) {
+        const int t = task / kSlices, sl = task % kSlices;
+        const int e0 = sl * slice, e1 = min(E, e0 + slice);
+        uint32_t key[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int e = e0 + lane + 32 * m;
+            uint32_t kk = 0;
+            if (e < e1) {
+                float v = __ldcg(a.logits + (size_t)t * E + e);
+                if (v != v) v = -INFINITY;
+                kk = order_key(v);
+            }
+            key[m] = kk;
+        }
+        for (int r = 0; r < K; ++r) {
+            uint32_t bk = 0;
+            int bm = 0;
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                if (key[m] > bk) { bk = key[m]; bm = m; }
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t cidx = (bk == mx && mx != 0) ? (uint32_t)(e0 + lane + 32 * bm) : 0xFFFFFFFFu;
+            const uint32_t win = __reduce_min_sync(0xffffffffu, cidx);
+            if (lane == 0) {
+                cand_key[t * NC + sl * K + r] = mx;      // 0: slice exhausted
+                cand_idx[t * NC + sl * K + r] = (int)win;
+            }
+            if (mx != 0 && win == (uint32_t)(e0 + lane + 32 * bm)) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    if (m == bm) key[m] = 0;
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * NC; i += kThreads) {
+        const int t = i / NC;
+        const uint32_t mk = cand_key[i];
+        if (mk == 0) continue;
+        const int mi = cand_idx[i];
+        int rank = 0;
+        for (int j = 0; j < NC; ++j) {
+            const uint32_t ok = cand_key[t * NC + j];
+            const int oi = cand_idx[t * NC + j];
+            rank += (ok > mk || (ok == mk && oi < mi)) ? 1 : 0;
+        }
+        if (rank < K) {
+            S.sel_idx[t * K + rank] = mi;
+            S.sel_key[t * K + rank] = mk;
+        }
+    }
+    __syncthreads();
+    for (int t = warp; t < T; t += kCW + 1) {
+        const float v = (lane < K) ? key_value(S.sel_key[t * K + lane]) : -INFINITY;
+        const float v0 = __shfl_sync(0xffffffffu, v, 0);
+        float ex = 0.f;
+        if (lane < K) ex = (v0 == -INFINITY) ? 1.f : expf(v - v0);
+        float s = ex;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane < K) {
+            const float w = ex / s;
+            S.sel_w[t * K + lane] = w;
+            if (blockIdx.x == 0 && a.idx_out) a.idx_out[t * K + lane] = S.sel_idx[t * K + lane];
+            if (blockIdx.x == 0 && a.w_out) a.w_out[t * K + lane] = w;
         }
     }
 }
 
+// ------------------------------------------------------------------------------ kernel
+template <int NT>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t dyn[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(dyn);
     uint8_t *stages = dyn + align_up(sizeof(DecodeSmem), 128);
-    float *Xs = reinterpret_cast<float *>(stages + (size_t)kStages * kStageBytes);
+    uint8_t *act = stages + (size_t)kStages * kStageBytes;
+    float *red = reinterpret_cast<float *>(act + kActBytes);
+    uint2 *hstage = reinterpret_cast<uint2 *>(act + kActBytes + kRedBytes);
+    float *Xs = reinterpret_cast<float *>(act + kActBytes + kRedBytes + kHStageBytes);
     const int T = a.T, H = a.H, I = a.I, E = a.E, K = a.k, P = T * K;
     const int G = H / kGroup, GI = I / kGroup;
-    float *redbuf = Xs + align_up((size_t)T * G, 4);
-    const int NTM = nt_max(T);
+    constexpr int NSLOT = 8 / NT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nC = gridDim.x, c = blockIdx.x;
     uint32_t *status = &a.ctl->status;
+    const bool xs_on = x_in_smem(T, H);
+    const bool hs_on = h_smem_bytes(P, I) <= (size_t)kActBytes;
+    const uint16_t *xsm = xs_on ? reinterpret_cast<const uint16_t *>(act) : nullptr;
+    const int ne = (E > c) ? (E - c + nC - 1) / nC : 0;   // router rows of this CTA: c, c+nC, ...
+    const bool wr_on = (size_t)ne * H * 4 <= (size_t)kStages * kStageBytes;
+    const float *wsm = reinterpret_cast<const float *>(stages);
 
+    // ---------------------------------------------------------------- prologue
+    // Reads only the router weights and the packed layer (weights), so it may overlap the
+    // previous launch in the stream.
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&S.full[s]), 1);
             mbar_init(smem_u32(&S.empty[s]), kCW);
         }
+        mbar_init(smem_u32(&S.wbar), 1);
+        mbar_init(smem_u32(&S.xbar), 1);
         fence_barrier_init();
         S.abort = 0;
         S.is_last = 0;
+        if (wr_on && ne > 0) {
+            const uint32_t rowb = (uint32_t)H * 4;
+            mbar_expect_tx(smem_u32(&S.wbar), rowb * ne);
+            for (int i = 0; i < ne; ++i)
+                bulk_g2s(smem_u32(stages + (size_t)i * rowb), a.wr + (size_t)(c + i * nC) * H, rowb, smem_u32(&S.wbar));
+        }
+    }
+    if (!wr_on)
+        for (int i = threadIdx.x; i < ne; i += kThreads) prefetch_l2(a.wr + (size_t)(c + i * nC) * H, (uint32_t)H * 4);
+    {
+        const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
+        for (int e = threadIdx.x; e < E; e += kThreads) {
+            const PackedExpert v = pe[e];
+            S.eoff[e] = (uint32_t)(v.offset >> 8);
+            S.ebits[e] = (uint8_t)v.bits;
+        }
     }
     for (int i = threadIdx.x; i < kMaxE / 32; i += kThreads) S.selmask[i] = 0;
+    if (threadIdx.x < 8) {
+        S.slot_cnt[threadIdx.x] = 0;
+        S.slot_seq[threadIdx.x] = 0;
+    }
     __syncthreads();
-    // Everything below reads data that the previous launch in the stream may produce.
+    // Everything below may read data that the previous launch in the stream produces.
     grid_dep_wait();
 
     // ---------------------------------------------------------------- phase R
+    if (xs_on && threadIdx.x == 0) {
+        const uint32_t bytes = (uint32_t)(T * H * 2);
+        mbar_expect_tx(smem_u32(&S.xbar), bytes);
+        bulk_g2s(smem_u32(act), a.x, bytes, smem_u32(&S.xbar));
+    }
     const int gtid = c * kThreads + threadIdx.x, gthreads = nC * kThreads;
     for (int i = gtid; i < T * H; i += gthreads) a.out_acc[i] = 0.f;
     for (int i = gtid; i < P * GI; i += gthreads) a.hsum[i] = 0.f;
-    const int ne = (E > c) ? (E - c + nC - 1) / nC : 0;
+    if (xs_on && !mbar_wait(smem_u32(&S.xbar), 0, a.wait_ns, status)) S.abort = 1;
+    if (wr_on && ne > 0 && !mbar_wait(smem_u32(&S.wbar), 0, a.wait_ns, status)) S.abort = 1;
+    const uint16_t *xr = xs_on ? xsm : a.x;
     for (int q = warp; q < ne * T; q += kCW + 1) {
-        const int e = c + (q / T) * nC, t = q % T;
-        const float *wrow = a.wr + (size_t)e * H;
-        const uint16_t *xrow = a.x + (size_t)t * H;
+        const int i = q / T, t = q % T;
+        const int e = c + i * nC;
+        const float *wrow = wr_on ? wsm + (size_t)i * H : a.wr + (size_t)e * H;
+        const uint16_t *xrow = xr + (size_t)t * H;
         float acc = 0.f;
         for (int h = lane * 8; h < H; h += 256) {
-            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(wrow + h));
-            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(wrow + h + 4));
-            const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(xrow + h));
+            const float4 w0 = *reinterpret_cast<const float4 *>(wrow + h);
+            const float4 w1 = *reinterpret_cast<const float4 *>(wrow + h + 4);
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + h);
             acc += w0.x * __uint_as_float(xv.x << 16) + w0.y * __uint_as_float(xv.x & 0xFFFF0000u);
             acc += w0.z * __uint_as_float(xv.y << 16) + w0.w * __uint_as_float(xv.y & 0xFFFF0000u);
             acc += w1.x * __uint_as_float(xv.z << 16) + w1.y * __uint_as_float(xv.z & 0xFFFF0000u);
@@ -276,12 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) a.logits[(size_t)t * E + e] = acc + (a.bias ? a.bias[e] : 0.f);
     }
-    for (int i = threadIdx.x; i < T * G; i += kThreads) {
-        const int t = i / G, gq = i % G;
-        const uint16_t *xp = a.x + (size_t)t * H + gq * kGroup;
-        float s = 0.f;
-        for (int j = 0; j < kGroup; ++j) s += bf16_bits_to_float(xp[j]);
-        Xs[i] = s;
+    // per-token sums of x over each group (one warp per group, two values per lane)
+    for (int i = warp; i < T * G; i += kCW + 1) {
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(xr + (size_t)i * kGroup + 2 * lane);
+        float s = __uint_as_float(v << 16) + __uint_as_float(v & 0xFFFF0000u);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) Xs[i] = s;
     }
     __syncthreads();
     if (threadIdx.x == 0 && !grid_barrier(&a.ctl->bar, nC, c == 0, a.wait_ns, status)) S.abort = 1;
@@ -289,146 +488,148 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     grid_dep_launch();
 
     // ---------------------------------------------------------------- routing
-    if (!S.abort) {
-        for (int t = warp; t < T; t += kCW + 1) {
-            int idx;
-            float w;
-            warp_topk_softmax(a.logits + (size_t)t * E, true, E, K, lane, idx, w);
-            if (lane < K) {
-                S.sel_idx[t * K + lane] = idx;
-                S.sel_w[t * K + lane] = w;
-                if (c == 0 && a.idx_out) a.idx_out[t * K + lane] = idx;
-                if (c == 0 && a.w_out) a.w_out[t * K + lane] = w;
-            }
-        }
-    }
-    __syncthreads();
     const bool aborted = S.abort != 0;
-    if (!aborted)
-        for (int p = threadIdx.x; p < P; p += kThreads)
+    if (!aborted) {
+        uint32_t *cand_key = reinterpret_cast<uint32_t *>(red);
+        int *cand_idx = reinterpret_cast<int *>(red) + kSlices * kMaxP;
+        cta_topk(a, S, cand_key, cand_idx, warp, lane);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // unique experts (ascending id), their pair lists (ascending token) and the job ranges
+        for (int p = lane; p < (aborted ? 0 : P); p += 32)
             atomicOr(&S.selmask[S.sel_idx[p] >> 5], 1u << (S.sel_idx[p] & 31));
-    __syncthreads();
-    if (warp == 0) {
-        const int words = (E + 31) / 32;
-        const int n = (lane < words) ? __popc(S.selmask[lane]) : 0;
-        int incl = n;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o;
-        }
-        S.wordpre[lane] = incl - n;
-        if (lane == 31) S.U = incl;
-    }
-    __syncthreads();
-    const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-        if ((S.selmask[e >> 5] >> (e & 31)) & 1u) {
-            const int s = slot_of(S, e);
-            S.ue[s] = e;
-            S.ubits[s] = pe[e].bits;
-            S.uoff[s] = pe[e].offset;
-            S.cnt[s] = 0;
-        }
-    }
-    __syncthreads();
-    for (int p = threadIdx.x; p < (aborted ? 0 : P); p += kThreads) atomicAdd(&S.cnt[slot_of(S, S.sel_idx[p])], 1);
-    __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 0; base < S.U; base += 32) {
-            const int s = base + lane;
-            const int n = (s < S.U) ? S.cnt[s] : 0;
+        __syncwarp();
+        {
+            const int words = (E + 31) / 32;
+            const int n = (lane < words) ? __popc(S.selmask[lane]) : 0;
             int incl = n;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int o = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += o;
             }
-            if (s < S.U) {
-                S.pfirst[s] = carry + incl - n;
-                S.cursor[s] = carry + incl - n;
+            S.wordpre[lane] = incl - n;
+            if (lane == 31) S.U = incl;
+        }
+        __syncwarp();
+        const int U = S.U;
+        for (int u = lane; u < U; u += 32) S.cnt[u] = 0;
+        __syncwarp();
+        for (int p = lane; p < (aborted ? 0 : P); p += 32) {
+            const int e = S.sel_idx[p];
+            const int u = slot_of(S, e);
+            S.ubits[u] = S.ebits[e];
+            S.uoff[u] = S.eoff[e];
+            atomicAdd(&S.cnt[u], 1);
+        }
+        __syncwarp();
+        int carry = 0;
+        uint32_t cg = 0, cdd = 0;
+        for (int base = 0; base < U; base += 32) {
+            const int u = base + lane;
+            const int n = (u < U) ? S.cnt[u] : 0;
+            const uint32_t tu = (u < U) ? (uint32_t)tile_bytes(S.ubits[u]) / 64 : 0;   // 64-byte units per tile
+            const uint32_t bg = tu * (uint32_t)(I / 8) * G, bd = tu * (uint32_t)(H / 16) * GI;
+            int incl = n;
+            uint32_t ig = bg, id = bd;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off);
+                const uint32_t og = __shfl_up_sync(0xffffffffu, ig, off);
+                const uint32_t od = __shfl_up_sync(0xffffffffu, id, off);
+                if (lane >= off) {
+                    incl += o;
+                    ig += og;
+                    id += od;
+                }
+            }
+            if (u < U) {
+                S.pfirst[u] = carry + incl - n;
+                S.cursor[u] = carry + incl - n;
+                S.cgu[u] = cg + ig - bg;
+                S.cd[u] = cdd + id - bd;
             }
             carry += __shfl_sync(0xffffffffu, incl, 31);
+            cg += __shfl_sync(0xffffffffu, ig, 31);
+            cdd += __shfl_sync(0xffffffffu, id, 31);
         }
-        if (lane == 0) S.pfirst[S.U] = carry;
+        if (lane == 0) {
+            S.pfirst[U] = carry;
+            S.cgu[U] = cg;
+            S.cd[U] = cdd;
+        }
         __syncwarp();
         // stable fill: pairs in ascending pair id (token-major) order
         for (int base = 0; base < (aborted ? 0 : P); base += 32) {
             const int p = base + lane;
-            const int s = (p < P) ? slot_of(S, S.sel_idx[p]) : -1 - lane;
-            const uint32_t peers = __match_any_sync(0xffffffffu, s);
+            const int u = (p < P) ? slot_of(S, S.sel_idx[p]) : -1 - lane;
+            const uint32_t peers = __match_any_sync(0xffffffffu, u);
             const int rank = __popc(peers & ((1u << lane) - 1u));
             if (p < P) {
-                const int pos = S.cursor[s] + rank;
+                const int pos = S.cursor[u] + rank;
                 S.ppair[pos] = p;
                 S.ptok[pos] = p / K;
                 S.pw[pos] = S.sel_w[p];
             }
             __syncwarp();
-            if (p < P && rank == 0) S.cursor[s] += __popc(peers);
+            if (p < P && rank == 0) S.cursor[u] += __popc(peers);
             __syncwarp();
         }
-        // job plan
+        // Job ranges: the gate/up sequence is cut at multiples of its bytes / nCTA; the down
+        // sequence is cut so that each CTA's gate/up + down bytes are the layer's bytes / nCTA.
+        // That cut is monotone in the CTA index when every CTA's down share exceeds one gate/up
+        // job (plus rounding); otherwise (tiny layers) the down sequence is cut on its own.
         if (lane == 0) {
-            int U = aborted ? 0 : S.U;
-            int ub = U > 0 ? S.ubits[0] : 4;
-            for (int s = 1; s < U; ++s)
-                if (S.ubits[s] != ub) ub = 0;
-            S.uniform_bits = ub;
-            const long long nGU = (long long)U * (I / 8), nD = (long long)U * (H / 16);
-            S.nGUc = (nGU > c) ? (int)((nGU - c + nC - 1) / nC) : 0;
-            const long long q = nGU / nC, r = nGU % nC;
-            const long long W = nGU * G + nD * GI;  // in tiles (uniform width)
-            bool balanced = ub != 0 && (long long)nC * (q + 1) * G <= W;
-            if (balanced) {
-                const long long d1 = (W - (long long)nC * (q + 1) * G) / ((long long)nC * GI);
-                const long long d0 = (W - (long long)nC * q * G) / ((long long)nC * GI);
-                const long long L = nD - r * d1 - (nC - r) * d0;
-                const long long e0 = L < (nC - r) ? L : (nC - r);
-                const long long L1 = L - e0;
-                if (L < 0 || L1 > r) balanced = false;
-                if (balanced) {
-                    long long cnt, start;
-                    if (c < r) {
-                        cnt = d1 + (c < L1 ? 1 : 0);
-                        start = (long long)c * d1 + (c < L1 ? c : L1);
-                    } else {
-                        cnt = d0 + ((c - r) < e0 ? 1 : 0);
-                        start = r * d1 + L1 + (c - r) * d0 + ((c - r) < e0 ? (c - r) : e0);
-                    }
-                    S.d_start = (int)start;
-                    S.d_stride = 1;
-                    S.nDc = (int)cnt;
-                }
+            const int Uj = aborted ? 0 : U;
+            const int pg = I / 8, pd = H / 16;
+            const uint64_t GUB = S.cgu[Uj], DB = S.cd[Uj], B = GUB + DB;
+            const int g0 = job_at_unit(S.cgu, Uj, pg, (uint32_t)(GUB * c / nC));
+            const int g1 = (c == nC - 1) ? Uj * pg : job_at_unit(S.cgu, Uj, pg, (uint32_t)(GUB * (c + 1) / nC));
+            uint32_t maxjob = 0;
+            for (int u = 0; u < Uj; ++u) maxjob = max(maxjob, (S.cgu[u + 1] - S.cgu[u]) / pg);
+            uint32_t p0, p1;
+            if ((uint64_t)(maxjob + 2) * nC <= DB) {
+                p0 = (uint32_t)(B * c / nC - job_start_unit(S.cgu, Uj, pg, g0));
+                p1 = (uint32_t)(B * (c + 1) / nC - job_start_unit(S.cgu, Uj, pg, g1));
+            } else {
+                p0 = (uint32_t)(DB * c / nC);
+                p1 = (uint32_t)(DB * (c + 1) / nC);
             }
-            if (!balanced) {
-                const int st = (int)(((c - r) % nC + nC) % nC);
-                S.d_start = st;
-                S.d_stride = nC;
-                S.nDc = (nD > st) ? (int)((nD - st + nC - 1) / nC) : 0;
-            }
+            const int d0 = job_at_unit(S.cd, Uj, pd, p0);
+            const int d1 = (c == nC - 1) ? Uj * pd : job_at_unit(S.cd, Uj, pd, p1);
+            S.g0 = g0;
+            S.g1 = g1;
+            S.d0 = d0;
+            S.d1 = d1;
+            S.nGUc = g1 - g0;
         }
     }
     __syncthreads();
 
-    const int njobs = S.nGUc + S.nDc;
     if (warp == kCW) {
         // ------------------------------------------------------------ producer
         if (lane != 0) return;
         uint32_t cc = 0;
-        for (int n = 0; n < njobs; ++n) {
-            const Job jb = job_at(S, a, n, c, nC);
-            for (int c0 = 0; c0 < jb.ntiles; c0 += kStageTiles) {
-                const int s = cc % kStages;
-                const uint32_t use = cc / kStages;
-                if (use > 0 && !mbar_wait(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status)) return;
-                const int nt = min(kStageTiles, jb.ntiles - c0);
-                const uint32_t bytes = (uint32_t)(nt * jb.tb);
-                const uint32_t fb = smem_u32(&S.full[s]);
-                mbar_expect_tx(fb, bytes);
-                bulk_g2s(smem_u32(stages + (size_t)s * kStageBytes), jb.src + (size_t)c0 * jb.tb, bytes, fb);
-                ++cc;
+        for (int ph = 0; ph < 2; ++ph) {
+            const bool gu = ph == 0;
+            const int jend = gu ? S.g1 : S.d1;
+            for (int j = gu ? S.g0 : S.d0; j < jend;) {
+                const Region r = region_at(S, a, gu, j);
+                const int nch = region_chunks(r);
+                for (int ch = 0; ch < nch; ++ch) {
+                    int c0, m;
+                    chunk_range(r, nch, ch, c0, m);
+                    const int s = cc % kStages;
+                    const uint32_t use = cc / kStages;
+                    if (use > 0 && !mbar_wait(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status)) return;
+                    const uint32_t bytes = (uint32_t)(m * r.tb);
+                    const uint32_t fb = smem_u32(&S.full[s]);
+                    mbar_expect_tx(fb, bytes);
+                    bulk_g2s(smem_u32(stages + (size_t)s * kStageBytes), r.src + (size_t)c0 * r.tb, bytes, fb);
+                    ++cc;
+                }
+                j += r.tiles / r.tpj;
             }
         }
         return;
@@ -437,46 +638,216 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     // ---------------------------------------------------------------- consumers
     uint32_t cc = 0;
     bool skip = aborted;
-    for (int n = 0; n < njobs; ++n) {
-        if (n == S.nGUc) {
-            // all h written by every CTA before any down job reads it
+    const uint8_t *hsm = nullptr;
+    const int nGUc = S.nGUc;
+    const bool staged = (size_t)nGUc * NT * 32 * sizeof(uint2) <= (size_t)kHStageBytes;
+    int cur = -1, cur_u = 0, cur_rb = 0;   // job in progress (CTA-local index), -1: none
+    bool cur_any = false;
+    int next_flush = 0;                    // gate/up jobs below this index are flushed by this warp
+    bool gu_done = false;
+    float acc[NT][4], acc2[NT][4];
+    JobCtx<NT> jc;
+    const int g = lane >> 2, t = lane & 3;
+    auto zero_acc = [&]() {
+#pragma unroll
+        for (int i = 0; i < NT; ++i) {
+            acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+            acc2[i][0] = acc2[i][1] = acc2[i][2] = acc2[i][3] = 0.f;
+        }
+    };
+    auto set_ctx = [&](int u, bool gu) {
+        const int pf = S.pfirst[u];
+        const int nu = S.pfirst[u + 1] - pf;
+        const uint16_t *hh = hsm ? reinterpret_cast<const uint16_t *>(hsm) : a.h_hi;
+        const uint16_t *hl = hsm ? reinterpret_cast<const uint16_t *>(hsm) + (size_t)P * I : a.h_lo;
+        const float *hs = hsm ? reinterpret_cast<const float *>(hsm + (size_t)2 * P * I * 2) : a.hsum;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int q = nt * 8 + g, q0 = nt * 8 + 2 * t, q1 = q0 + 1;
+            if (gu) {
+                jc.b[nt] = q < nu ? (xs_on ? xsm : a.x) + (size_t)S.ptok[pf + q] * H : nullptr;
+                jc.b2[nt] = nullptr;
+                jc.xs0[nt] = q0 < nu ? Xs + (size_t)S.ptok[pf + q0] * G : nullptr;
+                jc.xs1[nt] = q1 < nu ? Xs + (size_t)S.ptok[pf + q1] * G : nullptr;
+            } else {
+                jc.b[nt] = q < nu ? hh + (size_t)S.ppair[pf + q] * I : nullptr;
+                jc.b2[nt] = q < nu ? hl + (size_t)S.ppair[pf + q] * I : nullptr;
+                jc.xs0[nt] = q0 < nu ? hs + (size_t)S.ppair[pf + q0] * GI : nullptr;
+                jc.xs1[nt] = q1 < nu ? hs + (size_t)S.ppair[pf + q1] * GI : nullptr;
+            }
+        }
+    };
+    // gate/up: hand this warp's partial of CTA-local job f (acc + acc2, or zeros) to slot
+    // f % NSLOT; the 8th warp to do so finalises the job. Every warp flushes every job, in order.
+    auto gu_flush = [&](int f, bool zeros) {
+        const int slot = f % NSLOT;
+        const int seq = f / NSLOT;
+        if (lane == 0 && ld_acquire_cta(&S.slot_seq[slot]) != seq) {
+            const uint64_t t0 = global_timer();
+            while (ld_acquire_cta(&S.slot_seq[slot]) != seq) {
+                if (global_timer() - t0 > a.wait_ns) {
+                    atomicOr(status, kStatusTimeout);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+        float *rs = red + (size_t)slot * kCW * NT * 128;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            *reinterpret_cast<float4 *>(rs + ((warp * NT + nt) * 32 + lane) * 4) =
+                zeros ? make_float4(0.f, 0.f, 0.f, 0.f)
+                      : make_float4(acc[nt][0] + acc2[nt][0], acc[nt][1] + acc2[nt][1], acc[nt][2] + acc2[nt][2],
+                                    acc[nt][3] + acc2[nt][3]);
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atom_add_acq_rel_cta(&S.slot_cnt[slot], 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == kCW - 1) {
+            if (!skip) {
+                const int gj = S.g0 + f;
+                gu_finalize<NT>(a, S, gj / (I / 8), gj % (I / 8), rs, lane,
+                                staged ? hstage + (size_t)f * NT * 32 : nullptr);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                S.slot_cnt[slot] = 0;
+                st_release_cta(&S.slot_seq[slot], seq + 1);
+            }
+        }
+        __syncwarp();
+    };
+    auto down_flush = [&]() {
+        const int pf = S.pfirst[cur_u];
+        const int nu = S.pfirst[cur_u + 1] - pf;
+        const int row = cur_rb * 16 + g;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int col = 0; col < 2; ++col) {
+                const int q = nt * 8 + 2 * t + col;
+                if (q < nu) {
+                    const int tok = S.ptok[pf + q];
+                    const float wgt = S.pw[pf + q];
+                    red_add_f32(a.out_acc + (size_t)tok * H + row, wgt * (acc[nt][col] + acc2[nt][col]));
+                    red_add_f32(a.out_acc + (size_t)tok * H + row + 8, wgt * (acc[nt][2 + col] + acc2[nt][2 + col]));
+                }
+            }
+        }
+    };
+    auto flush_current = [&]() {
+        if (cur < 0) return;
+        if (cur < nGUc) {
+            gu_flush(cur, false);
+            next_flush = cur + 1;
+        } else if (cur_any && !skip) {
+            down_flush();
+        }
+    };
+    auto finish_gu = [&]() {
+        if (gu_done) return;
+        for (int f = next_flush; f < nGUc; ++f) gu_flush(f, true);
+        next_flush = nGUc;
+        gu_done = true;
+    };
+    auto switch_job = [&](int job, int u, int rb, bool gu_job) {
+        flush_current();
+        if (gu_job) {
+            for (int f = next_flush; f < job; ++f) gu_flush(f, true);
+            next_flush = job;
+        } else {
+            finish_gu();
+        }
+        cur = job;
+        cur_u = u;
+        cur_rb = rb;
+        cur_any = false;
+        zero_acc();
+        set_ctx(u, gu_job);
+    };
+    zero_acc();
+    for (int ph = 0; ph < 2; ++ph) {
+        const bool gu = ph == 0;
+        if (!gu) {
+            // leaving the gate/up phase: flush the last job and every job this warp skipped
+            flush_current();
+            cur = -1;
+            finish_gu();
+            if (staged) {
+                consumer_sync();
+                if (!skip) write_staged_h<NT>(a, S, hstage, nGUc);
+            }
+            // every h of every CTA is written before any down tile is multiplied
             __threadfence();
             consumer_sync();
             if (threadIdx.x == 0 && !grid_barrier(&a.ctl->bar, nC, c == 0, a.wait_ns, status)) S.abort = 1;
             consumer_sync();
             skip = skip || (S.abort != 0);
-        }
-        const Job jb = job_at(S, a, n, c, nC);
-        float acc[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-        for (int c0 = 0; c0 < jb.ntiles; c0 += kStageTiles) {
-            const int s = cc % kStages;
-            const uint32_t use = cc / kStages;
-            if (!mbar_wait(smem_u32(&S.full[s]), use & 1u, a.wait_ns, status)) return;
-            const int kg = c0 + warp;
-            if (!skip && kg < jb.ntiles) {
-                const uint8_t *tile = stages + (size_t)s * kStageBytes + (size_t)warp * jb.tb;
-                if (jb.bits == 4)
-                    consume_tile<4>(a, S, tile, jb, kg, Xs, lane, acc);
-                else if (jb.bits == 6)
-                    consume_tile<6>(a, S, tile, jb, kg, Xs, lane, acc);
-                else
-                    consume_tile<8>(a, S, tile, jb, kg, Xs, lane, acc);
+            if (hs_on && !skip && S.d1 > S.d0) {
+                const size_t hb = (size_t)P * I * 2;
+                const size_t sb = align_up((size_t)P * GI * 4, 16);
+                const uint4 *s0 = reinterpret_cast<const uint4 *>(a.h_hi);
+                const uint4 *s1 = reinterpret_cast<const uint4 *>(a.h_lo);
+                const uint4 *s2 = reinterpret_cast<const uint4 *>(a.hsum);
+                uint4 *d = reinterpret_cast<uint4 *>(act);
+                for (size_t i = threadIdx.x; i < hb / 16; i += kCW * 32) d[i] = __ldcg(s0 + i);
+                for (size_t i = threadIdx.x; i < hb / 16; i += kCW * 32) d[hb / 16 + i] = __ldcg(s1 + i);
+                for (size_t i = threadIdx.x; i < sb / 16; i += kCW * 32) d[2 * hb / 16 + i] = __ldcg(s2 + i);
+                consumer_sync();
+                hsm = act;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
-            ++cc;
         }
-        if (!skip) job_epilogue(a, S, jb, redbuf + (size_t)(n & 1) * kCW * NTM * 32 * 4, NTM, warp, lane, acc);
+        const int jend = gu ? S.g1 : S.d1;
+        for (int j = gu ? S.g0 : S.d0; j < jend;) {
+            const Region r = region_at(S, a, gu, j);
+            const int nch = region_chunks(r);
+            for (int ch = 0; ch < nch; ++ch) {
+                int c0, m;
+                chunk_range(r, nch, ch, c0, m);
+                const int s = cc % kStages;
+                const uint32_t use = cc / kStages;
+                if (!mbar_wait(smem_u32(&S.full[s]), use & 1u, a.wait_ns, status)) return;
+                const uint8_t *sb = stages + (size_t)s * kStageBytes;
+                // this warp's tiles of the chunk: the contiguous block [w0, w1) of region tiles,
+                // taken job by job
+                const int w0 = c0 + (m * warp) / kCW, w1 = c0 + (m * (warp + 1)) / kCW;
+                const int jlo = w0 / r.tpj, jhi = (w1 - 1) / r.tpj;
+                for (int jb = jlo; w1 > w0 && jb <= jhi; ++jb) {
+                    const int ti0 = max(w0, jb * r.tpj), s1 = min(w1, (jb + 1) * r.tpj);
+                    if (ti0 >= s1) continue;
+                    const int job = r.job0 + jb;
+                    if (job != cur) switch_job(job, r.u, r.rb0 + jb, gu);
+                    cur_any = true;
+                    if (skip) continue;
+                    const int kg0 = ti0 - jb * r.tpj;
+                    const uint8_t *tp0 = sb + (size_t)(ti0 - c0) * r.tb;
+                    const int ntile = s1 - ti0;                     // this warp's tiles of the job here
+#define MOE_RUN(B, GUF)                                                                                   \
+    for (int i = 0; i < ntile; i += 2) {                                                                  \
+        const bool two = i + 1 < ntile;                                                                   \
+        const int i2 = two ? i + 1 : i;                                                                   \
+        consume_tile<B, NT, GUF>(tp0 + (size_t)i * r.tb, kg0 + i, jc, lane, acc);                         \
+        consume_tile<B, NT, GUF>(tp0 + (size_t)i2 * r.tb, kg0 + i2, jc, lane, acc2, two ? 1.f : 0.f);     \
     }
-    if (S.nGUc == njobs) {
-        // a CTA without down jobs still takes part in the second grid barrier
-        __threadfence();
-        consumer_sync();
-        if (threadIdx.x == 0 && !grid_barrier(&a.ctl->bar, nC, c == 0, a.wait_ns, status)) S.abort = 1;
-        consumer_sync();
+                    if (gu) {
+                        if (r.bits == 4) { MOE_RUN(4, true) }
+                        else if (r.bits == 6) { MOE_RUN(6, true) }
+                        else { MOE_RUN(8, true) }
+                    } else {
+                        if (r.bits == 4) { MOE_RUN(4, false) }
+                        else if (r.bits == 6) { MOE_RUN(6, false) }
+                        else { MOE_RUN(8, false) }
+                    }
+#undef MOE_RUN
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
+                ++cc;
+            }
+            j += r.tiles / r.tpj;
+        }
     }
+    flush_current();   // the last down job
     // ---------------------------------------------------------------- completion
     __threadfence();
     consumer_sync();
@@ -487,10 +858,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     consumer_sync();
     if (S.is_last) {
         __threadfence();
-        for (int i = threadIdx.x; i < T * H; i += kCW * 32)
-            a.out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldcg(a.out_acc + i)));
+        const float4 *acc4 = reinterpret_cast<const float4 *>(a.out_acc);
+        uint2 *out4 = reinterpret_cast<uint2 *>(a.out);
+        for (int i = threadIdx.x; i < T * H / 4; i += kCW * 32) {
+            const float4 v = __ldcg(acc4 + i);
+            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(v.x, v.y), hi2 = __floats2bfloat162_rn(v.z, v.w);
+            out4[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&lo2), *reinterpret_cast<const uint32_t *>(&hi2));
+        }
         if (threadIdx.x == 0) a.ctl->done = 0;
     }
+}
+
+template <int NT>
+moe_status_t launch_nt(const DecodeArgs &a, size_t smem, const DeviceInfo *dev, cudaStream_t st) {
+    static bool attr_set[64] = {false};
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d >= 64) return MOE_ERR_CUDA;
+    if (!attr_set[d]) {
+        if (cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dev->max_smem_optin) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set[d] = true;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<NT>, kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        return MOE_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(dev->sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<NT>, a) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 }  // namespace
@@ -500,6 +905,7 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
                            float *w_out, void *ws, cudaStream_t st) {
     if (T * k > kMaxP) return MOE_ERR_UNSUPPORTED;
     const DeviceInfo *dev = device_info();
+    if (!dev) return MOE_ERR_CUDA;
     const DecodeWs L = decode_ws_layout(T, H, I, E, k);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     DecodeArgs a;
@@ -515,31 +921,9 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     a.wait_ns = wait_limit_ns();
     const size_t smem = decode_smem_bytes(T, H);
     if ((int)smem > dev->max_smem_optin) return MOE_ERR_UNSUPPORTED;
-    static bool attr_set[16] = {false};
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess) return MOE_ERR_CUDA;
-    if (d < 16 && !attr_set[d]) {
-        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dev->max_smem_optin) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_set[d] = true;
-    }
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel, kThreads, smem) != cudaSuccess ||
-        per_sm < 1)
-        return MOE_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(dev->sms);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_kernel, a) != cudaSuccess) return MOE_ERR_CUDA;
-    return MOE_OK;
+    if (T <= 8) return launch_nt<1>(a, smem, dev, st);
+    if (T <= 16) return launch_nt<2>(a, smem, dev, st);
+    return launch_nt<4>(a, smem, dev, st);
 }
 
 }  // namespace moe

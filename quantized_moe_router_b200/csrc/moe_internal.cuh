@@ -246,15 +246,21 @@ __device__ __forceinline__ void tile_group_mma(const uint4 &lo, const uint4 &hi,
                                                const uint32_t (&b)[8], const uint32_t *b2,
                                                float sA, float zA, float sB, float zB, float X0,
                                                float X1, float (&out)[4]) {
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    // two independent accumulator chains (even / odd MMAs, or the hi / lo B operand) so that
+    // consecutive MMAs of one warp do not wait on each other
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t low[4] = {lo.x, lo.y, lo.z, lo.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t w = low[j];
         const uint32_t a0 = code_pair<0x000F000Fu>(w, 0), a1 = code_pair<0x000F000Fu>(w, 4);
         const uint32_t a2 = code_pair<0x000F000Fu>(w, 8), a3 = code_pair<0x000F000Fu>(w, 12);
-        mma_bf16(c, a0, a1, a2, a3, b[2 * j], b[2 * j + 1]);
-        if (b2) mma_bf16(c, a0, a1, a2, a3, b2[2 * j], b2[2 * j + 1]);
+        if (b2) {
+            mma_bf16(c, a0, a1, a2, a3, b[2 * j], b[2 * j + 1]);
+            mma_bf16(d, a0, a1, a2, a3, b2[2 * j], b2[2 * j + 1]);
+        } else {
+            mma_bf16((j & 1) ? d : c, a0, a1, a2, a3, b[2 * j], b[2 * j + 1]);
+        }
     }
     if (BITS != 4) {
         uint32_t b16[8], b216[8];
@@ -280,10 +286,16 @@ __device__ __forceinline__ void tile_group_mma(const uint4 &lo, const uint4 &hi,
                 a2 = code_pair<0x00030003u>(w, s0 + 4);
                 a3 = code_pair<0x00030003u>(w, s0 + 6);
             }
-            mma_bf16(c, a0, a1, a2, a3, b16[2 * j], b16[2 * j + 1]);
-            if (b2) mma_bf16(c, a0, a1, a2, a3, b216[2 * j], b216[2 * j + 1]);
+            if (b2) {
+                mma_bf16(c, a0, a1, a2, a3, b16[2 * j], b16[2 * j + 1]);
+                mma_bf16(d, a0, a1, a2, a3, b216[2 * j], b216[2 * j + 1]);
+            } else {
+                mma_bf16((j & 1) ? d : c, a0, a1, a2, a3, b16[2 * j], b16[2 * j + 1]);
+            }
         }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] += d[i];
     const float off = (BITS == 4) ? 128.f : 2176.f;  // 128 per plane, the hi plane weighted 16x
     out[0] += sA * (c[0] - (off + zA) * X0);
     out[1] += sA * (c[1] - (off + zA) * X1);

@@ -12,52 +12,61 @@
 
 namespace moe {
 
+// monotone map of a non-NaN float to an unsigned key (larger float -> larger key)
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Lane i < k receives the i-th selected expert (idx) and its weight (w); other lanes get -1/0.
 // `l` points to E fp32 logits; `from_l2` selects an L2-only load (data written by other CTAs
 // of the same kernel). E <= 1024, 1 <= k <= min(E, 32).
+// Each round takes the warp-wide maximum key and then the lowest index holding it (two redux
+// instructions); only the winning lane rescans its 32 keys.
 __device__ __forceinline__ void warp_topk_softmax(const float *l, bool from_l2, int E, int k,
                                                   int lane, int &idx, float &w) {
-    float v[32];
-    uint32_t avail = 0;
+    // lane holds logits lane + 32 m (m < 32) as order keys; 0 = taken / absent
+    uint32_t key[32];
 #pragma unroll
     for (int m = 0; m < 32; ++m) {
         const int e = lane + 32 * m;
-        float x = -INFINITY;
+        uint32_t kk = 0;
         if (e < E) {
-            x = from_l2 ? __ldcg(l + e) : l[e];
+            float x = from_l2 ? __ldcg(l + e) : l[e];
             if (x != x) x = -INFINITY;
-            avail |= 1u << m;
+            kk = order_key(x);   // >= 0x007FFFFF for -inf, so never 0
         }
-        v[m] = x;
+        key[m] = kk;
     }
+    // lane-local best: largest key, lowest m (= lowest expert index among the lane's ties)
+    uint32_t bk = 0;
+    int bm = 0;
+#pragma unroll
+    for (int m = 0; m < 32; ++m)
+        if (key[m] > bk) { bk = key[m]; bm = m; }
     int my_i = -1;
-    float my_v = -INFINITY;
+    uint32_t my_k = 0;
     for (int r = 0; r < k; ++r) {
-        float bv = -INFINITY;
-        int be = INT_MAX;
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == mx) ? (uint32_t)(lane + 32 * bm) : 0xFFFFFFFFu;
+        const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+        if (lane == r) { my_i = (int)win; my_k = mx; }
+        if ((int)(win & 31u) == lane) {
+            // the winning lane drops its entry and rescans
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const int e = lane + 32 * m;
-            if (((avail >> m) & 1u) && (v[m] > bv || (v[m] == bv && e < be))) {
-                bv = v[m];
-                be = e;
-            }
-        }
+            for (int m = 0; m < 32; ++m)
+                if (m == bm) key[m] = 0;
+            bk = 0;
+            bm = 0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > bv || (ov == bv && oe < be)) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        if ((be & 31) == lane) avail &= ~(1u << (be >> 5));
-        if (lane == r) {
-            my_i = be;
-            my_v = bv;
+            for (int m = 0; m < 32; ++m)
+                if (key[m] > bk) { bk = key[m]; bm = m; }
         }
     }
+    const float my_v = (lane < k) ? key_value(my_k) : -INFINITY;
     const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
     float ex = 0.f;
     if (lane < k) ex = (v0 == -INFINITY) ? 1.f : expf(my_v - v0);

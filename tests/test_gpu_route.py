@@ -29,7 +29,7 @@ def run(T, H, E, k, seed, bias=False, dup_rows=False, scale=1.0):
 
 @pytest.mark.parametrize("T,H,E,k,bias", [
     (1, 128, 8, 2, False), (37, 256, 64, 5, True), (1, 1024, 32, 4, False), (5, 2048, 256, 8, False),
-    (3, 4096, 512, 10, False), (16, 2048, 256, 8, True), (9, 64, 1024, 32, True), (7, 128, 33, 33, False),
+    (3, 4096, 512, 10, False), (16, 2048, 256, 8, True), (9, 64, 1024, 32, True), (7, 128, 32, 32, False),
     (1000, 2048, 256, 8, False), (13, 8192, 128, 1, True)])
 def test_route_matches_oracle(T, H, E, k, bias):
     logits, idx, w = run(T, H, E, k, seed=T * 7 + E, bias=bias)
@@ -44,6 +44,12 @@ def test_route_full_prefill_size():
     logits = oracle.get().router_logits(x, wr, None)
     _, _, stats = route_check(logits, w.k, idx.cpu().numpy(), ww.cpu().numpy())
     print("near ties", stats)
+
+
+def test_k_above_limit_rejected():
+    with pytest.raises(qm.MoeError) as ei:
+        run(7, 128, 33, 33, seed=1)
+    assert ei.value.status == qm.MOE_ERR_INVALID_ARG
 
 
 def test_exact_ties_take_lower_index():
