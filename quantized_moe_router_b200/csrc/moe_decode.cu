@@ -38,7 +38,8 @@ namespace moe {
 namespace {
 
 constexpr int kCW = 8;                      // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;    // + one producer warp
+constexpr int kWarps = kCW + 2;             // + one producer warp + one gate/up epilogue warp
+constexpr int kThreads = kWarps * 32;
 constexpr int kStageBytes = 24576;          // bytes per bulk copy / pipeline stage
 constexpr int kStages = 4;
 constexpr int kActBytes = 49152;            // smem for x (routing + gate/up), then h (down)
@@ -103,6 +104,8 @@ __host__ __device__ inline size_t h_smem_bytes(int P, int I) {
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// consumers + the epilogue warp: every gate/up job of the CTA is finalised
+__device__ __forceinline__ void gu_done_sync() { asm volatile("bar.sync 2, 288;" ::: "memory"); }
 // CTA-scope acquire / release on shared-memory words (hand-off of partial sums between warps)
 __device__ __forceinline__ int ld_acquire_cta(const int *p) {
     int v;
@@ -251,7 +254,7 @@ __device__ void gu_finalize(const DecodeArgs &a, const DecodeSmem &S, int u, int
             const int q = nt * 8 + 2 * t + col;
             const bool valid = q < nu;
             const float gate = v[col], up = v[2 + col];
-            const float h = gate / (1.f + expf(-gate)) * up;
+            const float h = __fdividef(gate, 1.f + __expf(-gate)) * up;
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             his |= (uint32_t)__bfloat16_as_ushort(hi) << (16 * col);
@@ -311,7 +314,7 @@ __device__ void cta_topk(const DecodeArgs &a, DecodeSmem &S, uint32_t *cand_key,
     const int T = a.T, E = a.E, K = a.k;
     const int NC = kSlices * K;                 // candidates per token
     const int slice = (E + kSlices - 1) / kSlices;
-    for (int task = warp; task < T * kSlices; task += kCW + 1) {
+    for (int task = warp; task < T * kSlices; task += kWarps) {
         const int t = task / kSlices, sl = task % kSlices;
         const int e0 = sl * slice, e1 = min(E, e0 + slice);
         uint32_t key[4];
@@ -347,24 +350,37 @@ __device__ void cta_topk(const DecodeArgs &a, DecodeSmem &S, uint32_t *cand_key,
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < T * NC; i += kThreads) {
-        const int t = i / NC;
-        const uint32_t mk = cand_key[i];
-        if (mk == 0) continue;
-        const int mi = cand_idx[i];
-        int rank = 0;
-        for (int j = 0; j < NC; ++j) {
-            const uint32_t ok = cand_key[t * NC + j];
-            const int oi = cand_idx[t * NC + j];
-            rank += (ok > mk || (ok == mk && oi < mi)) ? 1 : 0;
+    // stage 2: per token, the k best of its 8k candidates (same order: key desc, index asc)
+    for (int t = warp; t < T; t += kWarps) {
+        uint32_t ck[8];
+        int ci[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int j = lane + 32 * m;
+            ck[m] = (j < NC) ? cand_key[t * NC + j] : 0u;
+            ci[m] = (j < NC) ? cand_idx[t * NC + j] : 0x7FFFFFFF;
         }
-        if (rank < K) {
-            S.sel_idx[t * K + rank] = mi;
-            S.sel_key[t * K + rank] = mk;
+        for (int r = 0; r < K; ++r) {
+            uint32_t bk = 0;
+            int bi = 0x7FFFFFFF, bm = 0;
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                if (ck[m] > bk || (ck[m] == bk && ck[m] != 0 && ci[m] < bi)) { bk = ck[m]; bi = ci[m]; bm = m; }
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t win = __reduce_min_sync(0xffffffffu, (bk == mx) ? (uint32_t)bi : 0xFFFFFFFFu);
+            if (lane == 0) {
+                S.sel_idx[t * K + r] = (int)win;
+                S.sel_key[t * K + r] = mx;
+            }
+            if (bk == mx && (uint32_t)bi == win) {
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    if (m == bm) ck[m] = 0;
+            }
         }
     }
     __syncthreads();
-    for (int t = warp; t < T; t += kCW + 1) {
+    for (int t = warp; t < T; t += kWarps) {
         const float v = (lane < K) ? key_value(S.sel_key[t * K + lane]) : -INFINITY;
         const float v0 = __shfl_sync(0xffffffffu, v, 0);
         float ex = 0.f;
@@ -455,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
     if (xs_on && !mbar_wait(smem_u32(&S.xbar), 0, a.wait_ns, status)) S.abort = 1;
     if (wr_on && ne > 0 && !mbar_wait(smem_u32(&S.wbar), 0, a.wait_ns, status)) S.abort = 1;
     const uint16_t *xr = xs_on ? xsm : a.x;
-    for (int q = warp; q < ne * T; q += kCW + 1) {
+    for (int q = warp; q < ne * T; q += kWarps) {
         const int i = q / T, t = q % T;
         const int e = c + i * nC;
         const float *wrow = wr_on ? wsm + (size_t)i * H : a.wr + (size_t)e * H;
@@ -475,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         if (lane == 0) a.logits[(size_t)t * E + e] = acc + (a.bias ? a.bias[e] : 0.f);
     }
     // per-token sums of x over each group (one warp per group, two values per lane)
-    for (int i = warp; i < T * G; i += kCW + 1) {
+    for (int i = warp; i < T * G; i += kWarps) {
         const uint32_t v = *reinterpret_cast<const uint32_t *>(xr + (size_t)i * kGroup + 2 * lane);
         float s = __uint_as_float(v << 16) + __uint_as_float(v & 0xFFFF0000u);
 #pragma unroll
@@ -495,8 +511,71 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         cta_topk(a, S, cand_key, cand_idx, warp, lane);
     }
     __syncthreads();
-    if (warp == 0) {
-        // unique experts (ascending id), their pair lists (ascending token) and the job ranges
+    if (warp == 0 && P <= 32) {
+        // unique experts (ascending id), their pair lists (ascending token) and the byte prefixes,
+        // one pair per lane
+        const bool v = lane < P && !aborted;
+        const int e = v ? S.sel_idx[lane] : 0x7FFFFFFF;
+        const uint32_t same = __match_any_sync(0xffffffffu, e);
+        const bool first = v && (__ffs(same) - 1 == lane);
+        int *tmp = reinterpret_cast<int *>(S.cursor);
+        tmp[lane] = first ? e : (v ? -1 - e : 0x7FFFFFFF);    // >= 0: first occurrence of an expert
+        __syncwarp();
+        int slot = 0, before = 0;                             // distinct experts / pairs with a smaller id
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const int ej = tmp[j];
+            const int id = ej >= 0 ? ej : -1 - ej;
+            if (ej != 0x7FFFFFFF && id < e) {
+                ++before;
+                slot += ej >= 0 ? 1 : 0;
+            }
+        }
+        const int U = __popc(__ballot_sync(0xffffffffu, first));
+        const uint32_t tu = first ? (uint32_t)tile_bytes(S.ebits[e]) / 64 : 0;    // 64-byte units per tile
+        if (first) {
+            S.ubits[slot] = S.ebits[e];
+            S.uoff[slot] = S.eoff[e];
+            S.pfirst[slot] = before;
+            S.cnt[slot] = __popc(same);
+        }
+        if (v) {
+            const int pos = before + __popc(same & ((1u << lane) - 1u));
+            S.ppair[pos] = lane;
+            S.ptok[pos] = lane / K;
+            S.pw[pos] = S.sel_w[lane];
+        }
+        __syncwarp();
+        // byte prefixes over slots (lane = slot)
+        const uint32_t ts = (lane < U) ? (uint32_t)tile_bytes(S.ubits[lane]) / 64 : 0;
+        const uint32_t bg = ts * (uint32_t)(I / 8) * G, bd = ts * (uint32_t)(H / 16) * GI;
+        uint32_t ig = bg, id = bd;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t og = __shfl_up_sync(0xffffffffu, ig, off);
+            const uint32_t od = __shfl_up_sync(0xffffffffu, id, off);
+            if (lane >= off) {
+                ig += og;
+                id += od;
+            }
+        }
+        if (lane < U) {
+            S.cgu[lane] = ig - bg;
+            S.cd[lane] = id - bd;
+        }
+        if (lane == U - 1) {
+            S.cgu[U] = ig;
+            S.cd[U] = id;
+        }
+        if (lane == 0) {
+            S.U = U;
+            S.pfirst[U] = aborted ? 0 : P;
+            if (U == 0) S.cgu[0] = S.cd[0] = 0;
+        }
+        (void)tu;
+        __syncwarp();
+    } else if (warp == 0) {
+        // unique experts (ascending id), their pair lists (ascending token) and the byte prefixes
         for (int p = lane; p < (aborted ? 0 : P); p += 32)
             atomicOr(&S.selmask[S.sel_idx[p] >> 5], 1u << (S.sel_idx[p] & 31));
         __syncwarp();
@@ -576,28 +655,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
             if (p < P && rank == 0) S.cursor[u] += __popc(peers);
             __syncwarp();
         }
+    }
+    if (warp == 0) {
         // Job ranges: the gate/up sequence is cut at multiples of its bytes / nCTA; the down
         // sequence is cut so that each CTA's gate/up + down bytes are the layer's bytes / nCTA.
         // That cut is monotone in the CTA index when every CTA's down share exceeds one gate/up
         // job (plus rounding); otherwise (tiny layers) the down sequence is cut on its own.
+        // 32-bit arithmetic: floor(X * c / nC) = (X / nC) * c + ((X % nC) * c) / nC
+        __syncwarp();
+        const int Uj = aborted ? 0 : S.U;
+        const int pg = I / 8, pd = H / 16;
+        const uint32_t GUB = S.cgu[Uj], DB = S.cd[Uj], B = GUB + DB;
+        auto cut = [&](uint32_t X, int cc) -> uint32_t {
+            return (X / nC) * (uint32_t)cc + ((X % nC) * (uint32_t)cc) / nC;
+        };
+        uint32_t mj = 0;                        // largest gate/up job (64-byte units)
+        for (int u = lane; u < Uj; u += 32) mj = max(mj, (S.cgu[u + 1] - S.cgu[u]) / pg);
+        mj = __reduce_max_sync(0xffffffffu, mj);
+        const bool mono = (uint64_t)(mj + 2) * nC <= DB;
+        // lane 0 / 1: the gate/up cut at c / c+1; then lanes 0 / 1: the down cut at c / c+1
+        int gcut = 0;
+        if (lane < 2) {
+            const int cc = c + lane;
+            gcut = (cc >= nC) ? Uj * pg : job_at_unit(S.cgu, Uj, pg, cut(GUB, cc));
+        }
+        const int g0 = __shfl_sync(0xffffffffu, gcut, 0), g1 = __shfl_sync(0xffffffffu, gcut, 1);
+        int dcut = 0;
+        if (lane < 2) {
+            const int cc = c + lane;
+            const int gj = lane == 0 ? g0 : g1;
+            const uint32_t pos = mono ? cut(B, cc) - job_start_unit(S.cgu, Uj, pg, gj) : cut(DB, cc);
+            dcut = (cc >= nC) ? Uj * pd : job_at_unit(S.cd, Uj, pd, pos);
+        }
+        const int d0 = __shfl_sync(0xffffffffu, dcut, 0), d1 = __shfl_sync(0xffffffffu, dcut, 1);
         if (lane == 0) {
-            const int Uj = aborted ? 0 : U;
-            const int pg = I / 8, pd = H / 16;
-            const uint64_t GUB = S.cgu[Uj], DB = S.cd[Uj], B = GUB + DB;
-            const int g0 = job_at_unit(S.cgu, Uj, pg, (uint32_t)(GUB * c / nC));
-            const int g1 = (c == nC - 1) ? Uj * pg : job_at_unit(S.cgu, Uj, pg, (uint32_t)(GUB * (c + 1) / nC));
-            uint32_t maxjob = 0;
-            for (int u = 0; u < Uj; ++u) maxjob = max(maxjob, (S.cgu[u + 1] - S.cgu[u]) / pg);
-            uint32_t p0, p1;
-            if ((uint64_t)(maxjob + 2) * nC <= DB) {
-                p0 = (uint32_t)(B * c / nC - job_start_unit(S.cgu, Uj, pg, g0));
-                p1 = (uint32_t)(B * (c + 1) / nC - job_start_unit(S.cgu, Uj, pg, g1));
-            } else {
-                p0 = (uint32_t)(DB * c / nC);
-                p1 = (uint32_t)(DB * (c + 1) / nC);
-            }
-            const int d0 = job_at_unit(S.cd, Uj, pd, p0);
-            const int d1 = (c == nC - 1) ? Uj * pd : job_at_unit(S.cd, Uj, pd, p1);
             S.g0 = g0;
             S.g1 = g1;
             S.d0 = d0;
@@ -634,13 +725,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
         return;
     }
+    const int nGUc = S.nGUc;
+    const bool staged = (size_t)nGUc * NT * 32 * sizeof(uint2) <= (size_t)kHStageBytes;
+    if (warp == kCW + 1) {
+        // ------------------------------------------------------------ gate/up epilogue
+        // Finalises the CTA's gate/up jobs in order as the 8 consumer warps flush their partials,
+        // so that no consumer warp stalls on SiLU-GLU and the h write.
+        for (int f = 0; f < nGUc; ++f) {
+            const int slot = f % NSLOT;
+            bool ok = true;
+            if (lane == 0 && ld_acquire_cta(&S.slot_cnt[slot]) != kCW) {
+                const uint64_t t0 = global_timer();
+                while (ld_acquire_cta(&S.slot_cnt[slot]) != kCW) {
+                    if (global_timer() - t0 > a.wait_ns) {
+                        atomicOr(status, kStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (ok && !aborted) {
+                const int gj = S.g0 + f;
+                gu_finalize<NT>(a, S, gj / (I / 8), gj % (I / 8), red + (size_t)slot * kCW * NT * 128, lane,
+                                staged ? hstage + (size_t)f * NT * 32 : nullptr);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                S.slot_cnt[slot] = 0;
+                st_release_cta(&S.slot_seq[slot], f / NSLOT + 1);
+            }
+        }
+        gu_done_sync();
+        return;
+    }
 
     // ---------------------------------------------------------------- consumers
     uint32_t cc = 0;
     bool skip = aborted;
     const uint8_t *hsm = nullptr;
-    const int nGUc = S.nGUc;
-    const bool staged = (size_t)nGUc * NT * 32 * sizeof(uint2) <= (size_t)kHStageBytes;
     int cur = -1, cur_u = 0, cur_rb = 0;   // job in progress (CTA-local index), -1: none
     bool cur_any = false;
     int next_flush = 0;                    // gate/up jobs below this index are flushed by this warp
@@ -678,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
         }
     };
     // gate/up: hand this warp's partial of CTA-local job f (acc + acc2, or zeros) to slot
-    // f % NSLOT; the 8th warp to do so finalises the job. Every warp flushes every job, in order.
+    // f % NSLOT for the epilogue warp. Every warp flushes every job, in order.
     auto gu_flush = [&](int f, bool zeros) {
         const int slot = f % NSLOT;
         const int seq = f / NSLOT;
@@ -700,21 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
                       : make_float4(acc[nt][0] + acc2[nt][0], acc[nt][1] + acc2[nt][1], acc[nt][2] + acc2[nt][2],
                                     acc[nt][3] + acc2[nt][3]);
         __syncwarp();
-        int old = 0;
-        if (lane == 0) old = atom_add_acq_rel_cta(&S.slot_cnt[slot], 1);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == kCW - 1) {
-            if (!skip) {
-                const int gj = S.g0 + f;
-                gu_finalize<NT>(a, S, gj / (I / 8), gj % (I / 8), rs, lane,
-                                staged ? hstage + (size_t)f * NT * 32 : nullptr);
-            }
-            __syncwarp();
-            if (lane == 0) {
-                S.slot_cnt[slot] = 0;
-                st_release_cta(&S.slot_seq[slot], seq + 1);
-            }
-        }
+        if (lane == 0) atom_add_acq_rel_cta(&S.slot_cnt[slot], 1);
         __syncwarp();
     };
     auto down_flush = [&]() {
@@ -773,10 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a)
             flush_current();
             cur = -1;
             finish_gu();
-            if (staged) {
-                consumer_sync();
-                if (!skip) write_staged_h<NT>(a, S, hstage, nGUc);
-            }
+            gu_done_sync();
+            if (staged && !skip) write_staged_h<NT>(a, S, hstage, nGUc);
             // every h of every CTA is written before any down tile is multiplied
             __threadfence();
             consumer_sync();
