@@ -31,6 +31,7 @@ SIGNATURES = {
     "moe_workspace_init": (_i, [_vp, _sz, _vp]),
     "moe_expert_forward_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_forward_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_forward_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_set_wait_limit_ns": (None, [_u64]),
 }
@@ -167,6 +168,17 @@ def forward_prefill(x, w_router, bias, packed, I, E, k, ws, out=None, idx_out=No
     """Prefill-path expert block (any T): returns out [T x H] bf16."""
     return _forward(lib().moe_expert_forward_prefill, "moe_expert_forward_prefill", x, w_router, bias, packed,
                     I, E, k, ws, out, idx_out, w_out, stream)
+
+
+def forward_decode_noalloc(x, w_router, bias, packed, I, E, k, out=None, idx_out=None, w_out=None, stream=None):
+    """Decode-path expert block using the library's fixed device scratch (no workspace)."""
+    T, H = x.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_expert_forward_decode_noalloc(_p(x), _p(w_router), _p(bias), _p(packed), T, H, I, E, k,
+                                                   _p(out), _p(idx_out), _p(w_out), _stream(stream)),
+           "moe_expert_forward_decode_noalloc")
+    return out
 
 
 def device_status(ws: torch.Tensor, stream=None) -> int:

@@ -75,6 +75,15 @@ moe_status_t forward_common(const uint16_t *x, const float *w_router, const floa
     return check_device();
 }
 
+// Scratch of moe_expert_forward_decode_noalloc: a fixed array in the library's own device memory,
+// zero-initialised when the library is loaded on a device and kept (with the last call's
+// contents) until the process exits. Host code may not use the array's name as an address; the
+// entry point resolves the device address once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = 4u << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64] = {nullptr};
+
 }  // namespace
 
 extern "C" {
@@ -158,6 +167,30 @@ moe_status_t moe_expert_forward_decode(const uint16_t *x, const float *w_router,
     if (s != MOE_OK) return s;
     if (T > kMaxT || (long long)T * k > 256 || H > 8192) return MOE_ERR_UNSUPPORTED;
     return launch_decode(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, ws, (cudaStream_t)stream);
+}
+
+moe_status_t moe_expert_forward_decode_noalloc(const uint16_t *x, const float *w_router, const float *bias,
+                                               const void *packed, int T, int H, int I, int E, int k, uint16_t *out,
+                                               int32_t *idx_out, float *w_out, moe_stream_t stream) {
+    const size_t need = moe_workspace_bytes(T, H, I, E, k, MOE_MODE_DECODE);
+    if (need == 0) return MOE_ERR_INVALID_ARG;
+    if (need > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return MOE_ERR_CUDA;
+    if (d < 0 || d >= 64) return MOE_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    {
+        // set-up, once per device and with that device current: the array's device address
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_addr[d]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+            g_noalloc_addr[d] = p;
+        }
+        scratch = g_noalloc_addr[d];
+    }
+    return moe_expert_forward_decode(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, scratch,
+                                     kNoAllocScratchBytes, stream);
 }
 
 moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router, const float *bias,
