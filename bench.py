@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="stack only this many layers of the workload (smaller case for profiling)")
     return ap.parse_args()
 
 
@@ -386,6 +388,9 @@ def main():
     args = parse()
     import synth
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, layers=min(args.layers, w.layers))
     if args.impl == "reference":
         run_reference(args, w)
     else:
