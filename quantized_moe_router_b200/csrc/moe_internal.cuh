@@ -92,7 +92,7 @@ inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
 }
 
 struct PrefillWs {
-    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, xsum, h_hi, h_lo, hsum, out_acc, total;
+    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, h, out_acc, total;
     int nblk;  // token blocks of the stable scatter
 };
 constexpr int kScatterTokens = 64;
@@ -109,10 +109,8 @@ inline PrefillWs prefill_ws_layout(int T, int H, int I, int E, int k) {
     w.blockhist = take((size_t)w.nblk * E * 4);
     w.pair_tok = take(P * 4);
     w.pair_w = take(P * 4);
-    w.xsum = take((size_t)T * (H / kGroup) * 4);
-    w.h_hi = take(P * I * 2);
-    w.h_lo = take(P * I * 2);
-    w.hsum = take(P * (I / kGroup) * 4);
+    w.nt_start = take((size_t)(E + 1) * 4);
+    w.h = take(P * I * 2);                 // bf16 h of every (token, expert) pair, bucket order
     w.out_acc = take((size_t)T * H * 4);
     w.total = o;
     return w;

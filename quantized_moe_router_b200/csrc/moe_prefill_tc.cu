@@ -1,0 +1,647 @@
+// moe_prefill_tc.cu -- the prefill grouped GEMMs on the 5th-generation tensor cores (tcgen05).
+//
+// In prefill the expert block is a dense contraction: after bucketing, expert e multiplies its
+// n_e tokens (about 128 at 4096 tokens, 256 experts, top-8) by its dequantised weights, and a
+// long prompt touches nearly every expert of a layer (the pages "Qwen-tin" and
+// "--moe-direct-io"). Both GEMMs run in one persistent kernel each (one CTA per SM) whose work
+// unit is (expert, 128 weight rows, up to 256 of the expert's tokens):
+//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, copy their
+//     lane fragments from HBM into a small ring with cp.async (3 K steps ahead), then write
+//     w = (q - z) * s as bf16 into a 128-byte-swizzled K-major shared tile A [128 x 64];
+//   * 2 loader warps gather the unit's token rows (x rows for gate/up, h rows for down) into a
+//     swizzled tile B [N x 64] with cp.async;
+//   * 1 warp issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128, N = tokens rounded up
+//     to 16) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
+//     each ring stage with tcgen05.commit;
+//   * 4 epilogue warps read the other accumulator with tcgen05.ld while the next unit runs:
+//     gate/up pairs each gate row with its up row (8 TMEM lanes apart), applies SiLU-GLU and
+//     stores h (bf16, bucket order) through a shared staging tile; down adds w * y into the
+//     fp32 output accumulator with red.add.
+// Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kTM = 128;                          // weight rows per unit (UMMA M)
+constexpr int kMaxN = 256;                        // tokens per unit (UMMA N limit)
+constexpr int kABStages = 3;
+constexpr int kABytes = kTM * 128;                // 128 rows x 64 bf16
+constexpr int kBBytes = kMaxN * 128;              // 256 rows x 64 bf16
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kRawAhead = 3;                      // K steps of packed tiles in flight per warp
+constexpr int kRawSlots = kRawAhead + 1;
+constexpr int kRawTile = 1280;                    // lane copies: lo 512 | hi 512 | scale/zero 256
+constexpr int kRawStage = 8 * kRawTile;
+constexpr int kStagingBytes = kMaxN * 128;        // h staging: 256 tokens x 64 bf16
+constexpr int kDqWarps = 8, kLdWarps = 2;
+constexpr int kMmaWarp = kDqWarps + kLdWarps;
+constexpr int kEpiWarp0 = kMmaWarp + 1;
+constexpr int kTcWarps = kEpiWarp0 + 4;
+constexpr int kTcThreads = kTcWarps * 32;
+constexpr uint32_t kTmemCols = 2 * kMaxN;         // two accumulators of 256 fp32 columns
+constexpr int kLoaderLag = 1;                     // K steps a loader keeps in flight before arriving
+constexpr int kBarEpi = 1, kBarLd = 2;            // named barriers (0 is __syncthreads)
+constexpr size_t kTcSmemBytes =
+    (size_t)kABStages * kStageBytes + (size_t)kRawSlots * kRawStage + kStagingBytes + 1024;
+
+struct TcArgs {
+    const uint8_t *packed;
+    int H, I, E;
+    const int32_t *counts, *offsets, *nt_start, *pair_tok;
+    const float *pair_w;
+    const uint16_t *act;  // gate/up: x [T x H]; down: h [pairs x I] in bucket order
+    uint16_t *h;          // gate/up output: h [pairs x I] bf16
+    float *out_acc;       // down output: [T x H] fp32
+    uint64_t wait_ns;
+    uint32_t *status;
+};
+
+struct TcShared {
+    uint64_t ab_full[kABStages];
+    uint64_t ab_empty[kABStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t fin;
+    uint32_t tmem_base;
+    volatile int abort;
+    int rows[kMaxN];  // loaders: activation row of each token of the current unit
+};
+
+// ------------------------------------------------------------------------------ work units
+// An expert's n tokens are cut into ceil(n / tile) N tiles of at most 256 (sizes rounded to 16).
+__host__ __device__ inline int ntile_size(int n) {
+    const int c = (n + kMaxN - 1) / kMaxN;
+    return c == 0 ? 0 : (((n + c - 1) / c + 15) & ~15);
+}
+__host__ __device__ inline int ntile_count(int n) {
+    const int s = ntile_size(n);
+    return s == 0 ? 0 : (n + s - 1) / s;
+}
+
+struct Unit {
+    int e, mt, n0, nn, nr, base;
+};
+
+// Unit u = (N tile u / mtiles, M tile u % mtiles); the expert owning an N tile is found by a
+// binary search of nt_start (exclusive prefix of the experts' N-tile counts).
+__device__ __forceinline__ Unit unit_at(const TcArgs &a, int u, int mtiles) {
+    Unit U;
+    const int ti = u / mtiles;
+    U.mt = u - ti * mtiles;
+    int lo = 0, hi = a.E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a.nt_start + mid) <= ti) lo = mid;
+        else hi = mid;
+    }
+    U.e = lo;
+    const int n_e = __ldg(a.counts + lo);
+    const int sz = ntile_size(n_e);
+    U.n0 = (ti - __ldg(a.nt_start + lo)) * sz;
+    U.nn = min(sz, n_e - U.n0);
+    U.nr = (U.nn + 15) & ~15;
+    U.base = __ldg(a.offsets + lo);
+    return U;
+}
+
+// ------------------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    // K-major operand, 128-byte swizzle: 8-row x 128-byte atoms stacked 1024 bytes apart
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;              // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset: next 8-row atom
+    d |= (uint64_t)1 << 46;              // descriptor version
+    d |= (uint64_t)2 << 61;              // SWIZZLE_128B
+    return d;
+}
+__device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
+    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Bounded mbarrier wait that also gives up when another role of the CTA has aborted.
+__device__ __forceinline__ bool tc_wait(TcShared &S, const TcArgs &a, uint64_t *bar, uint32_t parity) {
+    const uint32_t b = smem_u32(bar);
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if (mbar_try_wait(b, parity)) return true;
+        if (S.abort) return false;
+        if (global_timer() - t0 > a.wait_ns) {
+            atomicOr(a.status, kStatusTimeout);
+            S.abort = 1;
+            return false;
+        }
+    }
+}
+
+// byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled K-major tile
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// ------------------------------------------------------------------------------ dequantisation
+// A code nibble becomes an fp32 value by byte placement (prmt) under a fixed exponent byte:
+//   low nibble q of byte x  -> 0x3F0q0000 = 0.5 + q/256   (row g of the lane fragment)
+//   high nibble q of byte x -> 0x3F80(q<<4)00 = 1 + q/2048 (row g+8)
+// so w = (q - z) * s = f * S + C with S = 256 s (2048 s) and C = -(128 + z) s (-(2048 + z) s).
+// C is rounded once to fp32 (|error| <= 2^-24 |C|, far below the bf16 rounding of w).
+__device__ __forceinline__ float nib_float(uint32_t m, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(m), "r"(0x3F800000u), "r"(sel));
+    return __uint_as_float(r);
+}
+// (x0 * S + C, x1 * S + C) with one packed fp32x2 FMA, rounded to a bf16 pair (x0 in the low half)
+__device__ __forceinline__ uint32_t fma2_bf16(float x0, float x1, float S, float C) {
+    float r0, r1;
+    asm("{ .reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3}; mov.b64 b, {%4, %4}; mov.b64 c, {%5, %5};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\t"
+        "mov.b64 {%0, %1}, d; }"
+        : "=f"(r0), "=f"(r1)
+        : "f"(x0), "f"(x1), "f"(S), "f"(C));
+    const __nv_bfloat162 v = __floats2bfloat162_rn(r0, r1);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+// x * S + y * S2 + C for two elements (6/8-bit codes: the low and the high code plane)
+__device__ __forceinline__ uint32_t fma2_bf16_hi(float x0, float x1, float y0, float y1, float S, float S2,
+                                                 float C) {
+    float t0 = fmaf(x0, S, C), t1 = fmaf(x1, S, C);
+    t0 = fmaf(y0, S2, t0);
+    t1 = fmaf(y1, S2, t1);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(t0, t1);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile, from the
+// lane's fragment copies in `rawt`, stored into the swizzled A tile rows 16b+g and 16b+g+8.
+// Word j of the lo plane holds columns 16t+4j+{0,1,2,3} in bytes {0,2,1,3}: row g in the low
+// nibbles, row g+8 in the high nibbles.
+template <int BITS>
+__device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uint8_t *As, int b) {
+    const int g = L >> 2, t = L & 3;
+    const uint4 lo = *reinterpret_cast<const uint4 *>(rawt + 16 * L);
+    const uint2 sz = *reinterpret_cast<const uint2 *>(rawt + 1024 + 8 * L);
+    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
+    const uint32_t w[4] = {lo.x, lo.y, lo.z, lo.w};
+    uint32_t ra[8], rb[8];
+    if (BITS == 4) {
+        const float SA = 256.f * sA, CA = -(128.f + zA) * sA;
+        const float SB = 2048.f * sB, CB = -(2048.f + zB) * sB;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t m0 = w[j] & 0x0F0F0F0Fu, m1 = w[j] & 0xF0F0F0F0u;
+            ra[2 * j] = fma2_bf16(nib_float(m0, 0x7054), nib_float(m0, 0x7254), SA, CA);
+            ra[2 * j + 1] = fma2_bf16(nib_float(m0, 0x7154), nib_float(m0, 0x7354), SA, CA);
+            rb[2 * j] = fma2_bf16(nib_float(m1, 0x7604), nib_float(m1, 0x7624), SB, CB);
+            rb[2 * j + 1] = fma2_bf16(nib_float(m1, 0x7614), nib_float(m1, 0x7634), SB, CB);
+        }
+    } else if (BITS == 8) {
+        // q = lo + 16 hi, the hi plane in the same nibble arrangement
+        const uint4 hi = *reinterpret_cast<const uint4 *>(rawt + 512 + 16 * L);
+        const uint32_t v[4] = {hi.x, hi.y, hi.z, hi.w};
+        const float SA = 256.f * sA, SA2 = 4096.f * sA, CA = -(128.f + 2048.f + zA) * sA;
+        const float SB = 2048.f * sB, SB2 = 32768.f * sB, CB = -(2048.f + 32768.f + zB) * sB;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t m0 = w[j] & 0x0F0F0F0Fu, m1 = w[j] & 0xF0F0F0F0u;
+            const uint32_t h0 = v[j] & 0x0F0F0F0Fu, h1 = v[j] & 0xF0F0F0F0u;
+            ra[2 * j] = fma2_bf16_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), nib_float(h0, 0x7054),
+                                     nib_float(h0, 0x7254), SA, SA2, CA);
+            ra[2 * j + 1] = fma2_bf16_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), nib_float(h0, 0x7154),
+                                         nib_float(h0, 0x7354), SA, SA2, CA);
+            rb[2 * j] = fma2_bf16_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), nib_float(h1, 0x7604),
+                                     nib_float(h1, 0x7624), SB, SB2, CB);
+            rb[2 * j + 1] = fma2_bf16_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), nib_float(h1, 0x7614),
+                                         nib_float(h1, 0x7634), SB, SB2, CB);
+        }
+    } else {
+        // 6-bit: q = lo + 16 hi, hi in 2-bit fields (word j/2, pair s = 4(j&1) + r at bits 2s and
+        // 16 + 2s; r = 0: row g cols +0/+1, 1: row g+8 cols +0/+1, 2: row g +2/+3, 3: row g+8 +2/+3)
+        const uint2 hi = *reinterpret_cast<const uint2 *>(rawt + 512 + 8 * L);
+        const float SA = 256.f * sA, SA2 = 16.f * sA, CA = -(128.f + zA) * sA;
+        const float SB = 2048.f * sB, SB2 = 16.f * sB, CB = -(2048.f + zB) * sB;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t m0 = w[j] & 0x0F0F0F0Fu, m1 = w[j] & 0xF0F0F0F0u;
+            const uint32_t hv = (j < 2) ? hi.x : hi.y;
+            const int s0 = 8 * (j & 1);
+            auto f2 = [&](int sh) { return (float)((hv >> sh) & 3u); };
+            ra[2 * j] = fma2_bf16_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), f2(s0), f2(16 + s0), SA, SA2,
+                                     CA);
+            ra[2 * j + 1] = fma2_bf16_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), f2(s0 + 4), f2(20 + s0),
+                                         SA, SA2, CA);
+            rb[2 * j] = fma2_bf16_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), f2(s0 + 2), f2(18 + s0), SB,
+                                     SB2, CB);
+            rb[2 * j + 1] = fma2_bf16_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), f2(s0 + 6), f2(22 + s0),
+                                         SB, SB2, CB);
+        }
+    }
+    const int r0 = 16 * b + g, r1 = r0 + 8;
+    *reinterpret_cast<uint4 *>(As + sw128_off(r0, 2 * t)) = make_uint4(ra[0], ra[1], ra[2], ra[3]);
+    *reinterpret_cast<uint4 *>(As + sw128_off(r0, 2 * t + 1)) = make_uint4(ra[4], ra[5], ra[6], ra[7]);
+    *reinterpret_cast<uint4 *>(As + sw128_off(r1, 2 * t)) = make_uint4(rb[0], rb[1], rb[2], rb[3]);
+    *reinterpret_cast<uint4 *>(As + sw128_off(r1, 2 * t + 1)) = make_uint4(rb[4], rb[5], rb[6], rb[7]);
+}
+
+template <bool GU>
+struct Geometry {
+    int K, KG, mtiles, nrb;
+    size_t skip_tiles;  // tiles of an expert stored before this matrix's tiles
+    __device__ explicit Geometry(const TcArgs &a) {
+        K = GU ? a.H : a.I;
+        KG = K / kGroup;
+        nrb = GU ? a.I / 8 : a.H / 16;  // 16-row blocks of the matrix
+        mtiles = (nrb + 7) / 8;
+        skip_tiles = GU ? 0 : gu_tiles(a.H, a.I);
+    }
+};
+
+// Where one dequantiser warp's packed tile of a K step lives (nullptr: the row block is past
+// the matrix, which happens in the last M tile of a down matrix with H % 128 == 64).
+struct DqStep {
+    const uint8_t *tile;
+    int bits;
+};
+template <bool GU>
+__device__ __forceinline__ DqStep dq_step(const TcArgs &a, const Geometry<GU> &G, const Unit &U, int b, int kg) {
+    DqStep d;
+    const PackedExpert pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader))[U.e];
+    d.bits = pe.bits;
+    const int rb = 8 * U.mt + b;
+    if (rb >= G.nrb) {
+        d.tile = nullptr;
+        return d;
+    }
+    d.tile = a.packed + pe.offset + (G.skip_tiles + (size_t)rb * G.KG + kg) * tile_bytes(pe.bits);
+    return d;
+}
+
+// The lane's copies of one packed tile: lo 16 B, hi 8/16 B, its row pair's scale/zero entry 8 B.
+__device__ __forceinline__ void issue_fragment(const DqStep &d, uint32_t rawt, int L) {
+    if (d.tile == nullptr) return;
+    cp_async16(rawt + 16 * L, d.tile + 16 * L);
+    if (d.bits == 8) cp_async16(rawt + 512 + 16 * L, d.tile + kLoBytes + 16 * L);
+    if (d.bits == 6) cp_async8(rawt + 512 + 8 * L, d.tile + kLoBytes + 8 * L);
+    cp_async8(rawt + 1024 + 8 * L, d.tile + kLoBytes + hi_bytes(d.bits) + 8 * (L >> 2));
+}
+
+// ------------------------------------------------------------------------------ the kernel
+template <bool GU>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs a) {
+    extern __shared__ uint8_t tc_dyn[];
+    __shared__ TcShared S;
+    const uint32_t pad = (1024u - (smem_u32(tc_dyn) & 1023u)) & 1023u;
+    uint8_t *ring = tc_dyn + pad;                               // kABStages x [A | B]
+    uint8_t *raw = ring + (size_t)kABStages * kStageBytes;      // kRawSlots x 8 packed-tile copies
+    uint8_t *staging = raw + (size_t)kRawSlots * kRawStage;     // h tile of the gate/up epilogue
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Geometry<GU> G(a);
+    const int nunits = __ldg(a.nt_start + a.E) * G.mtiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kABStages; ++s) {
+            mbar_init(smem_u32(&S.ab_full[s]), kDqWarps + kLdWarps);
+            mbar_init(smem_u32(&S.ab_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&S.acc_full[s]), 1);
+            mbar_init(smem_u32(&S.acc_empty[s]), 4);
+        }
+        mbar_init(smem_u32(&S.fin), 1);
+        S.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp < kDqWarps) {
+        // ------------------------------------------------------------ dequantisers
+        const int b = warp;
+        // issue-side cursor, kRawAhead K steps ahead of the consuming loop
+        int iu = blockIdx.x, ikg = 0;
+        Unit IU{};
+        if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
+        auto issue_next = [&](uint32_t rslot) {
+            if (iu < nunits) {
+                const DqStep d = dq_step<GU>(a, G, IU, b, ikg);
+                issue_fragment(d, smem_u32(raw + (size_t)rslot * kRawStage + b * kRawTile), lane);
+                if (++ikg == G.KG) {
+                    ikg = 0;
+                    iu += gridDim.x;
+                    if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
+                }
+            }
+            cp_async_commit();
+        };
+        for (uint32_t p = 0; p < kRawAhead; ++p) issue_next(p);
+        uint32_t j = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            const Unit U = unit_at(a, u, G.mtiles);
+            for (int kg = 0; kg < G.KG; ++kg, ++j) {
+                issue_next((j + kRawAhead) % kRawSlots);
+                cp_async_wait<kRawAhead>();
+                const int slot = j % kABStages;
+                const uint32_t use = j / kABStages;
+                if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *As = ring + (size_t)slot * kStageBytes;
+                const DqStep d = dq_step<GU>(a, G, U, b, kg);
+                const uint8_t *rawt = raw + (size_t)(j % kRawSlots) * kRawStage + b * kRawTile;
+                if (d.tile == nullptr) {
+                    // row block past the matrix: zero rows (the epilogue skips them)
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    const int g = lane >> 2, t = lane & 3;
+                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t)) = z;
+                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t + 1)) = z;
+                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t)) = z;
+                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t + 1)) = z;
+                } else if (d.bits == 4) {
+                    dequant_fragment<4>(rawt, lane, As, b);
+                } else if (d.bits == 8) {
+                    dequant_fragment<8>(rawt, lane, As, b);
+                } else {
+                    dequant_fragment<6>(rawt, lane, As, b);
+                }
+                fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[slot]));
+            }
+        }
+        cp_async_wait<0>();
+    } else if (warp < kMmaWarp) {
+        // ------------------------------------------------------------ token-row loaders
+        const int lt = threadIdx.x - kDqWarps * 32;  // 0..63
+        const int c = lt & 7, r0 = lt >> 3;          // 16-byte chunk, first row (rows r0 + 8m)
+        uint32_t j = 0, pending = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            const Unit U = unit_at(a, u, G.mtiles);
+            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's row table is no longer read
+            for (int r = lt; r < U.nn; r += kLdWarps * 32)
+                S.rows[r] = GU ? __ldg(a.pair_tok + U.base + U.n0 + r) : U.base + U.n0 + r;
+            named_sync(kBarLd, kLdWarps * 32);
+            for (int kg = 0; kg < G.KG; ++kg, ++j) {
+                const int slot = j % kABStages;
+                const uint32_t use = j / kABStages;
+                if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t Bs = smem_u32(ring + (size_t)slot * kStageBytes + kABytes);
+                for (int r = r0; r < U.nr; r += 8) {
+                    const uint32_t dst = Bs + sw128_off(r, c);
+                    if (r < U.nn) {
+                        cp_async16(dst, a.act + (size_t)S.rows[r] * G.K + kg * kGroup + c * 8);
+                    } else {
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+                    }
+                }
+                cp_async_commit();
+                if (pending == kLoaderLag) {
+                    cp_async_wait<kLoaderLag>();
+                    fence_proxy_async();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[(j - kLoaderLag) % kABStages]));
+                } else {
+                    ++pending;
+                }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async();
+        __syncwarp();
+        // the K steps still owed an arrival (their copies are complete now)
+        if (lane == 0)
+            for (uint32_t q = j - pending; q < j; ++q) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issue
+        uint32_t j = 0, i = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++i) {
+            const Unit U = unit_at(a, u, G.mtiles);
+            const uint32_t buf = i & 1u;
+            if (i >= 2 && !tc_wait(S, a, &S.acc_empty[buf], ((i >> 1) - 1) & 1u)) break;
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(kTM, U.nr);
+            const uint32_t d_tmem = tmem + buf * kMaxN;
+            for (int kg = 0; kg < G.KG; ++kg, ++j) {
+                const int slot = j % kABStages;
+                if (!tc_wait(S, a, &S.ab_full[slot], (j / kABStages) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t As = smem_u32(ring + (size_t)slot * kStageBytes);
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(d_tmem, sw128_desc(As + 32 * kk), sw128_desc(As + kABytes + 32 * kk), idesc,
+                                  (kg > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(smem_u32(&S.ab_empty[slot]));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(smem_u32(&S.acc_full[buf]));
+            __syncwarp();
+        }
+        // every MMA issued by this warp has completed once `fin` flips; waited for (bounded) even
+        // after an abort, so that TMEM is released only when no MMA still writes it
+        if (lane == 0) umma_commit(smem_u32(&S.fin));
+        __syncwarp();
+        mbar_wait(smem_u32(&S.fin), 0, a.wait_ns, a.status);
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;          // this warp may read TMEM lanes 32q .. 32q+31
+        const int row = 32 * q + lane;   // accumulator row
+        const int et = threadIdx.x - kEpiWarp0 * 32;
+        uint32_t i = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
+            const Unit U = unit_at(a, u, G.mtiles);
+            const uint32_t buf = i & 1u;
+            if (!tc_wait(S, a, &S.acc_full[buf], (i >> 1) & 1u)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kMaxN;
+            if (GU) {
+                // row 16b + g: gate (g < 8) or up (g >= 8) of intermediate column 8b + (g & 7)
+                const bool gate = (row & 8) == 0;
+                const int col = 8 * (row >> 4) + (row & 7);
+                for (int c0 = 0; c0 < U.nr; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        // the gate lane finishes token c0+jj, its up partner token c0+jj+1
+                        const float send = __uint_as_float(gate ? v[jj + 1] : v[jj]);
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+                        const float gv = gate ? __uint_as_float(v[jj]) : recv;
+                        const float uv = gate ? recv : __uint_as_float(v[jj + 1]);
+                        const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                        const int tok = c0 + jj + (gate ? 0 : 1);
+                        reinterpret_cast<uint16_t *>(staging)[tok * 64 + col] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
+                named_sync(kBarEpi, 128);
+                // coalesced copy-out: 8 threads per 128-byte token row
+                const int cc = et & 7;
+                for (int tok = et >> 3; tok < U.nn; tok += 16) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(staging + tok * 128 + cc * 16);
+                    *reinterpret_cast<uint4 *>(a.h + (size_t)(U.base + U.n0 + tok) * a.I + 64 * U.mt + cc * 8) = val;
+                }
+                named_sync(kBarEpi, 128);
+            } else {
+                const int orow = kTM * U.mt + row;
+                const bool valid = orow < a.H;
+                for (int c0 = 0; c0 < U.nr; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int tok = c0 + jj;
+                        if (valid && tok < U.nn) {
+                            const int pos = U.base + U.n0 + tok;
+                            red_add_f32(a.out_acc + (size_t)__ldg(a.pair_tok + pos) * a.H + orow,
+                                        __ldg(a.pair_w + pos) * __uint_as_float(v[jj]));
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// Exclusive prefix of the experts' N-tile counts (nt_start[E] = total), one CTA of 1024 threads.
+__global__ void ntile_scan_kernel(const int32_t *counts, int E, int32_t *nt_start) {
+    __shared__ int warp_tot[32];
+    const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    const int c = e < E ? ntile_count(counts[e]) : 0;
+    int incl = c;
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int v = warp_tot[lane];
+        int iv = v;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, iv, off);
+            if (lane >= off) iv += o;
+        }
+        warp_tot[lane] = iv - v;
+    }
+    __syncthreads();
+    if (e < E) {
+        const int excl = warp_tot[w] + incl - c;
+        nt_start[e] = excl;
+        if (e == E - 1) nt_start[E] = excl + c;
+    }
+}
+
+}  // namespace
+
+int prefill_ntile_count(int n) { return ntile_count(n); }
+
+moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int H, int I, int E, const int32_t *counts,
+                                     const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
+                                     const float *pair_w, const uint16_t *x, uint16_t *h, float *out_acc,
+                                     uint32_t *status, cudaStream_t st) {
+    const DeviceInfo *dev = device_info();
+    if (dev == nullptr) return MOE_ERR_CUDA;
+    if ((int)(kTcSmemBytes + sizeof(TcShared)) > dev->max_smem_optin) return MOE_ERR_UNSUPPORTED;
+    static bool attr_set[64] = {};
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d >= 64) return MOE_ERR_CUDA;
+    if (!attr_set[d]) {
+        if (cudaFuncSetAttribute(tc_grouped_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kTcSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc_grouped_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kTcSmemBytes) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set[d] = true;
+    }
+    ntile_scan_kernel<<<1, 1024, 0, st>>>(counts, E, nt_start);
+    TcArgs a;
+    a.packed = packed;
+    a.H = H;
+    a.I = I;
+    a.E = E;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.nt_start = nt_start;
+    a.pair_tok = pair_tok;
+    a.pair_w = pair_w;
+    a.h = h;
+    a.out_acc = out_acc;
+    a.wait_ns = wait_limit_ns();
+    a.status = status;
+    const unsigned grid = (unsigned)dev->sms;
+    a.act = x;
+    tc_grouped_kernel<true><<<grid, kTcThreads, kTcSmemBytes, st>>>(a);
+    a.act = h;
+    tc_grouped_kernel<false><<<grid, kTcThreads, kTcSmemBytes, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe
