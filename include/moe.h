@@ -111,8 +111,9 @@ enum { MOE_MODE_DECODE = 0, MOE_MODE_PREFILL = 1 };
 /* Workspace bytes needed by a forward call of the given mode and shape (0 if invalid). */
 size_t moe_workspace_bytes(int T, int H, int I, int E, int k, int mode);
 
-/* Prepares a workspace (device, 256-byte aligned) for first use: clears its control words.
- * Needed once after allocation; the forward calls keep it consistent afterwards. */
+/* Prepares a workspace (device, 256-byte aligned) for first use: clears all ws_bytes of it
+ * (asynchronously on `stream`). Needed once after allocation; the forward calls keep it
+ * consistent afterwards. */
 moe_status_t moe_workspace_init(void *workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* Decode path, 1 <= T <= 32: one persistent kernel per call (routing, gate/up, SiLU-GLU,
@@ -166,11 +167,12 @@ moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router
 
 /* Synchronises `stream`, reads the workspace's device status word and maps it to a status:
  * MOE_OK, MOE_ERR_TIMEOUT (a bounded wait expired) or MOE_ERR_DEVICE_CHECK. A non-zero word
- * is cleared together with the workspace's other control words, so the workspace is ready for
- * the next call. */
+ * is cleared; the kernels leave the rest of the workspace ready for the next call even after
+ * an expired wait. */
 moe_status_t moe_get_device_status(void *workspace, moe_stream_t stream);
 
-/* Upper bound, in nanoseconds, of every device-side wait (grid barriers, copy completion).
+/* Upper bound, in nanoseconds, of every device-side wait (exchanges between CTAs, copy
+ * completion).
  * Default 2e9 (2 s). Values are clamped to [0, 6e10]; 0 makes every wait that is not
  * already satisfied expire at once, which tests use to exercise the timeout path. */
 void moe_set_wait_limit_ns(uint64_t ns);

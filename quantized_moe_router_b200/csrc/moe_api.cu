@@ -155,7 +155,7 @@ size_t moe_workspace_bytes(int T, int H, int I, int E, int k, int mode) {
 
 moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
     if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(Control)) return MOE_ERR_INVALID_ARG;
-    return cudaMemsetAsync(ws, 0, sizeof(Control), (cudaStream_t)stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_expert_forward_decode(const uint16_t *x, const float *w_router, const float *bias,
@@ -210,9 +210,10 @@ moe_status_t moe_get_device_status(void *ws, moe_stream_t stream) {
     uint32_t st = 0;
     if (cudaMemcpy(&st, &ctl->status, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (st) {
-        // every CTA of the failed call has exited (its waits are bounded and the stream is idle),
-        // so the barrier and completion words can be reset together with the status
-        if (cudaMemset(ctl, 0, sizeof(Control)) != cudaSuccess) return MOE_ERR_CUDA;
+        // every CTA of the failed call has exited (its waits are bounded and the stream is idle);
+        // only the status word is cleared: the completion count must keep growing so that no
+        // later call can take a stale logit entry for its own
+        if (cudaMemset(&ctl->status, 0, sizeof st) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (st & kStatusTimeout) return MOE_ERR_TIMEOUT;
     if (st & kStatusCheck) return MOE_ERR_DEVICE_CHECK;

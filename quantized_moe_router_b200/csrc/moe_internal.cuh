@@ -66,27 +66,37 @@ __host__ __device__ inline size_t packed_data_start(int E) {
 // ------------------------------------------------------------------------------------------
 // Workspace: [control 256 B][regions...], every region 256-B aligned.
 struct Control {
-    uint32_t bar;      // grid barrier word (self-resetting, see grid_barrier)
-    uint32_t status;   // device status bits (kStatus*)
-    uint32_t done;     // completion counter of the decode kernel
+    unsigned long long done;   // decode CTAs that have finished a call, ever (epoch = done / CTAs)
+    uint32_t status;           // device status bits (kStatus*)
     uint32_t pad[61];
 };
+static_assert(sizeof(Control) == 256, "control block size");
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusCheck = 2u;
+constexpr int kDecodeMaxP = 256;   // decode limit on T*k
 
+// Decode workspace, fixed regions first so that one workspace can serve decode calls of any
+// shape: logits, kMaxT x kMaxE 8-byte words {fp32 logit bits (low word), call tag (high word)}
+// (call t writes entry t * E + e); h_ready, finished gate/up row blocks per selected expert;
+// out_acc, fp32 [T x H] (up to kMaxT x kDecodeMaxH); then h_hi / h_lo, bf16 h of every
+// (token, slot) pair [T*k x I]. h_ready and out_acc are zero between calls: the last CTA of
+// every call clears what the call used.
+constexpr int kDecodeMaxH = 8192;
 struct DecodeWs {
-    size_t logits, h_hi, h_lo, hsum, out_acc, total;
+    size_t logits, h_ready, out_acc, h_hi, h_lo, total;
 };
 inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
+    (void)H;
+    (void)E;
     DecodeWs w;
     size_t o = 256;
     auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
     const size_t P = (size_t)T * k;
-    w.logits = take((size_t)T * E * 4);
+    w.logits = take((size_t)kMaxT * kMaxE * 8);
+    w.h_ready = take((size_t)kDecodeMaxP * 4);
+    w.out_acc = take((size_t)kMaxT * kDecodeMaxH * 4);
     w.h_hi = take(P * I * 2);
     w.h_lo = take(P * I * 2);
-    w.hsum = take(P * (I / kGroup) * 4);
-    w.out_acc = take((size_t)T * H * 4);
     w.total = o;
     return w;
 }
@@ -187,26 +197,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
 __device__ __forceinline__ void red_add_f32(float *p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
-// Grid-wide barrier over `nblocks` CTAs, called by ONE thread per CTA. The word's top bit flips
-// once per barrier (CTA 0 adds 2^31 - (n-1), the others 1), so it needs no reset between uses.
-// Bounded: returns false and sets the status word if the flip is not seen within limit_ns.
-__device__ __forceinline__ bool grid_barrier(uint32_t *bar, uint32_t nblocks, bool first_block,
-                                             uint64_t limit_ns, uint32_t *status) {
-    const uint32_t add = first_block ? (0x80000000u - (nblocks - 1u)) : 1u;
-    __threadfence();
-    const uint32_t old = atom_add_acq_rel(bar, add);
-    if (((ld_acquire(bar) ^ old) & 0x80000000u) != 0) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        if (((ld_acquire(bar) ^ old) & 0x80000000u) != 0) return true;
-        if (global_timer() - t0 > limit_ns) {
-            atomicOr(status, kStatusTimeout);
-            return false;
-        }
-        __nanosleep(32);
-    }
-}
-
 // bf16x2 operand from a code word: (word >> shift) & mask | bf16(128) in both halves, i.e.
 // the bf16 pair {128 + field_lo, 128 + field_hi}; exact for fields < 128.
 template <uint32_t MASK>

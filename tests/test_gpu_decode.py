@@ -113,3 +113,17 @@ def test_decode_graph_stack_matches_oracle():
         for l in range(L):
             check_block(o, synth.hidden(w, step, l), layers[l].wr_np, None, layers[l].expert_fn, w.E, w.H, w.I,
                         w.k, bf16_f64(stack.out[l]), stack.idx[l].cpu().numpy(), stack.wts[l].cpu().numpy())
+
+
+def test_decode_workspace_shared_across_shapes():
+    """One workspace, sized for the largest call, serves decode calls of different T, E and k in
+    any order (its fixed regions keep the call tags, accumulators and counters consistent)."""
+    rng = np.random.default_rng(11)
+    H, I = 128, 64
+    la = hand_layer(rng, 8, H, I, [4])
+    lb = hand_layer(rng, 20, H, I, [6, 4])
+    ws = qm.workspace(32, H, I, 20, 5, qm.MODE_DECODE)
+    for layer, E, k, T in ((la, 8, 2, 3), (lb, 20, 4, 11), (la, 8, 2, 1), (lb, 20, 5, 32), (la, 8, 1, 7)):
+        x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
+        out, idx, w = decode_call(layer, x, I, E, k, ws)
+        check_block(oracle.get(), x, layer.wr_np, layer.bias_np, layer.expert_fn, E, H, I, k, out, idx, w)
