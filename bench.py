@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "decode_t1_l48_h2048_e256_k8_i512_int4"
+PREFILL_WORKLOAD = "prefill_t4096_l8_h2048_e256_k8_i512_int4"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -43,6 +44,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement of the default run")
     ap.add_argument("--layers", type=int, default=0,
                     help="stack only this many layers of the workload (smaller case for profiling)")
     return ap.parse_args()
@@ -261,7 +263,24 @@ def run_ours(args, w):
     import synth.device as sd
     from quantized_moe_router_b200.runner import DecodeStack
     rank, world, local = dist_setup(args.gpus)
-    assert w.mode == "decode", "bench.py times the decode workloads"
+    if w.mode == "prefill":
+        res = run_prefill(args, w, world, rank)
+        line = {"metric": res.pop("metric"), "value": res.pop("value"), "unit": res.pop("unit"), "n_gpus": world,
+                "steps": res.pop("steps"), "warmup": max(args.warmup, 3), "ms_per_step": res.pop("ms_per_step"),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": res.pop("workload"), "tokens_per_step": w.T, "layers": w.layers, "H": w.H,
+                           "E": w.E, "k": w.k, "I": w.I, "weights": f"int{w.bits} group-64 affine",
+                           "l2": "no flush: each layer streams ~453 MB of expert weights (> 126 MB L2)",
+                           "parallelism": f"replicas x{world}"},
+                "gpu_launches": res["steps_launches"], **{k: v for k, v in res.items() if k != "steps_launches"}}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    assert w.mode == "decode", "bench.py times the decode and prefill workloads"
     layers, bits = build_layers(w)
     stack = DecodeStack(layers, w.T, w.H, w.I, w.E, w.k)
     nsteps = args.warmup + args.steps
@@ -373,6 +392,13 @@ def run_ours(args, w):
     }
     if e2e:
         line["e2e"] = e2e
+    if not args.no_prefill:
+        del layers, stack, xs
+        torch.cuda.empty_cache()
+        import synth
+        pre = run_prefill(args, synth.WORKLOADS[PREFILL_WORKLOAD], world, rank)
+        pre["gpu_launches"] = pre.pop("steps_launches")
+        line["prefill"] = pre
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t, tokens, threads = oracle_decode_sample(w, 1, w.layers)
         line["cpu_baseline"] = {"value": tokens / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -382,6 +408,99 @@ def run_ours(args, w):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------ prefill
+
+def prefill_flops(w):
+    """Expert-GEMM flops of one prefill layer: gate, up and down for every (token, expert) pair."""
+    return 2.0 * w.T * w.k * 3 * w.I * w.H
+
+
+def oracle_prefill_sample(w, ntok):
+    """Times the fp64 oracle on the first `ntok` tokens of layer 0 of prefill workload w.
+    Returns (seconds, tokens, threads)."""
+    import oracle
+    import synth
+    o = oracle.get()
+    wr = synth.router_weights(w, 0)
+    x = synth.hidden(w, 0, 0)[:ntok]
+    bits = synth.expert_bits(w, 0)
+    t0 = time.perf_counter()
+    logits = o.router_logits(x, wr, None)
+    idx, ww = o.topk(logits, w.k)
+    t_route = time.perf_counter() - t0
+    experts = [None] * w.E
+    for e in np.unique(idx):
+        experts[int(e)] = synth.expert_tensors(w, 0, int(e), int(bits[int(e)]))
+    t0 = time.perf_counter()
+    o.combine(x, experts, w.H, w.I, idx, ww)
+    return t_route + time.perf_counter() - t0, ntok, o.threads()
+
+
+def run_prefill(args, w, world, rank):
+    """One step = all w.T tokens through w.layers prefill layers (route + bucket + grouped GEMMs +
+    combine per layer), fresh x per layer. Returns the measurement as a dict."""
+    import torch
+    import synth.device as sd
+    import quantized_moe_router_b200 as qm
+    layers, _ = build_layers(w)
+    xs = torch.empty((w.layers, w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    for l in range(w.layers):
+        sd.hidden(w, 0, l, out=xs[l])
+    ws = qm.workspace(w.T, w.H, w.I, w.E, w.k, qm.MODE_PREFILL)
+    out = torch.empty((w.layers, w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for l, lw in enumerate(layers):
+            qm.prefill_route(xs[l], lw.wr, lw.bias, w.I, w.E, w.k, ws)
+            if ev:
+                ev[l][0].record(st)
+            qm.prefill_experts(xs[l], lw.packed, w.I, w.E, w.k, ws, out=out[l])
+            if ev:
+                ev[l][1].record(st)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    nsteps = max(1, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(w.layers)]
+           for _ in range(nsteps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(st)
+        for i in range(nsteps):
+            step(evs[i])
+        e1.record(st)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    gemm_ms = float(np.mean([ev[0].elapsed_time(ev[1]) for evl in evs for ev in evl]))
+    assert qm.device_status(ws) == qm.MOE_OK
+    _, bf16, peak_src = measured_peaks()
+    achieved = prefill_flops(w) / (gemm_ms * 1e-3) / 1e12
+    res = {
+        "workload": w.name, "metric": "prefill tokens/s (MoE expert block, all layers)",
+        "value": world * w.T * nsteps / (ms * 1e-3), "unit": "tokens/s", "steps": nsteps,
+        "ms_per_step": ms / nsteps, "ms_per_layer": ms / nsteps / w.layers,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                     "frac": achieved / bf16, "traffic": None, "peak_source": peak_src,
+                     "flops_per_launch": prefill_flops(w),
+                     "kernel": "expert phase (moe_prefill_experts: grouped gate/up + down GEMMs, combine)",
+                     "kernel_ms_per_launch": gemm_ms},
+        "clocks": clk.summary(),
+        # route, 3 bucketing kernels, N-tile scan, gate/up GEMM, down GEMM, bf16 conversion per layer
+        "steps_launches": nsteps * w.layers * 8,
+    }
+    del layers
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, tokens, threads = oracle_prefill_sample(w, 16)
+        res["cpu_baseline"] = {"value": tokens / (t * w.layers), "unit": "tokens/s", "cores": threads,
+                               "kind": "oracle",
+                               "sample": f"16 tokens of layer 0 (fp64 oracle), scaled to {w.layers} layers"}
+    return res
 
 
 def main():

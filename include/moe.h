@@ -165,6 +165,21 @@ moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router
                                         float *w_out, void *workspace, size_t ws_bytes,
                                         moe_stream_t stream);
 
+/* The two halves of moe_expert_forward_prefill, for callers that schedule them separately (for
+ * example to overlap the routing of one layer with other work, or to time the expert GEMMs).
+ * moe_prefill_route: routing (as moe_route_topk) and the bucketing of the T*k pairs per expert
+ * into the PREFILL workspace; idx_out / w_out (device) may be NULL. moe_prefill_experts: the
+ * grouped gate/up and down GEMMs and the combine over the buckets that the last
+ * moe_prefill_route left in the same workspace (same T, H, I, E, k), writing out (device)
+ * bf16 [T x H]; x must be the same hidden states. Arguments and limits as for
+ * moe_expert_forward_prefill. */
+moe_status_t moe_prefill_route(const uint16_t *x, const float *w_router, const float *bias, int T,
+                               int H, int I, int E, int k, int32_t *idx_out, float *w_out,
+                               void *workspace, size_t ws_bytes, moe_stream_t stream);
+moe_status_t moe_prefill_experts(const uint16_t *x, const void *packed, int T, int H, int I,
+                                 int E, int k, uint16_t *out, void *workspace, size_t ws_bytes,
+                                 moe_stream_t stream);
+
 /* Synchronises `stream`, reads the workspace's device status word and maps it to a status:
  * MOE_OK, MOE_ERR_TIMEOUT (a bounded wait expired) or MOE_ERR_DEVICE_CHECK. A non-zero word
  * is cleared; the kernels leave the rest of the workspace ready for the next call even after

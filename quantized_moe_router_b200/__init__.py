@@ -32,6 +32,8 @@ SIGNATURES = {
     "moe_expert_forward_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_forward_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_forward_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_prefill_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "moe_prefill_experts": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_set_wait_limit_ns": (None, [_u64]),
 }
@@ -168,6 +170,23 @@ def forward_prefill(x, w_router, bias, packed, I, E, k, ws, out=None, idx_out=No
     """Prefill-path expert block (any T): returns out [T x H] bf16."""
     return _forward(lib().moe_expert_forward_prefill, "moe_expert_forward_prefill", x, w_router, bias, packed,
                     I, E, k, ws, out, idx_out, w_out, stream)
+
+
+def prefill_route(x, w_router, bias, I, E, k, ws, idx_out=None, w_out=None, stream=None):
+    """Routing and bucketing of the prefill path into the workspace `ws`."""
+    T, H = x.shape
+    _check(lib().moe_prefill_route(_p(x), _p(w_router), _p(bias), T, H, I, E, k, _p(idx_out), _p(w_out), _p(ws),
+                                   ws.numel(), _stream(stream)), "moe_prefill_route")
+
+
+def prefill_experts(x, packed, I, E, k, ws, out=None, stream=None):
+    """Expert GEMMs and combine over the buckets of the last prefill_route on `ws`; returns out."""
+    T, H = x.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_prefill_experts(_p(x), _p(packed), T, H, I, E, k, _p(out), _p(ws), ws.numel(), _stream(stream)),
+           "moe_prefill_experts")
+    return out
 
 
 def forward_decode_noalloc(x, w_router, bias, packed, I, E, k, out=None, idx_out=None, w_out=None, stream=None):

@@ -16,6 +16,10 @@ moe_status_t launch_prefill(const uint16_t *x, const float *wr, const float *bia
                             cudaStream_t st);
 moe_status_t launch_route(const uint16_t *x, const float *wr, const float *bias, int T, int H, int E, int k,
                           int32_t *idx_out, float *w_out, cudaStream_t st);
+moe_status_t launch_prefill_route(const uint16_t *x, const float *wr, const float *bias, int T, int H, int I, int E,
+                                  int k, int32_t *idx_out, float *w_out, void *ws, cudaStream_t st);
+moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T, int H, int I, int E, int k,
+                                    uint16_t *out, void *ws, cudaStream_t st);
 moe_status_t launch_pack(const moe_expert_src_t *src, int E, int H, int I, void *packed, cudaStream_t st);
 size_t packed_layer_bytes(int E, int H, int I, const int32_t *bits);
 
@@ -201,6 +205,31 @@ moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router
                                     MOE_MODE_PREFILL);
     if (s != MOE_OK) return s;
     return launch_prefill(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, ws, (cudaStream_t)stream);
+}
+
+moe_status_t moe_prefill_route(const uint16_t *x, const float *w_router, const float *bias, int T, int H, int I,
+                               int E, int k, int32_t *idx_out, float *w_out, void *ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+    if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
+    if (!x || !w_router || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
+    if ((idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_workspace_bytes(T, H, I, E, k, MOE_MODE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = check_device();
+    if (d != MOE_OK) return d;
+    return launch_prefill_route(x, w_router, bias, T, H, I, E, k, idx_out, w_out, ws, (cudaStream_t)stream);
+}
+
+moe_status_t moe_prefill_experts(const uint16_t *x, const void *packed, int T, int H, int I, int E, int k,
+                                 uint16_t *out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
+    if (!x || !out || !ws || !packed_ok(packed)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(ws, 256) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_workspace_bytes(T, H, I, E, k, MOE_MODE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = check_device();
+    if (d != MOE_OK) return d;
+    return launch_prefill_experts(x, packed, T, H, I, E, k, out, ws, (cudaStream_t)stream);
 }
 
 moe_status_t moe_get_device_status(void *ws, moe_stream_t stream) {

@@ -108,9 +108,10 @@ __global__ void convert_kernel(const float *acc, uint16_t *out, size_t n) {
 
 }  // namespace
 
-moe_status_t launch_prefill(const uint16_t *x, const float *wr, const float *bias, const void *packed, int T, int H,
-                            int I, int E, int k, uint16_t *out, int32_t *idx_out, float *w_out, void *ws,
-                            cudaStream_t st) {
+// Routing and bucketing: idx / w of every (token, slot) pair, the experts' counts and offsets and
+// the pair lists (token, weight) in bucket order, all in the workspace.
+moe_status_t launch_prefill_route(const uint16_t *x, const float *wr, const float *bias, int T, int H, int I, int E,
+                                  int k, int32_t *idx_out, float *w_out, void *ws, cudaStream_t st) {
     const PrefillWs L = prefill_ws_layout(T, H, I, E, k);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     int32_t *idx = reinterpret_cast<int32_t *>(w8 + L.idx);
@@ -120,26 +121,42 @@ moe_status_t launch_prefill(const uint16_t *x, const float *wr, const float *bia
     int32_t *bh = reinterpret_cast<int32_t *>(w8 + L.blockhist);
     int32_t *ptok = reinterpret_cast<int32_t *>(w8 + L.pair_tok);
     float *pw = reinterpret_cast<float *>(w8 + L.pair_w);
-    float *oacc = reinterpret_cast<float *>(w8 + L.out_acc);
     const size_t P = (size_t)T * k;
     moe_status_t s = launch_route(x, wr, bias, T, H, E, k, idx, wt, st);
     if (s != MOE_OK) return s;
     if (idx_out && cudaMemcpyAsync(idx_out, idx, P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (w_out && cudaMemcpyAsync(w_out, wt, P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaMemsetAsync(oacc, 0, (size_t)T * H * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     bucket_hist_kernel<<<L.nblk, 256, E * sizeof(int), st>>>(idx, T, k, E, bh);
     bucket_scan_kernel<<<1, 1024, 0, st>>>(bh, L.nblk, E, counts, offsets);
     bucket_scatter_kernel<<<L.nblk, 32, E * sizeof(int), st>>>(idx, wt, T, k, E, bh, ptok, pw);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
-    s = launch_tc_prefill_gemms(static_cast<const uint8_t *>(packed), H, I, E, counts, offsets,
-                                reinterpret_cast<int32_t *>(w8 + L.nt_start), ptok, pw, x,
-                                reinterpret_cast<uint16_t *>(w8 + L.h), oacc,
-                                &reinterpret_cast<Control *>(w8)->status, st);
+// The expert GEMMs over the buckets that launch_prefill_route left in the workspace, and the
+// conversion of the fp32 accumulator to bf16.
+moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T, int H, int I, int E, int k,
+                                    uint16_t *out, void *ws, cudaStream_t st) {
+    const PrefillWs L = prefill_ws_layout(T, H, I, E, k);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    float *oacc = reinterpret_cast<float *>(w8 + L.out_acc);
+    if (cudaMemsetAsync(oacc, 0, (size_t)T * H * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status_t s = launch_tc_prefill_gemms(
+        static_cast<const uint8_t *>(packed), H, I, E, reinterpret_cast<const int32_t *>(w8 + L.counts),
+        reinterpret_cast<const int32_t *>(w8 + L.offsets), reinterpret_cast<int32_t *>(w8 + L.nt_start),
+        reinterpret_cast<const int32_t *>(w8 + L.pair_tok), reinterpret_cast<const float *>(w8 + L.pair_w), x,
+        reinterpret_cast<uint16_t *>(w8 + L.h), oacc, &reinterpret_cast<Control *>(w8)->status, st);
     if (s != MOE_OK) return s;
     const size_t n = (size_t)T * H;
     convert_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 256, 0, st>>>(oacc, out, n);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t launch_prefill(const uint16_t *x, const float *wr, const float *bias, const void *packed, int T, int H,
+                            int I, int E, int k, uint16_t *out, int32_t *idx_out, float *w_out, void *ws,
+                            cudaStream_t st) {
+    const moe_status_t s = launch_prefill_route(x, wr, bias, T, H, I, E, k, idx_out, w_out, ws, st);
+    if (s != MOE_OK) return s;
+    return launch_prefill_experts(x, packed, T, H, I, E, k, out, ws, st);
 }
 
 }  // namespace moe
