@@ -101,8 +101,12 @@ inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
     return w;
 }
 
+// Prefill workspace. x16: the hidden states as fp16 scaled by 2^-xexp[t] per token; h: fp16 h of
+// every (token, expert) pair in bucket order, scaled by 2^-hexp per 16-column block; fexp: the
+// largest hexp of each pair; nt_start: N-tile prefix of the experts ([E] = total, [E+1] = the
+// largest N tile, rows rounded to 16).
 struct PrefillWs {
-    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, h, out_acc, total;
+    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, x16, xexp, h, hexp, fexp, out_acc, total;
     int nblk;  // token blocks of the stable scatter
 };
 constexpr int kScatterTokens = 64;
@@ -119,8 +123,12 @@ inline PrefillWs prefill_ws_layout(int T, int H, int I, int E, int k) {
     w.blockhist = take((size_t)w.nblk * E * 4);
     w.pair_tok = take(P * 4);
     w.pair_w = take(P * 4);
-    w.nt_start = take((size_t)(E + 1) * 4);
-    w.h = take(P * I * 2);                 // bf16 h of every (token, expert) pair, bucket order
+    w.nt_start = take((size_t)(E + 2) * 4);
+    w.x16 = take((size_t)T * H * 2);
+    w.xexp = take((size_t)T * 4);
+    w.h = take(P * I * 2);
+    w.hexp = take(P * (I / 16));
+    w.fexp = take(P * 4);
     w.out_acc = take((size_t)T * H * 4);
     w.total = o;
     return w;

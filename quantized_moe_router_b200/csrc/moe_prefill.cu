@@ -14,10 +14,11 @@ namespace moe {
 
 moe_status_t launch_route(const uint16_t *x, const float *wr, const float *bias, int T, int H, int E, int k,
                           int32_t *idx_out, float *w_out, cudaStream_t st);
-moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int H, int I, int E, const int32_t *counts,
+moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I, int E, int k, const int32_t *counts,
                                      const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
-                                     const float *pair_w, const uint16_t *x, uint16_t *h, float *out_acc,
-                                     uint32_t *status, cudaStream_t st);
+                                     const float *pair_w, const uint16_t *x, uint16_t *x16, int32_t *xexp,
+                                     uint16_t *h16, int8_t *hexp, int32_t *fexp, float *out_acc, uint32_t *status,
+                                     cudaStream_t st);
 
 namespace {
 
@@ -141,10 +142,12 @@ moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T
     float *oacc = reinterpret_cast<float *>(w8 + L.out_acc);
     if (cudaMemsetAsync(oacc, 0, (size_t)T * H * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     moe_status_t s = launch_tc_prefill_gemms(
-        static_cast<const uint8_t *>(packed), H, I, E, reinterpret_cast<const int32_t *>(w8 + L.counts),
+        static_cast<const uint8_t *>(packed), T, H, I, E, k, reinterpret_cast<const int32_t *>(w8 + L.counts),
         reinterpret_cast<const int32_t *>(w8 + L.offsets), reinterpret_cast<int32_t *>(w8 + L.nt_start),
         reinterpret_cast<const int32_t *>(w8 + L.pair_tok), reinterpret_cast<const float *>(w8 + L.pair_w), x,
-        reinterpret_cast<uint16_t *>(w8 + L.h), oacc, &reinterpret_cast<Control *>(w8)->status, st);
+        reinterpret_cast<uint16_t *>(w8 + L.x16), reinterpret_cast<int32_t *>(w8 + L.xexp),
+        reinterpret_cast<uint16_t *>(w8 + L.h), reinterpret_cast<int8_t *>(w8 + L.hexp),
+        reinterpret_cast<int32_t *>(w8 + L.fexp), oacc, &reinterpret_cast<Control *>(w8)->status, st);
     if (s != MOE_OK) return s;
     const size_t n = (size_t)T * H;
     convert_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 256, 0, st>>>(oacc, out, n);

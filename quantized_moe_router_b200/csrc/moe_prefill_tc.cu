@@ -3,20 +3,25 @@
 // In prefill the expert block is a dense contraction: after bucketing, expert e multiplies its
 // n_e tokens (about 128 at 4096 tokens, 256 experts, top-8) by its dequantised weights, and a
 // long prompt touches nearly every expert of a layer (the pages "Qwen-tin" and
-// "--moe-direct-io"). Both GEMMs run in one persistent kernel each (one CTA per SM) whose work
+// "--moe-direct-io"). Both GEMMs run as one persistent kernel each (one CTA per SM) whose work
 // unit is (expert, 128 weight rows, up to 256 of the expert's tokens):
-//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, copy their
-//     lane fragments from HBM into a small ring with cp.async (3 K steps ahead), then write
-//     w = (q - z) * s as bf16 into a 128-byte-swizzled K-major shared tile A [128 x 64];
-//   * 2 loader warps gather the unit's token rows (x rows for gate/up, h rows for down) into a
-//     swizzled tile B [N x 64] with cp.async;
-//   * 1 warp issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128, N = tokens rounded up
+//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, copy their lane
+//     fragments from HBM into a ring of raw slots with cp.async (completion tracked per slot by
+//     an mbarrier, so the look-ahead depth is whatever shared memory allows, up to 12 K steps),
+//     then write w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile A [128 x 64];
+//   * 4 loader warps copy the unit's token rows into a swizzled tile B [N x 64] with cp.async:
+//     gate/up reads x16 (the hidden states as fp16, scaled per token by a power of two so that
+//     no value overflows), down reads h16 and rescales each 16-column block in place to the
+//     pair's common exponent;
+//   * 1 warp issues tcgen05.mma (kind::f16, fp16 x fp16 -> fp32, M = 128, N = tokens rounded up
 //     to 16) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
 //     each ring stage with tcgen05.commit;
 //   * 4 epilogue warps read the other accumulator with tcgen05.ld while the next unit runs:
-//     gate/up pairs each gate row with its up row (8 TMEM lanes apart), applies SiLU-GLU and
-//     stores h (bf16, bucket order) through a shared staging tile; down adds w * y into the
-//     fp32 output accumulator with red.add.
+//     gate/up undoes the token scale, pairs each gate row with its up row (8 TMEM lanes apart),
+//     applies SiLU-GLU and stores h as fp16 with one power-of-two exponent per 16 columns; down
+//     undoes the pair's exponent and adds w * y into the fp32 output accumulator with red.add.
+// fp16 operands (11-bit significands) keep the block within its error bound where bf16
+// operands (8-bit) would not; every scaling is by a power of two and exact.
 // Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
 #include "moe_internal.cuh"
 
@@ -27,33 +32,33 @@ namespace {
 constexpr int kTM = 128;                          // weight rows per unit (UMMA M)
 constexpr int kMaxN = 256;                        // tokens per unit (UMMA N limit)
 constexpr int kABStages = 3;
-constexpr int kABytes = kTM * 128;                // 128 rows x 64 bf16
-constexpr int kBBytes = kMaxN * 128;              // 256 rows x 64 bf16
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kRawAhead = 3;                      // K steps of packed tiles in flight per warp
-constexpr int kRawSlots = kRawAhead + 1;
-constexpr int kRawTile = 1280;                    // lane copies: lo 512 | hi 512 | scale/zero 256
-constexpr int kRawStage = 8 * kRawTile;
-constexpr int kStagingBytes = kMaxN * 128;        // h staging: 256 tokens x 64 bf16
-constexpr int kDqWarps = 8, kLdWarps = 2;
+constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
+constexpr int kRawTile = 1280;                    // lane copies of one tile: lo 512 | hi 512 | scale/zero 256
+constexpr int kRawStep = 8 * kRawTile;            // one K step of the 8 dequantiser warps
+constexpr int kMaxRaw = 12;                       // raw ring slots (K steps) at most
+constexpr int kDqWarps = 8, kLdWarps = 4;
 constexpr int kMmaWarp = kDqWarps + kLdWarps;
 constexpr int kEpiWarp0 = kMmaWarp + 1;
 constexpr int kTcWarps = kEpiWarp0 + 4;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr uint32_t kTmemCols = 2 * kMaxN;         // two accumulators of 256 fp32 columns
-constexpr int kLoaderLag = 1;                     // K steps a loader keeps in flight before arriving
+constexpr int kLoaderLag = kABStages - 1;         // K steps a loader keeps in flight before arriving
 constexpr int kBarEpi = 1, kBarLd = 2;            // named barriers (0 is __syncthreads)
-constexpr size_t kTcSmemBytes =
-    (size_t)kABStages * kStageBytes + (size_t)kRawSlots * kRawStage + kStagingBytes + 1024;
+constexpr int kMaxSub = 64;                       // 16-column blocks of a down row (I <= 1024)
 
 struct TcArgs {
     const uint8_t *packed;
     int H, I, E;
     const int32_t *counts, *offsets, *nt_start, *pair_tok;
     const float *pair_w;
-    const uint16_t *act;  // gate/up: x [T x H]; down: h [pairs x I] in bucket order
-    uint16_t *h;          // gate/up output: h [pairs x I] bf16
-    float *out_acc;       // down output: [T x H] fp32
+    const uint16_t *act;   // gate/up: x16 [T x H]; down: h16 [pairs x I] in bucket order
+    const int32_t *xexp;   // gate/up: per-token exponent of x16
+    const int8_t *hexp;    // down: per-pair, per-16-column exponents of h16
+    const int32_t *fexp;   // down: per-pair largest hexp
+    uint16_t *h;           // gate/up output: h16
+    int8_t *hexp_out;      // gate/up output: exponents of h16
+    float *out_acc;        // down output: [T x H] fp32
+    int smem_bytes;        // dynamic shared memory of the launch
     uint64_t wait_ns;
     uint32_t *status;
 };
@@ -64,13 +69,15 @@ struct TcShared {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t fin;
+    uint64_t rawbar[kDqWarps][kMaxRaw];
     uint32_t tmem_base;
     volatile int abort;
-    int rows[kMaxN];  // loaders: activation row of each token of the current unit
+    int rows[kMaxN];          // loaders: activation row of each token of the current unit
+    int rowexp[kMaxN];        // loaders (down): the row's common exponent
 };
 
 // ------------------------------------------------------------------------------ work units
-// An expert's n tokens are cut into ceil(n / tile) N tiles of at most 256 (sizes rounded to 16).
+// An expert's n tokens are cut into ceil(n / 256) N tiles of equal size (rounded up to 16).
 __host__ __device__ inline int ntile_size(int n) {
     const int c = (n + kMaxN - 1) / kMaxN;
     return c == 0 ? 0 : (((n + c - 1) / c + 15) & ~15);
@@ -116,12 +123,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     d |= (uint64_t)2 << 61;              // SWIZZLE_128B
     return d;
 }
-__device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
-    // D fp32, A and B bf16, both K-major, N >> 3 at bit 17, M >> 4 at bit 24
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_f16_f32(int M, int N) {
+    // D fp32 (bits 4-5 = 1), A and B fp16 (format 0), both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
@@ -147,6 +154,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 }
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on `bar` once every cp.async this thread issued so far has completed (the barrier's
+// expected count includes this arrival)
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -174,19 +186,29 @@ __device__ __forceinline__ bool tc_wait(TcShared &S, const TcArgs &a, uint64_t *
 // byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled K-major tile
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// 2^e as fp32 for |e| <= 126
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+// the exponent f with 2^14 <= max|v| * 2^-f < 2^15 (0 when max|v| is 0), from the bits of max|v|
+__device__ __forceinline__ int scale_exp(float vmax) {
+    const uint32_t b = __float_as_uint(vmax);
+    if (b == 0u) return 0;
+    const int e = (int)((b >> 23) & 0xFF) - 127;
+    return max(-100, min(100, e - 14));
+}
+
 // ------------------------------------------------------------------------------ dequantisation
 // A code nibble becomes an fp32 value by byte placement (prmt) under a fixed exponent byte:
 //   low nibble q of byte x  -> 0x3F0q0000 = 0.5 + q/256   (row g of the lane fragment)
 //   high nibble q of byte x -> 0x3F80(q<<4)00 = 1 + q/2048 (row g+8)
 // so w = (q - z) * s = f * S + C with S = 256 s (2048 s) and C = -(128 + z) s (-(2048 + z) s).
-// C is rounded once to fp32 (|error| <= 2^-24 |C|, far below the bf16 rounding of w).
+// C is rounded once to fp32 (|error| <= 2^-24 |C|, far below the fp16 rounding of w).
 __device__ __forceinline__ float nib_float(uint32_t m, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(m), "r"(0x3F800000u), "r"(sel));
     return __uint_as_float(r);
 }
-// (x0 * S + C, x1 * S + C) with one packed fp32x2 FMA, rounded to a bf16 pair (x0 in the low half)
-__device__ __forceinline__ uint32_t fma2_bf16(float x0, float x1, float S, float C) {
+// (x0 * S + C, x1 * S + C) with one packed fp32x2 FMA, rounded to an fp16 pair (x0 in the low half)
+__device__ __forceinline__ uint32_t fma2_h(float x0, float x1, float S, float C) {
     float r0, r1;
     asm("{ .reg .b64 a, b, c, d;\n\t"
         "mov.b64 a, {%2, %3}; mov.b64 b, {%4, %4}; mov.b64 c, {%5, %5};\n\t"
@@ -194,21 +216,20 @@ __device__ __forceinline__ uint32_t fma2_bf16(float x0, float x1, float S, float
         "mov.b64 {%0, %1}, d; }"
         : "=f"(r0), "=f"(r1)
         : "f"(x0), "f"(x1), "f"(S), "f"(C));
-    const __nv_bfloat162 v = __floats2bfloat162_rn(r0, r1);
+    const __half2 v = __floats2half2_rn(r0, r1);
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 // x * S + y * S2 + C for two elements (6/8-bit codes: the low and the high code plane)
-__device__ __forceinline__ uint32_t fma2_bf16_hi(float x0, float x1, float y0, float y1, float S, float S2,
-                                                 float C) {
+__device__ __forceinline__ uint32_t fma2_h_hi(float x0, float x1, float y0, float y1, float S, float S2, float C) {
     float t0 = fmaf(x0, S, C), t1 = fmaf(x1, S, C);
     t0 = fmaf(y0, S2, t0);
     t1 = fmaf(y1, S2, t1);
-    const __nv_bfloat162 v = __floats2bfloat162_rn(t0, t1);
+    const __half2 v = __floats2half2_rn(t0, t1);
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile, from the
-// lane's fragment copies in `rawt`, stored into the swizzled A tile rows 16b+g and 16b+g+8.
+// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile, from the lane's
+// fragment copies in `rawt`, stored as fp16 into the swizzled A tile rows 16b+g and 16b+g+8.
 // Word j of the lo plane holds columns 16t+4j+{0,1,2,3} in bytes {0,2,1,3}: row g in the low
 // nibbles, row g+8 in the high nibbles.
 template <int BITS>
@@ -225,10 +246,10 @@ __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uin
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t m0 = w[j] & 0x0F0F0F0Fu, m1 = w[j] & 0xF0F0F0F0u;
-            ra[2 * j] = fma2_bf16(nib_float(m0, 0x7054), nib_float(m0, 0x7254), SA, CA);
-            ra[2 * j + 1] = fma2_bf16(nib_float(m0, 0x7154), nib_float(m0, 0x7354), SA, CA);
-            rb[2 * j] = fma2_bf16(nib_float(m1, 0x7604), nib_float(m1, 0x7624), SB, CB);
-            rb[2 * j + 1] = fma2_bf16(nib_float(m1, 0x7614), nib_float(m1, 0x7634), SB, CB);
+            ra[2 * j] = fma2_h(nib_float(m0, 0x7054), nib_float(m0, 0x7254), SA, CA);
+            ra[2 * j + 1] = fma2_h(nib_float(m0, 0x7154), nib_float(m0, 0x7354), SA, CA);
+            rb[2 * j] = fma2_h(nib_float(m1, 0x7604), nib_float(m1, 0x7624), SB, CB);
+            rb[2 * j + 1] = fma2_h(nib_float(m1, 0x7614), nib_float(m1, 0x7634), SB, CB);
         }
     } else if (BITS == 8) {
         // q = lo + 16 hi, the hi plane in the same nibble arrangement
@@ -240,14 +261,14 @@ __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uin
         for (int j = 0; j < 4; ++j) {
             const uint32_t m0 = w[j] & 0x0F0F0F0Fu, m1 = w[j] & 0xF0F0F0F0u;
             const uint32_t h0 = v[j] & 0x0F0F0F0Fu, h1 = v[j] & 0xF0F0F0F0u;
-            ra[2 * j] = fma2_bf16_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), nib_float(h0, 0x7054),
-                                     nib_float(h0, 0x7254), SA, SA2, CA);
-            ra[2 * j + 1] = fma2_bf16_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), nib_float(h0, 0x7154),
-                                         nib_float(h0, 0x7354), SA, SA2, CA);
-            rb[2 * j] = fma2_bf16_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), nib_float(h1, 0x7604),
-                                     nib_float(h1, 0x7624), SB, SB2, CB);
-            rb[2 * j + 1] = fma2_bf16_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), nib_float(h1, 0x7614),
-                                         nib_float(h1, 0x7634), SB, SB2, CB);
+            ra[2 * j] = fma2_h_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), nib_float(h0, 0x7054),
+                                  nib_float(h0, 0x7254), SA, SA2, CA);
+            ra[2 * j + 1] = fma2_h_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), nib_float(h0, 0x7154),
+                                      nib_float(h0, 0x7354), SA, SA2, CA);
+            rb[2 * j] = fma2_h_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), nib_float(h1, 0x7604),
+                                  nib_float(h1, 0x7624), SB, SB2, CB);
+            rb[2 * j + 1] = fma2_h_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), nib_float(h1, 0x7614),
+                                      nib_float(h1, 0x7634), SB, SB2, CB);
         }
     } else {
         // 6-bit: q = lo + 16 hi, hi in 2-bit fields (word j/2, pair s = 4(j&1) + r at bits 2s and
@@ -261,14 +282,13 @@ __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uin
             const uint32_t hv = (j < 2) ? hi.x : hi.y;
             const int s0 = 8 * (j & 1);
             auto f2 = [&](int sh) { return (float)((hv >> sh) & 3u); };
-            ra[2 * j] = fma2_bf16_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), f2(s0), f2(16 + s0), SA, SA2,
-                                     CA);
-            ra[2 * j + 1] = fma2_bf16_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), f2(s0 + 4), f2(20 + s0),
-                                         SA, SA2, CA);
-            rb[2 * j] = fma2_bf16_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), f2(s0 + 2), f2(18 + s0), SB,
-                                     SB2, CB);
-            rb[2 * j + 1] = fma2_bf16_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), f2(s0 + 6), f2(22 + s0),
-                                         SB, SB2, CB);
+            ra[2 * j] = fma2_h_hi(nib_float(m0, 0x7054), nib_float(m0, 0x7254), f2(s0), f2(16 + s0), SA, SA2, CA);
+            ra[2 * j + 1] = fma2_h_hi(nib_float(m0, 0x7154), nib_float(m0, 0x7354), f2(s0 + 4), f2(20 + s0), SA,
+                                      SA2, CA);
+            rb[2 * j] = fma2_h_hi(nib_float(m1, 0x7604), nib_float(m1, 0x7624), f2(s0 + 2), f2(18 + s0), SB, SB2,
+                                  CB);
+            rb[2 * j + 1] = fma2_h_hi(nib_float(m1, 0x7614), nib_float(m1, 0x7634), f2(s0 + 6), f2(22 + s0), SB,
+                                      SB2, CB);
         }
     }
     const int r0 = 16 * b + g, r1 = r0 + 8;
@@ -320,18 +340,42 @@ __device__ __forceinline__ void issue_fragment(const DqStep &d, uint32_t rawt, i
     cp_async8(rawt + 1024 + 8 * L, d.tile + kLoBytes + hi_bytes(d.bits) + 8 * (L >> 2));
 }
 
+// 2^d as an fp16 pair for d <= 0 (subnormal below 2^-14, zero below 2^-24)
+__device__ __forceinline__ uint32_t h2_pow2(int d) {
+    uint32_t b = 0;
+    if (d >= -14) b = (uint32_t)(15 + d) << 10;
+    else if (d >= -24) b = 1u << (24 + d);
+    return b | (b << 16);
+}
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
 // ------------------------------------------------------------------------------ the kernel
 template <bool GU>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs a) {
     extern __shared__ uint8_t tc_dyn[];
     __shared__ TcShared S;
+    __shared__ int ep_i[kMaxN];     // epilogue: token of each column (down) / unused (gate/up)
+    __shared__ float ep_f[kMaxN];   // epilogue: 2^xexp of each column (gate/up) / w * 2^fexp (down)
     const uint32_t pad = (1024u - (smem_u32(tc_dyn) & 1023u)) & 1023u;
-    uint8_t *ring = tc_dyn + pad;                               // kABStages x [A | B]
-    uint8_t *raw = ring + (size_t)kABStages * kStageBytes;      // kRawSlots x 8 packed-tile copies
-    uint8_t *staging = raw + (size_t)kRawSlots * kRawStage;     // h tile of the gate/up epilogue
+    uint8_t *base = tc_dyn + pad;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Geometry<GU> G(a);
     const int nunits = __ldg(a.nt_start + a.E) * G.mtiles;
+    const int nr_max = __ldg(a.nt_start + a.E + 1);
+    const int SUB = a.I / 16;                                  // 16-column blocks of an h row
+    // shared memory: kABStages x [A 16 KB | B nr_max x 128 B], then the h staging tile (gate/up)
+    // or the per-row exponent table (down), then the raw ring
+    const uint32_t bbytes = (uint32_t)align_up((size_t)(nr_max > 0 ? nr_max : 16) * 128, 1024);
+    const uint32_t stage_bytes = kABytes + bbytes;
+    uint8_t *ring = base;
+    uint8_t *side = ring + (size_t)kABStages * stage_bytes;
+    const uint32_t side_bytes = (uint32_t)align_up(GU ? (size_t)nr_max * 128 : (size_t)nr_max * SUB, 1024);
+    uint8_t *raw = side + side_bytes;
+    int R = (int)(((long long)a.smem_bytes - (long long)pad - (long long)(raw - base)) / kRawStep);
+    R = R > kMaxRaw ? kMaxRaw : R;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kABStages; ++s) {
@@ -343,7 +387,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
             mbar_init(smem_u32(&S.acc_empty[s]), 4);
         }
         mbar_init(smem_u32(&S.fin), 1);
-        S.abort = 0;
+        for (int b = 0; b < kDqWarps; ++b)
+            for (int s = 0; s < kMaxRaw; ++s) mbar_init(smem_u32(&S.rawbar[b][s]), 32);
+        S.abort = (R < 2) ? 1 : 0;
+        if (R < 2) atomicOr(a.status, kStatusCheck);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -356,43 +403,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    const bool run = !S.abort;
 
     if (warp < kDqWarps) {
         // ------------------------------------------------------------ dequantisers
         const int b = warp;
-        // issue-side cursor, kRawAhead K steps ahead of the consuming loop
         int iu = blockIdx.x, ikg = 0;
         Unit IU{};
         if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
-        auto issue_next = [&](uint32_t rslot) {
+        uint32_t issued = 0;
+        // issue-side cursor, R - 1 K steps ahead of the consuming loop; every lane arrives on the
+        // slot's barrier once its own copies of that slot have landed
+        auto issue_next = [&]() {
+            const uint32_t slot = issued % (uint32_t)R;
             if (iu < nunits) {
                 const DqStep d = dq_step<GU>(a, G, IU, b, ikg);
-                issue_fragment(d, smem_u32(raw + (size_t)rslot * kRawStage + b * kRawTile), lane);
+                issue_fragment(d, smem_u32(raw + (size_t)slot * kRawStep + b * kRawTile), lane);
                 if (++ikg == G.KG) {
                     ikg = 0;
                     iu += gridDim.x;
                     if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
                 }
             }
-            cp_async_commit();
+            cp_async_arrive(smem_u32(&S.rawbar[b][slot]));
+            ++issued;
         };
-        for (uint32_t p = 0; p < kRawAhead; ++p) issue_next(p);
+        if (run)
+            for (int p = 0; p < R - 1; ++p) issue_next();
         uint32_t j = 0;
-        bool ok = true;
+        bool ok = run;
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
             for (int kg = 0; kg < G.KG; ++kg, ++j) {
-                issue_next((j + kRawAhead) % kRawSlots);
-                cp_async_wait<kRawAhead>();
+                issue_next();
+                if (!tc_wait(S, a, &S.rawbar[b][j % R], (j / R) & 1u)) {
+                    ok = false;
+                    break;
+                }
                 const int slot = j % kABStages;
                 const uint32_t use = j / kABStages;
                 if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
                     ok = false;
                     break;
                 }
-                uint8_t *As = ring + (size_t)slot * kStageBytes;
+                uint8_t *As = ring + (size_t)slot * stage_bytes;
                 const DqStep d = dq_step<GU>(a, G, U, b, kg);
-                const uint8_t *rawt = raw + (size_t)(j % kRawSlots) * kRawStage + b * kRawTile;
+                const uint8_t *rawt = raw + (size_t)(j % R) * kRawStep + b * kRawTile;
                 if (d.tile == nullptr) {
                     // row block past the matrix: zero rows (the epilogue skips them)
                     const uint4 z = make_uint4(0, 0, 0, 0);
@@ -413,62 +469,104 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                 if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[slot]));
             }
         }
-        cp_async_wait<0>();
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ token-row loaders
-        const int lt = threadIdx.x - kDqWarps * 32;  // 0..63
-        const int c = lt & 7, r0 = lt >> 3;          // 16-byte chunk, first row (rows r0 + 8m)
+        const int lt = threadIdx.x - kDqWarps * 32;  // 0..127
+        const int c = lt & 7, r0 = lt >> 3;          // 16-byte chunk, first row (rows r0 + 16m)
+        int8_t *subd = reinterpret_cast<int8_t *>(side);   // down: hexp - fexp of each (row, block)
         uint32_t j = 0, pending = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        uint32_t scl[kLoaderLag + 1][4];             // down: packed rescale exponents per pending step
+        bool ok = run;
+        // down: rescale this thread's chunks of a landed step in place (16 rows at most per thread)
+        auto rescale = [&](uint32_t step, int nn, int nr) {
+            uint8_t *Bs = ring + (size_t)(step % kABStages) * stage_bytes + kABytes;
+            const uint32_t *sc = scl[step % (kLoaderLag + 1)];
+            for (int r = r0, m = 0; r < nr; r += 16, ++m) {
+                if (r >= nn) continue;
+                const int d = (int)(int8_t)((sc[m >> 2] >> (8 * (m & 3))) & 0xFF);
+                if (d == 0) continue;
+                uint4 *p = reinterpret_cast<uint4 *>(Bs + sw128_off(r, c));
+                const uint32_t f = h2_pow2(d);
+                uint4 v = *p;
+                v.x = hmul2_bits(v.x, f);
+                v.y = hmul2_bits(v.y, f);
+                v.z = hmul2_bits(v.z, f);
+                v.w = hmul2_bits(v.w, f);
+                *p = v;
+            }
+        };
+        int pnn[kLoaderLag + 1], pnr[kLoaderLag + 1];
+        // every loader walks all units through the same named barriers; after an expired wait it
+        // only skips the work
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
-            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's row table is no longer read
-            for (int r = lt; r < U.nn; r += kLdWarps * 32)
-                S.rows[r] = GU ? __ldg(a.pair_tok + U.base + U.n0 + r) : U.base + U.n0 + r;
+            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's tables are no longer read
+            for (int r = lt; r < U.nn; r += kLdWarps * 32) {
+                const int pos = U.base + U.n0 + r;
+                S.rows[r] = GU ? __ldg(a.pair_tok + pos) : pos;
+                if (!GU) S.rowexp[r] = __ldg(a.fexp + pos);
+            }
             named_sync(kBarLd, kLdWarps * 32);
-            for (int kg = 0; kg < G.KG; ++kg, ++j) {
+            if (!GU) {
+                for (int i = lt; i < U.nn * SUB; i += kLdWarps * 32) {
+                    const int r = i / SUB, sb = i - r * SUB;
+                    subd[i] = (int8_t)max(-127, (int)__ldg(a.hexp + (size_t)(U.base + U.n0 + r) * SUB + sb) - S.rowexp[r]);
+                }
+                named_sync(kBarLd, kLdWarps * 32);
+            }
+            for (int kg = 0; kg < G.KG && ok; ++kg, ++j) {
                 const int slot = j % kABStages;
                 const uint32_t use = j / kABStages;
                 if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
                     ok = false;
                     break;
                 }
-                const uint32_t Bs = smem_u32(ring + (size_t)slot * kStageBytes + kABytes);
-                for (int r = r0; r < U.nr; r += 8) {
+                const uint32_t Bs = smem_u32(ring + (size_t)slot * stage_bytes + kABytes);
+                uint32_t *sc = scl[j % (kLoaderLag + 1)];
+                sc[0] = sc[1] = sc[2] = sc[3] = 0;
+                for (int r = r0, m = 0; r < U.nr; r += 16, ++m) {
                     const uint32_t dst = Bs + sw128_off(r, c);
                     if (r < U.nn) {
                         cp_async16(dst, a.act + (size_t)S.rows[r] * G.K + kg * kGroup + c * 8);
+                        if (!GU) sc[m >> 2] |= (uint32_t)(uint8_t)subd[r * SUB + kg * 4 + (c >> 1)] << (8 * (m & 3));
                     } else {
                         asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
                     }
                 }
+                pnn[j % (kLoaderLag + 1)] = U.nn;
+                pnr[j % (kLoaderLag + 1)] = U.nr;
                 cp_async_commit();
                 if (pending == kLoaderLag) {
                     cp_async_wait<kLoaderLag>();
+                    const uint32_t q = j - kLoaderLag;
+                    if (!GU) rescale(q, pnn[q % (kLoaderLag + 1)], pnr[q % (kLoaderLag + 1)]);
                     fence_proxy_async();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[(j - kLoaderLag) % kABStages]));
+                    if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
                 } else {
                     ++pending;
                 }
             }
         }
         cp_async_wait<0>();
-        fence_proxy_async();
-        __syncwarp();
         // the K steps still owed an arrival (their copies are complete now)
-        if (lane == 0)
-            for (uint32_t q = j - pending; q < j; ++q) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
+        for (uint32_t q = j - pending; ok && q < j; ++q) {
+            if (!GU) rescale(q, pnn[q % (kLoaderLag + 1)], pnr[q % (kLoaderLag + 1)]);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
+        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         uint32_t j = 0, i = 0;
-        bool ok = true;
+        bool ok = run;
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++i) {
             const Unit U = unit_at(a, u, G.mtiles);
             const uint32_t buf = i & 1u;
             if (i >= 2 && !tc_wait(S, a, &S.acc_empty[buf], ((i >> 1) - 1) & 1u)) break;
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(kTM, U.nr);
+            const uint32_t idesc = idesc_f16_f32(kTM, U.nr);
             const uint32_t d_tmem = tmem + buf * kMaxN;
             for (int kg = 0; kg < G.KG; ++kg, ++j) {
                 const int slot = j % kABStages;
@@ -477,12 +575,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 tc_fence_after();
-                const uint32_t As = smem_u32(ring + (size_t)slot * kStageBytes);
+                const uint32_t As = smem_u32(ring + (size_t)slot * stage_bytes);
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d_tmem, sw128_desc(As + 32 * kk), sw128_desc(As + kABytes + 32 * kk), idesc,
-                                  (kg > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(d_tmem, sw128_desc(As + 32 * kk), sw128_desc(As + kABytes + 32 * kk), idesc,
+                                 (kg > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(smem_u32(&S.ab_empty[slot]));
                 }
                 __syncwarp();
@@ -502,17 +600,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         const int row = 32 * q + lane;   // accumulator row
         const int et = threadIdx.x - kEpiWarp0 * 32;
         uint32_t i = 0;
+        bool ok = run;
+        // every epilogue warp walks all units through the same named barriers; after an expired
+        // wait it only skips the work
         for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
             const Unit U = unit_at(a, u, G.mtiles);
             const uint32_t buf = i & 1u;
-            if (!tc_wait(S, a, &S.acc_full[buf], (i >> 1) & 1u)) break;
+            // per-column tables of this unit (filled while its MMAs run)
+            named_sync(kBarEpi, 128);
+            for (int r = et; ok && r < U.nn; r += 128) {
+                const int pos = U.base + U.n0 + r;
+                if (GU) {
+                    ep_f[r] = exp2i(__ldg(a.xexp + __ldg(a.pair_tok + pos)));
+                } else {
+                    ep_i[r] = __ldg(a.pair_tok + pos);
+                    ep_f[r] = __ldg(a.pair_w + pos) * exp2i(__ldg(a.fexp + pos));
+                }
+            }
+            named_sync(kBarEpi, 128);
+            if (ok && !tc_wait(S, a, &S.acc_full[buf], (i >> 1) & 1u)) ok = false;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kMaxN;
             if (GU) {
                 // row 16b + g: gate (g < 8) or up (g >= 8) of intermediate column 8b + (g & 7)
                 const bool gate = (row & 8) == 0;
                 const int col = 8 * (row >> 4) + (row & 7);
-                for (int c0 = 0; c0 < U.nr; c0 += 16) {
+                uint16_t *stg = reinterpret_cast<uint16_t *>(side);
+                for (int c0 = 0; ok && c0 < U.nr; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(taddr + c0, v);
 #pragma unroll
@@ -520,44 +634,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                         // the gate lane finishes token c0+jj, its up partner token c0+jj+1
                         const float send = __uint_as_float(gate ? v[jj + 1] : v[jj]);
                         const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-                        const float gv = gate ? __uint_as_float(v[jj]) : recv;
-                        const float uv = gate ? recv : __uint_as_float(v[jj + 1]);
-                        const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
                         const int tok = c0 + jj + (gate ? 0 : 1);
-                        reinterpret_cast<uint16_t *>(staging)[tok * 64 + col] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(hv));
+                        const float xs = ep_f[tok < U.nn ? tok : 0];
+                        const float gv = (gate ? __uint_as_float(v[jj]) : recv) * xs;
+                        const float uv = (gate ? recv : __uint_as_float(v[jj + 1])) * xs;
+                        const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                        // one exponent per 16 columns of this token: the max over the 16 lanes
+                        // that hold the token (gate lanes 0-7, 16-23 or up lanes 8-15, 24-31)
+                        const uint32_t hb = (tok < U.nn) ? (__float_as_uint(hv) & 0x7FFFFFFFu) : 0u;
+                        const uint32_t mx = gate ? __reduce_max_sync(0x00FF00FFu, hb) : __reduce_max_sync(0xFF00FF00u, hb);
+                        const int f = scale_exp(__uint_as_float(mx));
+                        stg[tok * 64 + col] = __half_as_ushort(__float2half_rn(hv * exp2i(-f)));
+                        if ((lane & 23) == 0 && tok < U.nn)   // lane 0 (gate group) or lane 8 (up group)
+                            a.hexp_out[(size_t)(U.base + U.n0 + tok) * SUB + 4 * U.mt + q] = (int8_t)f;
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
+                if (ok && lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
                 named_sync(kBarEpi, 128);
                 // coalesced copy-out: 8 threads per 128-byte token row
                 const int cc = et & 7;
-                for (int tok = et >> 3; tok < U.nn; tok += 16) {
-                    const uint4 val = *reinterpret_cast<const uint4 *>(staging + tok * 128 + cc * 16);
+                for (int tok = et >> 3; ok && tok < U.nn; tok += 16) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(side + tok * 128 + cc * 16);
                     *reinterpret_cast<uint4 *>(a.h + (size_t)(U.base + U.n0 + tok) * a.I + 64 * U.mt + cc * 8) = val;
                 }
-                named_sync(kBarEpi, 128);
             } else {
                 const int orow = kTM * U.mt + row;
                 const bool valid = orow < a.H;
-                for (int c0 = 0; c0 < U.nr; c0 += 16) {
+                for (int c0 = 0; ok && c0 < U.nr; c0 += 16) {
                     uint32_t v[16];
                     tmem_ld16(taddr + c0, v);
 #pragma unroll
                     for (int jj = 0; jj < 16; ++jj) {
                         const int tok = c0 + jj;
-                        if (valid && tok < U.nn) {
-                            const int pos = U.base + U.n0 + tok;
-                            red_add_f32(a.out_acc + (size_t)__ldg(a.pair_tok + pos) * a.H + orow,
-                                        __ldg(a.pair_w + pos) * __uint_as_float(v[jj]));
-                        }
+                        if (valid && tok < U.nn)
+                            red_add_f32(a.out_acc + (size_t)ep_i[tok] * a.H + orow, ep_f[tok] * __uint_as_float(v[jj]));
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
+                if (ok && lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
             }
         }
     }
@@ -570,59 +687,122 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     }
 }
 
-// Exclusive prefix of the experts' N-tile counts (nt_start[E] = total), one CTA of 1024 threads.
+// Exclusive prefix of the experts' N-tile counts (nt_start[E] = total) and the largest N tile in
+// rows (nt_start[E + 1]); one CTA of 1024 threads.
 __global__ void ntile_scan_kernel(const int32_t *counts, int E, int32_t *nt_start) {
     __shared__ int warp_tot[32];
+    __shared__ int warp_max[32];
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
-    const int c = e < E ? ntile_count(counts[e]) : 0;
-    int incl = c;
+    const int n = e < E ? counts[e] : 0;
+    const int c = ntile_count(n);
+    const int sz = (ntile_size(n) + 15) & ~15;
+    int incl = c, mx = sz;
     for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
     if (lane == 31) warp_tot[w] = incl;
+    if (lane == 0) warp_max[w] = mx;
     __syncthreads();
     if (w == 0) {
         const int v = warp_tot[lane];
-        int iv = v;
+        int iv = v, m = warp_max[lane];
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(0xffffffffu, iv, off);
             if (lane >= off) iv += o;
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
         }
         warp_tot[lane] = iv - v;
+        if (lane == 0) warp_max[0] = m;
     }
     __syncthreads();
     if (e < E) {
         const int excl = warp_tot[w] + incl - c;
         nt_start[e] = excl;
-        if (e == E - 1) nt_start[E] = excl + c;
+        if (e == E - 1) {
+            nt_start[E] = excl + c;
+            nt_start[E + 1] = warp_max[0];
+        }
     }
+}
+
+// x16[t] = fp16(x[t] * 2^-xexp[t]) with the per-token exponent chosen so that no value exceeds
+// 2^15 (xexp = 0 unless some |x| >= 2^15); one warp per token.
+__global__ void x16_kernel(const uint16_t *x, int T, int H, uint16_t *x16, int32_t *xexp) {
+    const int lane = threadIdx.x & 31;
+    for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += gridDim.x * (blockDim.x / 32)) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        uint32_t mx = 0;
+        for (int i = lane; i < H / 8; i += 32) {
+            const uint4 v = __ldg(src + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx = max(mx, max((w[j] << 16) & 0x7FFFFFFFu, w[j] & 0x7FFF0000u));
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        const uint32_t e = (mx >> 23) & 0xFF;
+        const int f = (mx != 0u && (int)e - 127 >= 15) ? (int)e - 127 - 14 : 0;
+        const float sc = exp2i(-f);
+        uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * H);
+        for (int i = lane; i < H / 8; i += 32) {
+            const uint4 v = __ldg(src + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __half2 hv = __floats2half2_rn(__uint_as_float(w[j] << 16) * sc, __uint_as_float(w[j] & 0xFFFF0000u) * sc);
+                o[j] = *reinterpret_cast<const uint32_t *>(&hv);
+            }
+            dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (lane == 0) xexp[t] = f;
+    }
+}
+
+// fexp[p] = the largest of the pair's 16-column exponents hexp[p][*]; one thread per pair.
+__global__ void fexp_kernel(const int8_t *hexp, int P, int SUB, int32_t *fexp) {
+    for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
+        int m = -128;
+        for (int s = 0; s < SUB; ++s) m = max(m, (int)hexp[(size_t)p * SUB + s]);
+        fexp[p] = m;
+    }
+}
+
+template <bool GU>
+moe_status_t launch_tc(const TcArgs &a0, const DeviceInfo *dev, cudaStream_t st) {
+    TcArgs a = a0;
+    a.smem_bytes = dev->max_smem_optin - (int)sizeof(TcShared) - 2 * kMaxN * 4 - 256;
+    static bool attr_set[64] = {};
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return MOE_ERR_CUDA;
+    if (!attr_set[d]) {
+        if (cudaFuncSetAttribute(tc_grouped_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 a.smem_bytes) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_set[d] = true;
+    }
+    tc_grouped_kernel<GU><<<(unsigned)dev->sms, kTcThreads, a.smem_bytes, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
 
-int prefill_ntile_count(int n) { return ntile_count(n); }
-
-moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int H, int I, int E, const int32_t *counts,
+moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I, int E, int k, const int32_t *counts,
                                      const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
-                                     const float *pair_w, const uint16_t *x, uint16_t *h, float *out_acc,
-                                     uint32_t *status, cudaStream_t st) {
+                                     const float *pair_w, const uint16_t *x, uint16_t *x16, int32_t *xexp,
+                                     uint16_t *h16, int8_t *hexp, int32_t *fexp, float *out_acc, uint32_t *status,
+                                     cudaStream_t st) {
     const DeviceInfo *dev = device_info();
     if (dev == nullptr) return MOE_ERR_CUDA;
-    if ((int)(kTcSmemBytes + sizeof(TcShared)) > dev->max_smem_optin) return MOE_ERR_UNSUPPORTED;
-    static bool attr_set[64] = {};
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess || d >= 64) return MOE_ERR_CUDA;
-    if (!attr_set[d]) {
-        if (cudaFuncSetAttribute(tc_grouped_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kTcSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tc_grouped_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kTcSmemBytes) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_set[d] = true;
-    }
+    if (I / 16 > kMaxSub) return MOE_ERR_UNSUPPORTED;
+    const size_t P = (size_t)T * k;
     ntile_scan_kernel<<<1, 1024, 0, st>>>(counts, E, nt_start);
-    TcArgs a;
+    {
+        const unsigned blocks = (unsigned)((T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096);
+        x16_kernel<<<blocks, 256, 0, st>>>(x, T, H, x16, xexp);
+    }
+    TcArgs a{};
     a.packed = packed;
     a.H = H;
     a.I = I;
@@ -632,15 +812,21 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int H, int I, int E,
     a.nt_start = nt_start;
     a.pair_tok = pair_tok;
     a.pair_w = pair_w;
-    a.h = h;
+    a.xexp = xexp;
+    a.h = h16;
+    a.hexp_out = hexp;
+    a.hexp = hexp;
+    a.fexp = fexp;
     a.out_acc = out_acc;
     a.wait_ns = wait_limit_ns();
     a.status = status;
-    const unsigned grid = (unsigned)dev->sms;
-    a.act = x;
-    tc_grouped_kernel<true><<<grid, kTcThreads, kTcSmemBytes, st>>>(a);
-    a.act = h;
-    tc_grouped_kernel<false><<<grid, kTcThreads, kTcSmemBytes, st>>>(a);
+    a.act = x16;
+    moe_status_t s = launch_tc<true>(a, dev, st);
+    if (s != MOE_OK) return s;
+    fexp_kernel<<<(unsigned)((P + 255) / 256 < 4096 ? (P + 255) / 256 : 4096), 256, 0, st>>>(hexp, (int)P, I / 16, fexp);
+    a.act = h16;
+    s = launch_tc<false>(a, dev, st);
+    if (s != MOE_OK) return s;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

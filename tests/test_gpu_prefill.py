@@ -58,3 +58,24 @@ def test_prefill_agrees_with_decode_on_small_batch():
     o = oracle.get()
     out_p, idx_p, w_p = prefill_call(layer, x, w.I, w.E, w.k)
     check_block(o, x, layer.wr_np, layer.bias_np, layer.expert_fn, w.E, w.H, w.I, w.k, out_p, idx_p, w_p)
+
+
+def test_prefill_route_then_experts_matches_oracle():
+    """The two halves of the prefill entry point, called separately on one workspace."""
+    rng = np.random.default_rng(77)
+    E, H, I, k, T = 12, 192, 128, 3, 257
+    exs = [pins.make_expert(rng, H, I, 4)[0] for e in range(E)]
+    wr = (rng.normal(0, 1, (E, H)) / np.sqrt(H)).astype(np.float32)
+    layer = HandLayer(exs, wr, None, H, I)
+    x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
+    xd = to_dev_bf16(x)
+    ws = qm.workspace(T, H, I, E, k, qm.MODE_PREFILL)
+    idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+    w = torch.zeros((T, k), dtype=torch.float32, device="cuda")
+    qm.prefill_route(xd, layer.wr, None, I, E, k, ws, idx_out=idx, w_out=w)
+    out = qm.prefill_experts(xd, layer.packed, I, E, k, ws)
+    assert qm.device_status(ws) == qm.MOE_OK
+    check_block(oracle.get(), x, wr, None, layer.expert_fn, E, H, I, k, bf16_f64(out), idx.cpu().numpy(),
+                w.cpu().numpy())
+    out2, idx2, _ = prefill_call(layer, x, I, E, k)
+    assert np.array_equal(idx2, idx.cpu().numpy())
