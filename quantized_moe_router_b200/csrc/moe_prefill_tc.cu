@@ -5,21 +5,25 @@
 // long prompt touches nearly every expert of a layer (the pages "Qwen-tin" and
 // "--moe-direct-io"). Both GEMMs run as one persistent kernel each (one CTA per SM) whose work
 // unit is (expert, 128 weight rows, up to 256 of the expert's tokens):
-//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, copy their lane
-//     fragments from HBM into a ring of raw slots with cp.async (completion tracked per slot by
-//     an mbarrier, so the look-ahead depth is whatever shared memory allows, up to 12 K steps),
-//     then write w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile A [128 x 64];
-//   * 4 loader warps copy the unit's token rows into a swizzled tile B [N x 64] with cp.async:
+//   * 1 producer warp streams the unit's packed tiles from HBM into a ring of raw slots with 1-D
+//     bulk copies (one per row block and K chunk of up to 4 tiles; the copy engine, not the
+//     load/store path, so the token-row loads below do not queue behind the weight stream);
+//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, read their tile
+//     from the raw slot and write w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile
+//     A [128 x 64];
+//   * 4 loader warps copy the unit's token rows into a swizzled tile B [N x 64] with cp.async and
+//     never wait for them: each thread's copies arrive on the stage's mbarrier when they land.
 //     gate/up reads x16 (the hidden states as fp16, scaled per token by a power of two so that
-//     no value overflows), down reads h16 and rescales each 16-column block in place to the
-//     pair's common exponent;
+//     no value overflows), down reads h16 (fp16, scaled per pair);
 //   * 1 warp issues tcgen05.mma (kind::f16, fp16 x fp16 -> fp32, M = 128, N = tokens rounded up
-//     to 16) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
+//     to 16; after each stage's barrier it fences the generic-proxy writes of that stage for the
+//     tensor core) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
 //     each ring stage with tcgen05.commit;
 //   * 4 epilogue warps read the other accumulator with tcgen05.ld while the next unit runs:
 //     gate/up undoes the token scale, pairs each gate row with its up row (8 TMEM lanes apart),
-//     applies SiLU-GLU and stores h as fp16 with one power-of-two exponent per 16 columns; down
-//     undoes the pair's exponent and adds w * y into the fp32 output accumulator with red.add.
+//     applies SiLU-GLU and stores h as fp16 with one power-of-two exponent per 16 columns (a small
+//     kernel between the GEMMs brings each pair's h to one common exponent); down undoes the
+//     pair's exponent and adds w * y into the fp32 output accumulator with red.add.
 // fp16 operands (11-bit significands) keep the block within its error bound where bf16
 // operands (8-bit) would not; every scaling is by a power of two and exact.
 // Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
@@ -33,16 +37,14 @@ constexpr int kTM = 128;                          // weight rows per unit (UMMA 
 constexpr int kMaxN = 256;                        // tokens per unit (UMMA N limit)
 constexpr int kABStages = 3;
 constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
-constexpr int kRawTile = 1280;                    // lane copies of one tile: lo 512 | hi 512 | scale/zero 256
-constexpr int kRawStep = 8 * kRawTile;            // one K step of the 8 dequantiser warps
-constexpr int kMaxRaw = 12;                       // raw ring slots (K steps) at most
+constexpr int kMaxRaw = 8;                        // raw ring slots (K chunks) at most
 constexpr int kDqWarps = 8, kLdWarps = 4;
 constexpr int kMmaWarp = kDqWarps + kLdWarps;
 constexpr int kEpiWarp0 = kMmaWarp + 1;
-constexpr int kTcWarps = kEpiWarp0 + 4;
+constexpr int kProdWarp = kEpiWarp0 + 4;
+constexpr int kTcWarps = kProdWarp + 1;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr uint32_t kTmemCols = 2 * kMaxN;         // two accumulators of 256 fp32 columns
-constexpr int kLoaderLag = kABStages - 1;         // K steps a loader keeps in flight before arriving
 constexpr int kBarEpi = 1, kBarLd = 2;            // named barriers (0 is __syncthreads)
 constexpr int kMaxSub = 64;                       // 16-column blocks of a down row (I <= 1024)
 
@@ -53,8 +55,7 @@ struct TcArgs {
     const float *pair_w;
     const uint16_t *act;   // gate/up: x16 [T x H]; down: h16 [pairs x I] in bucket order
     const int32_t *xexp;   // gate/up: per-token exponent of x16
-    const int8_t *hexp;    // down: per-pair, per-16-column exponents of h16
-    const int32_t *fexp;   // down: per-pair largest hexp
+    const int32_t *fexp;   // down: per-pair exponent of h16
     uint16_t *h;           // gate/up output: h16
     int8_t *hexp_out;      // gate/up output: exponents of h16
     float *out_acc;        // down output: [T x H] fp32
@@ -69,11 +70,11 @@ struct TcShared {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t fin;
-    uint64_t rawbar[kDqWarps][kMaxRaw];
+    uint64_t raw_full[kMaxRaw];
+    uint64_t raw_empty[kMaxRaw];
     uint32_t tmem_base;
     volatile int abort;
     int rows[kMaxN];          // loaders: activation row of each token of the current unit
-    int rowexp[kMaxN];        // loaders (down): the row's common exponent
 };
 
 // ------------------------------------------------------------------------------ work units
@@ -149,20 +150,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// L2 policy of the token rows, which every M tile of their expert reads (evict last)
+__device__ __forceinline__ uint64_t l2_policy_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
+}
+// 16 zero bytes through the same path (source size 0: nothing is read)
+__device__ __forceinline__ void cp_async16_zero(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(dst), "l"(src) : "memory");
 }
 // arrive on `bar` once every cp.async this thread issued so far has completed (the barrier's
 // expected count includes this arrival)
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -173,7 +179,7 @@ __device__ __forceinline__ bool tc_wait(TcShared &S, const TcArgs &a, uint64_t *
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = global_timer();
     while (true) {
-        if (mbar_try_wait(b, parity)) return true;
+        if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
         if (S.abort) return false;
         if (global_timer() - t0 > a.wait_ns) {
             atomicOr(a.status, kStatusTimeout);
@@ -228,15 +234,15 @@ __device__ __forceinline__ uint32_t fma2_h_hi(float x0, float x1, float y0, floa
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile, from the lane's
-// fragment copies in `rawt`, stored as fp16 into the swizzled A tile rows 16b+g and 16b+g+8.
+// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile (its image in
+// shared memory at `rawt`), stored as fp16 into the swizzled A tile rows 16b+g and 16b+g+8.
 // Word j of the lo plane holds columns 16t+4j+{0,1,2,3} in bytes {0,2,1,3}: row g in the low
 // nibbles, row g+8 in the high nibbles.
 template <int BITS>
 __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uint8_t *As, int b) {
     const int g = L >> 2, t = L & 3;
     const uint4 lo = *reinterpret_cast<const uint4 *>(rawt + 16 * L);
-    const uint2 sz = *reinterpret_cast<const uint2 *>(rawt + 1024 + 8 * L);
+    const uint2 sz = *reinterpret_cast<const uint2 *>(rawt + kLoBytes + hi_bytes(BITS) + 8 * g);
     const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
     const uint32_t w[4] = {lo.x, lo.y, lo.z, lo.w};
     uint32_t ra[8], rb[8];
@@ -331,15 +337,6 @@ __device__ __forceinline__ DqStep dq_step(const TcArgs &a, const Geometry<GU> &G
     return d;
 }
 
-// The lane's copies of one packed tile: lo 16 B, hi 8/16 B, its row pair's scale/zero entry 8 B.
-__device__ __forceinline__ void issue_fragment(const DqStep &d, uint32_t rawt, int L) {
-    if (d.tile == nullptr) return;
-    cp_async16(rawt + 16 * L, d.tile + 16 * L);
-    if (d.bits == 8) cp_async16(rawt + 512 + 16 * L, d.tile + kLoBytes + 16 * L);
-    if (d.bits == 6) cp_async8(rawt + 512 + 8 * L, d.tile + kLoBytes + 8 * L);
-    cp_async8(rawt + 1024 + 8 * L, d.tile + kLoBytes + hi_bytes(d.bits) + 8 * (L >> 2));
-}
-
 // 2^d as an fp16 pair for d <= 0 (subnormal below 2^-14, zero below 2^-24)
 __device__ __forceinline__ uint32_t h2_pow2(int d) {
     uint32_t b = 0;
@@ -366,20 +363,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     const int nunits = __ldg(a.nt_start + a.E) * G.mtiles;
     const int nr_max = __ldg(a.nt_start + a.E + 1);
     const int SUB = a.I / 16;                                  // 16-column blocks of an h row
-    // shared memory: kABStages x [A 16 KB | B nr_max x 128 B], then the h staging tile (gate/up)
-    // or the per-row exponent table (down), then the raw ring
+    // shared memory: kABStages x [A 16 KB | B nr_max x 128 B], then the h staging tile (gate/up),
+    // then the raw ring
     const uint32_t bbytes = (uint32_t)align_up((size_t)(nr_max > 0 ? nr_max : 16) * 128, 1024);
     const uint32_t stage_bytes = kABytes + bbytes;
     uint8_t *ring = base;
     uint8_t *side = ring + (size_t)kABStages * stage_bytes;
-    const uint32_t side_bytes = (uint32_t)align_up(GU ? (size_t)nr_max * 128 : (size_t)nr_max * SUB, 1024);
+    const uint32_t side_bytes = GU ? (uint32_t)align_up((size_t)nr_max * 128, 1024) : 0u;
     uint8_t *raw = side + side_bytes;
-    int R = (int)(((long long)a.smem_bytes - (long long)pad - (long long)(raw - base)) / kRawStep);
+    // K chunks of KC tiles per row block (KC divides the unit's K steps, so chunks never straddle
+    // units); a raw slot holds one chunk of the 8 row blocks at the layer's widest tile
+    const int KC = (G.KG % 4 == 0) ? 4 : ((G.KG % 2 == 0) ? 2 : 1);
+    int tb_max = 0;
+    {
+        const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
+        for (int e = 0; e < a.E; ++e) tb_max = max(tb_max, tile_bytes(pe[e].bits));
+    }
+    const uint32_t slot_bytes = (uint32_t)(8 * KC * tb_max);
+    int R = (int)(((long long)a.smem_bytes - (long long)pad - (long long)(raw - base)) / slot_bytes);
     R = R > kMaxRaw ? kMaxRaw : R;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kABStages; ++s) {
-            mbar_init(smem_u32(&S.ab_full[s]), kDqWarps + kLdWarps);
+            mbar_init(smem_u32(&S.ab_full[s]), kDqWarps + kLdWarps * 32);
             mbar_init(smem_u32(&S.ab_empty[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -387,8 +393,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
             mbar_init(smem_u32(&S.acc_empty[s]), 4);
         }
         mbar_init(smem_u32(&S.fin), 1);
-        for (int b = 0; b < kDqWarps; ++b)
-            for (int s = 0; s < kMaxRaw; ++s) mbar_init(smem_u32(&S.rawbar[b][s]), 32);
+        for (int s = 0; s < kMaxRaw; ++s) {
+            mbar_init(smem_u32(&S.raw_full[s]), 1);
+            mbar_init(smem_u32(&S.raw_empty[s]), kDqWarps);
+        }
         S.abort = (R < 2) ? 1 : 0;
         if (R < 2) atomicOr(a.status, kStatusCheck);
         fence_barrier_init();
@@ -408,35 +416,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     if (warp < kDqWarps) {
         // ------------------------------------------------------------ dequantisers
         const int b = warp;
-        int iu = blockIdx.x, ikg = 0;
-        Unit IU{};
-        if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
-        uint32_t issued = 0;
-        // issue-side cursor, R - 1 K steps ahead of the consuming loop; every lane arrives on the
-        // slot's barrier once its own copies of that slot have landed
-        auto issue_next = [&]() {
-            const uint32_t slot = issued % (uint32_t)R;
-            if (iu < nunits) {
-                const DqStep d = dq_step<GU>(a, G, IU, b, ikg);
-                issue_fragment(d, smem_u32(raw + (size_t)slot * kRawStep + b * kRawTile), lane);
-                if (++ikg == G.KG) {
-                    ikg = 0;
-                    iu += gridDim.x;
-                    if (iu < nunits) IU = unit_at(a, iu, G.mtiles);
-                }
-            }
-            cp_async_arrive(smem_u32(&S.rawbar[b][slot]));
-            ++issued;
-        };
-        if (run)
-            for (int p = 0; p < R - 1; ++p) issue_next();
         uint32_t j = 0;
         bool ok = run;
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
             for (int kg = 0; kg < G.KG; ++kg, ++j) {
-                issue_next();
-                if (!tc_wait(S, a, &S.rawbar[b][j % R], (j / R) & 1u)) {
+                const uint32_t chunk = j / KC;
+                const uint32_t rs = chunk % R;
+                if (j % KC == 0 && !tc_wait(S, a, &S.raw_full[rs], (chunk / R) & 1u)) {
                     ok = false;
                     break;
                 }
@@ -448,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                 }
                 uint8_t *As = ring + (size_t)slot * stage_bytes;
                 const DqStep d = dq_step<GU>(a, G, U, b, kg);
-                const uint8_t *rawt = raw + (size_t)(j % R) * kRawStep + b * kRawTile;
+                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + (int)(j % KC)) * tile_bytes(d.bits);
                 if (d.tile == nullptr) {
                     // row block past the matrix: zero rows (the epilogue skips them)
                     const uint4 z = make_uint4(0, 0, 0, 0);
@@ -466,55 +453,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                 }
                 fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[slot]));
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&S.ab_full[slot]));
+                    if (j % KC == (uint32_t)KC - 1) mbar_arrive(smem_u32(&S.raw_empty[rs]));
+                }
             }
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ token-row loaders
         const int lt = threadIdx.x - kDqWarps * 32;  // 0..127
         const int c = lt & 7, r0 = lt >> 3;          // 16-byte chunk, first row (rows r0 + 16m)
-        int8_t *subd = reinterpret_cast<int8_t *>(side);   // down: hexp - fexp of each (row, block)
-        uint32_t j = 0, pending = 0;
-        uint32_t scl[kLoaderLag + 1][4];             // down: packed rescale exponents per pending step
+        const uint64_t pol = l2_policy_last();
+        uint32_t j = 0;
         bool ok = run;
-        // down: rescale this thread's chunks of a landed step in place (16 rows at most per thread)
-        auto rescale = [&](uint32_t step, int nn, int nr) {
-            uint8_t *Bs = ring + (size_t)(step % kABStages) * stage_bytes + kABytes;
-            const uint32_t *sc = scl[step % (kLoaderLag + 1)];
-            for (int r = r0, m = 0; r < nr; r += 16, ++m) {
-                if (r >= nn) continue;
-                const int d = (int)(int8_t)((sc[m >> 2] >> (8 * (m & 3))) & 0xFF);
-                if (d == 0) continue;
-                uint4 *p = reinterpret_cast<uint4 *>(Bs + sw128_off(r, c));
-                const uint32_t f = h2_pow2(d);
-                uint4 v = *p;
-                v.x = hmul2_bits(v.x, f);
-                v.y = hmul2_bits(v.y, f);
-                v.z = hmul2_bits(v.z, f);
-                v.w = hmul2_bits(v.w, f);
-                *p = v;
-            }
-        };
-        int pnn[kLoaderLag + 1], pnr[kLoaderLag + 1];
         // every loader walks all units through the same named barriers; after an expired wait it
         // only skips the work
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
-            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's tables are no longer read
+            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's row table is no longer read
             for (int r = lt; r < U.nn; r += kLdWarps * 32) {
                 const int pos = U.base + U.n0 + r;
                 S.rows[r] = GU ? __ldg(a.pair_tok + pos) : pos;
-                if (!GU) S.rowexp[r] = __ldg(a.fexp + pos);
             }
             named_sync(kBarLd, kLdWarps * 32);
-            if (!GU) {
-                for (int i = lt; i < U.nn * SUB; i += kLdWarps * 32) {
-                    const int r = i / SUB, sb = i - r * SUB;
-                    subd[i] = (int8_t)max(-127, (int)__ldg(a.hexp + (size_t)(U.base + U.n0 + r) * SUB + sb) - S.rowexp[r]);
-                }
-                named_sync(kBarLd, kLdWarps * 32);
-            }
             for (int kg = 0; kg < G.KG && ok; ++kg, ++j) {
                 const int slot = j % kABStages;
                 const uint32_t use = j / kABStages;
@@ -523,40 +484,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 const uint32_t Bs = smem_u32(ring + (size_t)slot * stage_bytes + kABytes);
-                uint32_t *sc = scl[j % (kLoaderLag + 1)];
-                sc[0] = sc[1] = sc[2] = sc[3] = 0;
-                for (int r = r0, m = 0; r < U.nr; r += 16, ++m) {
+                for (int r = r0; r < U.nr; r += 16) {
                     const uint32_t dst = Bs + sw128_off(r, c);
-                    if (r < U.nn) {
-                        cp_async16(dst, a.act + (size_t)S.rows[r] * G.K + kg * kGroup + c * 8);
-                        if (!GU) sc[m >> 2] |= (uint32_t)(uint8_t)subd[r * SUB + kg * 4 + (c >> 1)] << (8 * (m & 3));
-                    } else {
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-                    }
+                    if (r < U.nn) cp_async16(dst, a.act + (size_t)S.rows[r] * G.K + kg * kGroup + c * 8, pol);
+                    else cp_async16_zero(dst, a.act);
                 }
-                pnn[j % (kLoaderLag + 1)] = U.nn;
-                pnr[j % (kLoaderLag + 1)] = U.nr;
-                cp_async_commit();
-                if (pending == kLoaderLag) {
-                    cp_async_wait<kLoaderLag>();
-                    const uint32_t q = j - kLoaderLag;
-                    if (!GU) rescale(q, pnn[q % (kLoaderLag + 1)], pnr[q % (kLoaderLag + 1)]);
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
-                } else {
-                    ++pending;
-                }
+                // arrives on the stage's barrier once this thread's copies have landed
+                cp_async_arrive(smem_u32(&S.ab_full[slot]));
             }
         }
-        cp_async_wait<0>();
-        // the K steps still owed an arrival (their copies are complete now)
-        for (uint32_t q = j - pending; ok && q < j; ++q) {
-            if (!GU) rescale(q, pnn[q % (kLoaderLag + 1)], pnr[q % (kLoaderLag + 1)]);
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&S.ab_full[q % kABStages]));
-        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         uint32_t j = 0, i = 0;
@@ -574,6 +511,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     ok = false;
                     break;
                 }
+                fence_proxy_async();  // the loaders' cp.async writes of this stage -> the tensor core
                 tc_fence_after();
                 const uint32_t As = smem_u32(ring + (size_t)slot * stage_bytes);
                 if (lane == 0) {
@@ -594,6 +532,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         if (lane == 0) umma_commit(smem_u32(&S.fin));
         __syncwarp();
         mbar_wait(smem_u32(&S.fin), 0, a.wait_ns, a.status);
+    } else if (warp == kProdWarp) {
+        // ------------------------------------------------------------ weight producer (one thread)
+        if (lane == 0 && run) {
+            const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
+            uint32_t chunk = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+                const Unit U = unit_at(a, u, G.mtiles);
+                const PackedExpert ex = pe[U.e];
+                const int tb = tile_bytes(ex.bits);
+                const uint8_t *mat = a.packed + ex.offset + G.skip_tiles * tb;
+                const int nb = min(8, G.nrb - 8 * U.mt);   // row blocks of this M tile
+                for (int k0 = 0; k0 < G.KG; k0 += KC, ++chunk) {
+                    const uint32_t rs = chunk % R;
+                    if (chunk >= (uint32_t)R && !tc_wait(S, a, &S.raw_empty[rs], ((chunk / R) - 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&S.raw_full[rs]);
+                    mbar_expect_tx(fb, (uint32_t)(nb * KC * tb));
+                    for (int b = 0; b < nb; ++b)
+                        bulk_g2s(smem_u32(raw + (size_t)rs * slot_bytes + (size_t)b * KC * tb),
+                                 mat + ((size_t)(8 * U.mt + b) * G.KG + k0) * tb, (uint32_t)(KC * tb), fb);
+                }
+            }
+            // copies still in flight land before the CTA may exit
+            for (uint32_t q = chunk > (uint32_t)R ? chunk - R : 0; q < chunk; ++q)
+                mbar_wait(smem_u32(&S.raw_full[q % R]), (q / R) & 1u, a.wait_ns, a.status);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;          // this warp may read TMEM lanes 32q .. 32q+31
@@ -760,12 +727,30 @@ __global__ void x16_kernel(const uint16_t *x, int T, int H, uint16_t *x16, int32
     }
 }
 
-// fexp[p] = the largest of the pair's 16-column exponents hexp[p][*]; one thread per pair.
-__global__ void fexp_kernel(const int8_t *hexp, int P, int SUB, int32_t *fexp) {
-    for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
+// Brings each pair's h16 to one exponent: fexp[p] = max over its 16-column exponents hexp[p][*],
+// and every block is multiplied by 2^(hexp - fexp) in place (exact unless the block falls into
+// fp16's subnormal range, where its contribution is negligible). One warp per pair.
+__global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, int P, int I, int32_t *fexp) {
+    const int lane = threadIdx.x & 31;
+    const int SUB = I / 16;
+    for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
         int m = -128;
-        for (int s = 0; s < SUB; ++s) m = max(m, (int)hexp[(size_t)p * SUB + s]);
-        fexp[p] = m;
+        for (int sb = lane; sb < SUB; sb += 32) m = max(m, (int)hexp[(size_t)p * SUB + sb]);
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) fexp[p] = m;
+        // 8 fp16 per 16-byte chunk, two chunks per 16-column block
+        uint4 *row = reinterpret_cast<uint4 *>(h16 + (size_t)p * I);
+        for (int ch = lane; ch < I / 8; ch += 32) {
+            const int d = (int)hexp[(size_t)p * SUB + ch / 2] - m;
+            if (d == 0) continue;
+            const uint32_t f = h2_pow2(d);
+            uint4 v = row[ch];
+            v.x = hmul2_bits(v.x, f);
+            v.y = hmul2_bits(v.y, f);
+            v.z = hmul2_bits(v.z, f);
+            v.w = hmul2_bits(v.w, f);
+            row[ch] = v;
+        }
     }
 }
 
@@ -815,7 +800,6 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I,
     a.xexp = xexp;
     a.h = h16;
     a.hexp_out = hexp;
-    a.hexp = hexp;
     a.fexp = fexp;
     a.out_acc = out_acc;
     a.wait_ns = wait_limit_ns();
@@ -823,7 +807,7 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I,
     a.act = x16;
     moe_status_t s = launch_tc<true>(a, dev, st);
     if (s != MOE_OK) return s;
-    fexp_kernel<<<(unsigned)((P + 255) / 256 < 4096 ? (P + 255) / 256 : 4096), 256, 0, st>>>(hexp, (int)P, I / 16, fexp);
+    h16_rescale_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(h16, hexp, (int)P, I, fexp);
     a.act = h16;
     s = launch_tc<false>(a, dev, st);
     if (s != MOE_OK) return s;
