@@ -101,7 +101,8 @@ inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
     return w;
 }
 
-// Prefill workspace. x16: the hidden states as fp16 scaled by 2^-xexp[t] per token; h: fp16 h of
+// Prefill workspace. x16: the hidden states of every (token, expert) pair in bucket order as fp16
+// scaled by 2^-xexp[t] per token; h: fp16 h of
 // every (token, expert) pair in bucket order, scaled by 2^-hexp per 16-column block; fexp: the
 // largest hexp of each pair; nt_start: N-tile prefix of the experts ([E] = total, [E+1] = the
 // largest N tile, rows rounded to 16).
@@ -124,7 +125,7 @@ inline PrefillWs prefill_ws_layout(int T, int H, int I, int E, int k) {
     w.pair_tok = take(P * 4);
     w.pair_w = take(P * 4);
     w.nt_start = take((size_t)(E + 2) * 4);
-    w.x16 = take((size_t)T * H * 2);
+    w.x16 = take(P * H * 2);
     w.xexp = take((size_t)T * 4);
     w.h = take(P * I * 2);
     w.hexp = take(P * (I / 16));

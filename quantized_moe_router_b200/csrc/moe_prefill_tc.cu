@@ -11,13 +11,12 @@
 //   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, read their tile
 //     from the raw slot and write w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile
 //     A [128 x 64];
-//   * 4 loader warps copy the unit's token rows into a swizzled tile B [N x 64] with cp.async and
-//     never wait for them: each thread's copies arrive on the stage's mbarrier when they land.
-//     gate/up reads x16 (the hidden states as fp16, scaled per token by a power of two so that
-//     no value overflows), down reads h16 (fp16, scaled per pair);
+//   * 1 loader thread brings the unit's token rows into a swizzled tile B [N x 64] with 2-D tensor
+//     copies (TMA, 64 rows each, the 128-byte swizzle applied by the copy engine): gate/up reads
+//     x16, the pairs' hidden states in bucket order as fp16 (scaled per token by a power of two
+//     so that no value overflows), down reads h16 (fp16, scaled per pair);
 //   * 1 warp issues tcgen05.mma (kind::f16, fp16 x fp16 -> fp32, M = 128, N = tokens rounded up
-//     to 16; after each stage's barrier it fences the generic-proxy writes of that stage for the
-//     tensor core) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
+//     to 16) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
 //     each ring stage with tcgen05.commit;
 //   * 4 epilogue warps read the other accumulator with tcgen05.ld while the next unit runs:
 //     gate/up undoes the token scale, pairs each gate row with its up row (8 TMEM lanes apart),
@@ -27,6 +26,9 @@
 // fp16 operands (11-bit significands) keep the block within its error bound where bf16
 // operands (8-bit) would not; every scaling is by a power of two and exact.
 // Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -38,14 +40,15 @@ constexpr int kMaxN = 256;                        // tokens per unit (UMMA N lim
 constexpr int kABStages = 3;
 constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
 constexpr int kMaxRaw = 8;                        // raw ring slots (K chunks) at most
-constexpr int kDqWarps = 8, kLdWarps = 4;
+constexpr int kDqWarps = 8, kLdWarps = 1;
+constexpr int kRowBox = 64;                       // token rows per tensor copy
 constexpr int kMmaWarp = kDqWarps + kLdWarps;
 constexpr int kEpiWarp0 = kMmaWarp + 1;
 constexpr int kProdWarp = kEpiWarp0 + 4;
 constexpr int kTcWarps = kProdWarp + 1;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr uint32_t kTmemCols = 2 * kMaxN;         // two accumulators of 256 fp32 columns
-constexpr int kBarEpi = 1, kBarLd = 2;            // named barriers (0 is __syncthreads)
+constexpr int kBarEpi = 1;                        // named barrier of the epilogue warps (0 is __syncthreads)
 constexpr int kMaxSub = 64;                       // 16-column blocks of a down row (I <= 1024)
 
 struct TcArgs {
@@ -53,7 +56,7 @@ struct TcArgs {
     int H, I, E;
     const int32_t *counts, *offsets, *nt_start, *pair_tok;
     const float *pair_w;
-    const uint16_t *act;   // gate/up: x16 [T x H]; down: h16 [pairs x I] in bucket order
+    const uint16_t *act;   // gate/up: x16 [pairs x H]; down: h16 [pairs x I], both in bucket order
     const int32_t *xexp;   // gate/up: per-token exponent of x16
     const int32_t *fexp;   // down: per-pair exponent of h16
     uint16_t *h;           // gate/up output: h16
@@ -74,7 +77,6 @@ struct TcShared {
     uint64_t raw_empty[kMaxRaw];
     uint32_t tmem_base;
     volatile int abort;
-    int rows[kMaxN];          // loaders: activation row of each token of the current unit
 };
 
 // ------------------------------------------------------------------------------ work units
@@ -149,25 +151,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-// L2 policy of the token rows, which every M tile of their expert reads (evict last)
-__device__ __forceinline__ uint64_t l2_policy_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
-                 : "memory");
-}
-// 16 zero bytes through the same path (source size 0: nothing is read)
-__device__ __forceinline__ void cp_async16_zero(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(dst), "l"(src) : "memory");
-}
-// arrive on `bar` once every cp.async this thread issued so far has completed (the barrier's
-// expected count includes this arrival)
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -351,7 +334,7 @@ __device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
 
 // ------------------------------------------------------------------------------ the kernel
 template <bool GU>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs a) {
+__global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t tc_dyn[];
     __shared__ TcShared S;
     __shared__ int ep_i[kMaxN];     // epilogue: token of each column (down) / unused (gate/up)
@@ -365,7 +348,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     const int SUB = a.I / 16;                                  // 16-column blocks of an h row
     // shared memory: kABStages x [A 16 KB | B nr_max x 128 B], then the h staging tile (gate/up),
     // then the raw ring
-    const uint32_t bbytes = (uint32_t)align_up((size_t)(nr_max > 0 ? nr_max : 16) * 128, 1024);
+    const uint32_t bbytes = (uint32_t)align_up((size_t)(nr_max > 0 ? nr_max : 16), kRowBox) * 128;
     const uint32_t stage_bytes = kABytes + bbytes;
     uint8_t *ring = base;
     uint8_t *side = ring + (size_t)kABStages * stage_bytes;
@@ -385,7 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kABStages; ++s) {
-            mbar_init(smem_u32(&S.ab_full[s]), kDqWarps + kLdWarps * 32);
+            mbar_init(smem_u32(&S.ab_full[s]), kDqWarps + 1);
             mbar_init(smem_u32(&S.ab_empty[s]), 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -460,40 +443,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
             }
         }
     } else if (warp < kMmaWarp) {
-        // ------------------------------------------------------------ token-row loaders
-        const int lt = threadIdx.x - kDqWarps * 32;  // 0..127
-        const int c = lt & 7, r0 = lt >> 3;          // 16-byte chunk, first row (rows r0 + 16m)
-        const uint64_t pol = l2_policy_last();
-        uint32_t j = 0;
-        bool ok = run;
-        // every loader walks all units through the same named barriers; after an expired wait it
-        // only skips the work
-        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-            const Unit U = unit_at(a, u, G.mtiles);
-            named_sync(kBarLd, kLdWarps * 32);  // the previous unit's row table is no longer read
-            for (int r = lt; r < U.nn; r += kLdWarps * 32) {
-                const int pos = U.base + U.n0 + r;
-                S.rows[r] = GU ? __ldg(a.pair_tok + pos) : pos;
-            }
-            named_sync(kBarLd, kLdWarps * 32);
-            for (int kg = 0; kg < G.KG && ok; ++kg, ++j) {
-                const int slot = j % kABStages;
-                const uint32_t use = j / kABStages;
-                if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
-                    ok = false;
-                    break;
+        // ------------------------------------------------------------ token-row loader (one thread)
+        if (lane == 0 && run) {
+            uint32_t j = 0;
+            bool ok = true;
+            const uint64_t tm = reinterpret_cast<uint64_t>(&tmap);
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+                const Unit U = unit_at(a, u, G.mtiles);
+                const int nb = (U.nr + kRowBox - 1) / kRowBox;
+                for (int kg = 0; kg < G.KG; ++kg, ++j) {
+                    const int slot = j % kABStages;
+                    const uint32_t use = j / kABStages;
+                    if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t Bs = smem_u32(ring + (size_t)slot * stage_bytes + kABytes);
+                    const uint32_t fb = smem_u32(&S.ab_full[slot]);
+                    mbar_expect_tx(fb, (uint32_t)(nb * kRowBox * 128));
+                    // rows past the unit's tokens belong to the next bucket (or lie past the
+                    // matrix and read as zeros); their columns are never used
+                    for (int i = 0; i < nb; ++i)
+                        asm volatile(
+                            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                            ::"r"(Bs + (uint32_t)(i * kRowBox * 128)), "l"(tm), "r"(kg * kGroup),
+                            "r"(U.base + U.n0 + i * kRowBox), "r"(fb)
+                            : "memory");
                 }
-                const uint32_t Bs = smem_u32(ring + (size_t)slot * stage_bytes + kABytes);
-                for (int r = r0; r < U.nr; r += 16) {
-                    const uint32_t dst = Bs + sw128_off(r, c);
-                    if (r < U.nn) cp_async16(dst, a.act + (size_t)S.rows[r] * G.K + kg * kGroup + c * 8, pol);
-                    else cp_async16_zero(dst, a.act);
-                }
-                // arrives on the stage's barrier once this thread's copies have landed
-                cp_async_arrive(smem_u32(&S.ab_full[slot]));
             }
+            // copies still in flight land before the CTA may exit
+            for (uint32_t q = j > (uint32_t)kABStages ? j - kABStages : 0; q < j; ++q)
+                mbar_wait(smem_u32(&S.ab_full[q % kABStages]), (q / kABStages) & 1u, a.wait_ns, a.status);
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         uint32_t j = 0, i = 0;
@@ -511,7 +492,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     ok = false;
                     break;
                 }
-                fence_proxy_async();  // the loaders' cp.async writes of this stage -> the tensor core
                 tc_fence_after();
                 const uint32_t As = smem_u32(ring + (size_t)slot * stage_bytes);
                 if (lane == 0) {
@@ -694,9 +674,9 @@ __global__ void ntile_scan_kernel(const int32_t *counts, int E, int32_t *nt_star
     }
 }
 
-// x16[t] = fp16(x[t] * 2^-xexp[t]) with the per-token exponent chosen so that no value exceeds
-// 2^15 (xexp = 0 unless some |x| >= 2^15); one warp per token.
-__global__ void x16_kernel(const uint16_t *x, int T, int H, uint16_t *x16, int32_t *xexp) {
+// xexp[t]: the exponent that keeps every |x[t] * 2^-xexp[t]| below 2^15 (0 unless some |x| >= 2^15);
+// one warp per token.
+__global__ void xexp_kernel(const uint16_t *x, int T, int H, int32_t *xexp) {
     const int lane = threadIdx.x & 31;
     for (int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += gridDim.x * (blockDim.x / 32)) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
@@ -708,10 +688,20 @@ __global__ void x16_kernel(const uint16_t *x, int T, int H, uint16_t *x16, int32
             for (int j = 0; j < 4; ++j) mx = max(mx, max((w[j] << 16) & 0x7FFFFFFFu, w[j] & 0x7FFF0000u));
         }
         mx = __reduce_max_sync(0xffffffffu, mx);
-        const uint32_t e = (mx >> 23) & 0xFF;
-        const int f = (mx != 0u && (int)e - 127 >= 15) ? (int)e - 127 - 14 : 0;
-        const float sc = exp2i(-f);
-        uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * H);
+        const int e = (int)((mx >> 23) & 0xFF) - 127;
+        if (lane == 0) xexp[t] = (mx != 0u && e >= 15) ? e - 14 : 0;
+    }
+}
+
+// x16[p] = fp16(x[pair_tok[p]] * 2^-xexp[token]) for every pair p in bucket order; one warp per pair.
+__global__ void x16_gather_kernel(const uint16_t *x, const int32_t *pair_tok, const int32_t *xexp, int P, int H,
+                                  uint16_t *x16) {
+    const int lane = threadIdx.x & 31;
+    for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
+        const int t = __ldg(pair_tok + p);
+        const float sc = exp2i(-__ldg(xexp + t));
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)p * H);
         for (int i = lane; i < H / 8; i += 32) {
             const uint4 v = __ldg(src + i);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -723,7 +713,6 @@ __global__ void x16_kernel(const uint16_t *x, int T, int H, uint16_t *x16, int32
             }
             dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        if (lane == 0) xexp[t] = f;
     }
 }
 
@@ -754,8 +743,29 @@ __global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, int P, int
     }
 }
 
+// 2-D tensor map of a row-major fp16 matrix [rows x cols] read in boxes of 64 columns (128 bytes,
+// 128-byte swizzle) by kRowBox rows; rows past the matrix read as zeros.
+bool make_row_map(CUtensorMap *map, const void *base, int rows, int cols) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return false;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kGroup, (cuuint32_t)kRowBox};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool GU>
-moe_status_t launch_tc(const TcArgs &a0, const DeviceInfo *dev, cudaStream_t st) {
+moe_status_t launch_tc(const TcArgs &a0, const CUtensorMap &map, const DeviceInfo *dev, cudaStream_t st) {
     TcArgs a = a0;
     a.smem_bytes = dev->max_smem_optin - (int)sizeof(TcShared) - 2 * kMaxN * 4 - 256;
     static bool attr_set[64] = {};
@@ -767,7 +777,7 @@ moe_status_t launch_tc(const TcArgs &a0, const DeviceInfo *dev, cudaStream_t st)
             return MOE_ERR_CUDA;
         attr_set[d] = true;
     }
-    tc_grouped_kernel<GU><<<(unsigned)dev->sms, kTcThreads, a.smem_bytes, st>>>(a);
+    tc_grouped_kernel<GU><<<(unsigned)dev->sms, kTcThreads, a.smem_bytes, st>>>(a, map);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -782,11 +792,12 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I,
     if (dev == nullptr) return MOE_ERR_CUDA;
     if (I / 16 > kMaxSub) return MOE_ERR_UNSUPPORTED;
     const size_t P = (size_t)T * k;
+    CUtensorMap xmap, hmap;
+    if (!make_row_map(&xmap, x16, (int)P, H) || !make_row_map(&hmap, h16, (int)P, I)) return MOE_ERR_CUDA;
     ntile_scan_kernel<<<1, 1024, 0, st>>>(counts, E, nt_start);
-    {
-        const unsigned blocks = (unsigned)((T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096);
-        x16_kernel<<<blocks, 256, 0, st>>>(x, T, H, x16, xexp);
-    }
+    xexp_kernel<<<(unsigned)((T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096), 256, 0, st>>>(x, T, H, xexp);
+    x16_gather_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(x, pair_tok, xexp, (int)P,
+                                                                                           H, x16);
     TcArgs a{};
     a.packed = packed;
     a.H = H;
@@ -805,11 +816,11 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I,
     a.wait_ns = wait_limit_ns();
     a.status = status;
     a.act = x16;
-    moe_status_t s = launch_tc<true>(a, dev, st);
+    moe_status_t s = launch_tc<true>(a, xmap, dev, st);
     if (s != MOE_OK) return s;
     h16_rescale_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(h16, hexp, (int)P, I, fexp);
     a.act = h16;
-    s = launch_tc<false>(a, dev, st);
+    s = launch_tc<false>(a, hmap, dev, st);
     if (s != MOE_OK) return s;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
