@@ -300,26 +300,6 @@ struct Geometry {
     }
 };
 
-// Where one dequantiser warp's packed tile of a K step lives (nullptr: the row block is past
-// the matrix, which happens in the last M tile of a down matrix with H % 128 == 64).
-struct DqStep {
-    const uint8_t *tile;
-    int bits;
-};
-template <bool GU>
-__device__ __forceinline__ DqStep dq_step(const TcArgs &a, const Geometry<GU> &G, const Unit &U, int b, int kg) {
-    DqStep d;
-    const PackedExpert pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader))[U.e];
-    d.bits = pe.bits;
-    const int rb = 8 * U.mt + b;
-    if (rb >= G.nrb) {
-        d.tile = nullptr;
-        return d;
-    }
-    d.tile = a.packed + pe.offset + (G.skip_tiles + (size_t)rb * G.KG + kg) * tile_bytes(pe.bits);
-    return d;
-}
-
 // 2^d as an fp16 pair for d <= 0 (subnormal below 2^-14, zero below 2^-24)
 __device__ __forceinline__ uint32_t h2_pow2(int d) {
     uint32_t b = 0;
@@ -401,8 +381,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         const int b = warp;
         uint32_t j = 0;
         bool ok = run;
+        const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
+            // per unit: the expert's width and whether this warp's row block exists
+            const int bits = __ldg(&pe[U.e].bits);
+            const int tb = tile_bytes(bits);
+            const bool have = 8 * U.mt + b < G.nrb;
             for (int kg = 0; kg < G.KG; ++kg, ++j) {
                 const uint32_t chunk = j / KC;
                 const uint32_t rs = chunk % R;
@@ -417,9 +402,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 uint8_t *As = ring + (size_t)slot * stage_bytes;
-                const DqStep d = dq_step<GU>(a, G, U, b, kg);
-                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + (int)(j % KC)) * tile_bytes(d.bits);
-                if (d.tile == nullptr) {
+                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + (int)(j % KC)) * tb;
+                if (!have) {
                     // row block past the matrix: zero rows (the epilogue skips them)
                     const uint4 z = make_uint4(0, 0, 0, 0);
                     const int g = lane >> 2, t = lane & 3;
@@ -427,9 +411,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t + 1)) = z;
                     *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t)) = z;
                     *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t + 1)) = z;
-                } else if (d.bits == 4) {
+                } else if (bits == 4) {
                     dequant_fragment<4>(rawt, lane, As, b);
-                } else if (d.bits == 8) {
+                } else if (bits == 8) {
                     dequant_fragment<8>(rawt, lane, As, b);
                 } else {
                     dequant_fragment<6>(rawt, lane, As, b);
