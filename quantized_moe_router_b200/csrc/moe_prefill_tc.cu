@@ -198,14 +198,8 @@ __device__ __forceinline__ float nib_float(uint32_t m, uint32_t sel) {
 }
 // (x0 * S + C, x1 * S + C) with one packed fp32x2 FMA, rounded to an fp16 pair (x0 in the low half)
 __device__ __forceinline__ uint32_t fma2_h(float x0, float x1, float S, float C) {
-    float r0, r1;
-    asm("{ .reg .b64 a, b, c, d;\n\t"
-        "mov.b64 a, {%2, %3}; mov.b64 b, {%4, %4}; mov.b64 c, {%5, %5};\n\t"
-        "fma.rn.f32x2 d, a, b, c;\n\t"
-        "mov.b64 {%0, %1}, d; }"
-        : "=f"(r0), "=f"(r1)
-        : "f"(x0), "f"(x1), "f"(S), "f"(C));
-    const __half2 v = __floats2half2_rn(r0, r1);
+    const float2 r = __ffma2_rn(make_float2(x0, x1), make_float2(S, S), make_float2(C, C));
+    const __half2 v = __floats2half2_rn(r.x, r.y);
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 // x * S + y * S2 + C for two elements (6/8-bit codes: the low and the high code plane)
