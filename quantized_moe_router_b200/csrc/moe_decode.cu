@@ -65,6 +65,9 @@ struct DecodeArgs {
     float *out_acc;
     uint32_t *h_ready;
     uint64_t wait_ns;
+    double rnC;     // 1 / number of CTAs
+    int lrep;       // copies of the logit words (a power of two)
+    int lstride;    // words between copies
 };
 
 struct __align__(16) DecodeSmem {
@@ -93,6 +96,8 @@ struct __align__(16) DecodeSmem {
     float pw[kMaxP];
     int sel_idx[kMaxP];
     float sel_w[kMaxP];
+    float lpart[kWarps];                // slice sums of the router dot products
+    __align__(16) uint32_t plist[32];   // plan scratch: packed pair list
 };
 
 // accumulator slots of NT n-tiles: 16 rows x 8*NT columns fp32, laid out as the MMA fragments
@@ -265,8 +270,11 @@ __device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const 
     const float sA = keep * half_lo(sz.x), zA = half_hi(sz.x), sB = keep * half_lo(sz.y), zB = half_hi(sz.y);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+        // Up to two n-tiles every lane loads: a column without a token reads a valid row (the
+        // first pair's) and produces accumulator columns that nothing reads, with no divergent
+        // branch per tile. Four n-tiles keep the guard (their registers are tight).
         uint32_t b[8] = {0, 0, 0, 0, 0, 0, 0, 0}, b2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (jc.has[nt]) {
+        if (NT <= 2 || jc.has[nt]) {
             uint4 v0, v1, w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
             if (jc.bg) {
                 const uint4 *p = reinterpret_cast<const uint4 *>(jc.b[nt] + kg * kGroup + 16 * t);
@@ -291,8 +299,8 @@ __device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const 
             b2[0] = w0.x; b2[1] = w0.y; b2[2] = w0.z; b2[3] = w0.w;
             b2[4] = w1.x; b2[5] = w1.y; b2[6] = w1.z; b2[7] = w1.w;
         }
-        const float X0 = jc.has0[nt] ? lds32f(jc.xs0[nt] + kg * 4) : 0.f;
-        const float X1 = jc.has1[nt] ? lds32f(jc.xs1[nt] + kg * 4) : 0.f;
+        const float X0 = (NT <= 2 || jc.has0[nt]) ? lds32f(jc.xs0[nt] + kg * 4) : 0.f;
+        const float X1 = (NT <= 2 || jc.has1[nt]) ? lds32f(jc.xs1[nt] + kg * 4) : 0.f;
         tile_group_mma<BITS>(lo, hi8, hi6, b, GU ? nullptr : b2, sA, zA, sB, zB, X0, X1, acc[nt]);
     }
 }
@@ -325,14 +333,49 @@ __device__ __forceinline__ void run_tiles(const uint8_t *job_base, int tb, int k
 }
 
 // ------------------------------------------------------------------------------ routing
-// Token t's top-k from the exchanged logit words (M words per lane, E <= 32 M): polls until
-// every word carries `tag`, then selects (larger logit first, equal logits -> lower index, NaN
-// as -inf) and forms the softmax over the selected logits. Lane i < k receives the i-th expert
-// and its weight. Returns false (warp-uniformly) when the wait expires.
+// Largest key of a lane's M keys and its position; on equal keys the lower position (the lower
+// expert index) wins, since a tournament node keeps its left entry unless the right one is larger.
 template <int M>
-__device__ bool token_topk(const DecodeArgs &a, int t, uint32_t tag, int lane, int &idx, float &w) {
-    const unsigned long long *row = a.logits + (size_t)t * a.E;
-    uint32_t key[M];
+__device__ __forceinline__ void lane_best(const uint32_t (&key)[M], uint32_t &bk, int &bm) {
+    uint32_t k2[M];
+    int m2[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        k2[i] = key[i];
+        m2[i] = i;
+    }
+#pragma unroll
+    for (int w = 1; w < M; w <<= 1)
+#pragma unroll
+        for (int i = 0; i + w < M; i += 2 * w)
+            if (k2[i + w] > k2[i]) {
+                k2[i] = k2[i + w];
+                m2[i] = m2[i + w];
+            }
+    bk = k2[0];
+    bm = m2[0];
+}
+
+// One comparator of a descending sort of (key, position) pairs: equal keys keep the lower
+// position (the lower expert index) first.
+// Written with selects: a divergent branch per comparator costs far more than the swap.
+__device__ __forceinline__ void sort_ce(uint32_t &ki, int &mi, uint32_t &kj, int &mj) {
+    const bool sw = (kj > ki) | ((kj == ki) & (mj < mi));
+    const uint32_t k0 = sw ? kj : ki, k1 = sw ? ki : kj;
+    const int m0 = sw ? mj : mi, m1 = sw ? mi : mj;
+    ki = k0;
+    kj = k1;
+    mi = m0;
+    mj = m1;
+}
+
+// Polls token t's exchanged logit words (M per lane: expert lane + 32 m) until every word
+// carries `tag`, as order keys (0 where absent; NaN as -inf). False (warp-uniformly) when the
+// wait expires.
+template <int M>
+__device__ __forceinline__ bool poll_keys(const DecodeArgs &a, int t, uint32_t tag, int lane, uint32_t (&key)[M]) {
+    const unsigned long long *row =
+        a.logits + (size_t)(blockIdx.x & (unsigned)(a.lrep - 1)) * a.lstride + (size_t)t * a.E;
     uint64_t t0 = 0;
     for (int it = 0;; ++it) {
         bool ok = true;
@@ -349,7 +392,7 @@ __device__ bool token_topk(const DecodeArgs &a, int t, uint32_t tag, int lane, i
             }
             key[m] = kk;
         }
-        if (__all_sync(0xffffffffu, ok)) break;
+        if (__all_sync(0xffffffffu, ok)) return true;
         int expired = 0;
         if (lane == 0) {
             const uint64_t now = global_timer();
@@ -360,39 +403,143 @@ __device__ bool token_topk(const DecodeArgs &a, int t, uint32_t tag, int lane, i
         if (__shfl_sync(0xffffffffu, expired, 0)) return false;
         __nanosleep(32);
     }
-    uint32_t bk = 0;
-    int bm = 0;
-#pragma unroll
-    for (int m = 0; m < M; ++m)
-        if (key[m] > bk) { bk = key[m]; bm = m; }
-    int my_i = -1;
-    uint32_t my_k = 0;
-    for (int r = 0; r < a.k; ++r) {
+}
+
+// The softmax weights of a selection, from the rounds' maxima in round order (every lane sees
+// them all): lane r < k keeps exp(l_r - l_0), and the sum runs over the rounds in order.
+struct SoftmaxAcc {
+    float v0 = 0.f, s = 0.f, my_e = 0.f;
+    __device__ __forceinline__ void add(uint32_t mx, int r, int lane) {
+        const float v = key_value(mx);
+        v0 = (r == 0) ? v : v0;
+        const float ex = (v0 == -INFINITY) ? 1.f : expf(v - v0);
+        s += ex;
+        my_e = (lane == r) ? ex : my_e;
+    }
+};
+__device__ __forceinline__ void store_weights(const DecodeArgs &a, DecodeSmem &S, int t, int lane, int c,
+                                              const SoftmaxAcc &sm) {
+    if (lane < a.k) {
+        const float w = sm.my_e / sm.s;
+        S.sel_w[t * a.k + lane] = w;
+        if (c == 0 && a.w_out) a.w_out[t * a.k + lane] = w;
+    }
+}
+
+// Exact selection (larger logit first, equal logits -> lower index) of token t, up to 1024
+// experts: each round the maximum key, then the lowest index holding it; the winning lane
+// rescans its keys. Out of line: it serves wide expert counts and ties of the fast selection.
+__device__ __noinline__ bool token_topk_wide(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t tag, int lane, int c) {
+    uint32_t key[32];
+    if (!poll_keys<32>(a, t, tag, lane, key)) return false;
+    const int K = a.k;
+    SoftmaxAcc sm;
+    uint32_t bk;
+    int bm;
+    lane_best<32>(key, bk, bm);
+    for (int r = 0; r < K; ++r) {
         const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
-        const uint32_t cand = (bk == mx) ? (uint32_t)(lane + 32 * bm) : 0xFFFFFFFFu;
-        const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-        if (lane == r) { my_i = (int)win; my_k = mx; }
+        const uint32_t win = __reduce_min_sync(0xffffffffu, bk == mx ? (uint32_t)(lane + 32 * bm) : 0xFFFFFFFFu);
+        if (lane == r) {
+            S.sel_idx[t * K + r] = (int)win;
+            if (c == 0 && a.idx_out) a.idx_out[t * K + r] = (int)win;
+        }
         if ((int)(win & 31u) == lane) {
 #pragma unroll
-            for (int m = 0; m < M; ++m)
+            for (int m = 0; m < 32; ++m)
                 if (m == bm) key[m] = 0;
-            bk = 0;
-            bm = 0;
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-                if (key[m] > bk) { bk = key[m]; bm = m; }
+            lane_best<32>(key, bk, bm);
         }
+        sm.add(mx, r, lane);
     }
-    const float my_v = (lane < a.k) ? key_value(my_k) : -INFINITY;
-    const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-    float ex = 0.f;
-    if (lane < a.k) ex = (v0 == -INFINITY) ? 1.f : expf(my_v - v0);
-    float s = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    idx = my_i;
-    w = (lane < a.k) ? ex / s : 0.f;
+    store_weights(a, S, t, lane, c, sm);
     return true;
+}
+
+// Top-k of token t (E <= 256: 8 keys per lane), written to S.sel_idx / S.sel_w[t * k + i] (and
+// idx_out / w_out from CTA 0); false (warp-uniformly) when the wait for the logits expires.
+// Each lane sorts its keys once (equal keys: lower index first); a round takes the maximum of
+// the lanes' heads and the lane holding it pops its head, a register shift. When two lanes hold
+// that maximum the exact routine redoes the selection.
+__device__ bool token_topk(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t tag, int lane, int c) {
+    uint32_t sk[8];
+    if (!poll_keys<8>(a, t, tag, lane, sk)) return false;
+    int sm_[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) sm_[m] = m;
+    sort_ce(sk[0], sm_[0], sk[2], sm_[2]); sort_ce(sk[1], sm_[1], sk[3], sm_[3]);
+    sort_ce(sk[4], sm_[4], sk[6], sm_[6]); sort_ce(sk[5], sm_[5], sk[7], sm_[7]);
+    sort_ce(sk[0], sm_[0], sk[4], sm_[4]); sort_ce(sk[1], sm_[1], sk[5], sm_[5]);
+    sort_ce(sk[2], sm_[2], sk[6], sm_[6]); sort_ce(sk[3], sm_[3], sk[7], sm_[7]);
+    sort_ce(sk[0], sm_[0], sk[1], sm_[1]); sort_ce(sk[2], sm_[2], sk[3], sm_[3]);
+    sort_ce(sk[4], sm_[4], sk[5], sm_[5]); sort_ce(sk[6], sm_[6], sk[7], sm_[7]);
+    sort_ce(sk[2], sm_[2], sk[4], sm_[4]); sort_ce(sk[3], sm_[3], sk[5], sm_[5]);
+    sort_ce(sk[1], sm_[1], sk[4], sm_[4]); sort_ce(sk[3], sm_[3], sk[6], sm_[6]);
+    sort_ce(sk[1], sm_[1], sk[2], sm_[2]); sort_ce(sk[3], sm_[3], sk[4], sm_[4]);
+    sort_ce(sk[5], sm_[5], sk[6], sm_[6]);
+    const int K = a.k;
+    SoftmaxAcc sm;
+    uint32_t tied = 0;
+    int *sel = S.sel_idx + t * K;
+    for (int r = 0; r < K; ++r) {
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, sk[0]);
+        const bool win = sk[0] == mx;
+        const uint32_t b = __ballot_sync(0xffffffffu, win);
+        tied |= b & (b - 1u);
+        if (win) sel[r] = lane + 32 * sm_[0];
+        // the winner shifts its list (selects, no branch)
+#pragma unroll
+        for (int m = 0; m < 7; ++m) {
+            sk[m] = win ? sk[m + 1] : sk[m];
+            sm_[m] = win ? sm_[m + 1] : sm_[m];
+        }
+        sk[7] = win ? 0u : sk[7];
+        sm.add(mx, r, lane);
+    }
+    if (tied) return token_topk_wide(a, S, t, tag, lane, c);
+    __syncwarp();
+    if (c == 0 && a.idx_out && lane < K) a.idx_out[t * K + lane] = sel[lane];
+    store_weights(a, S, t, lane, c, sm);
+    return true;
+}
+
+// floor(X * cc / nC) without an integer division: the quotient taken through the double
+// reciprocal of nC (X * cc < 2^53 is exact in double, and the estimate is floor or floor - 1)
+// and corrected once.
+__device__ __forceinline__ uint32_t cut_units(uint32_t X, int cc, int nC, double rnC) {
+    const unsigned long long n = (unsigned long long)X * (unsigned)cc;
+    unsigned long long q = (unsigned long long)((double)n * rnC);
+    q += ((q + 1ull) * (unsigned)nC <= n) ? 1ull : 0ull;
+    return (uint32_t)q;
+}
+// Smallest r with r * d >= n, for results below 2^16: the truncated float quotient (relative
+// error below 2^-20, so within 0.07 of n / d) is floor(n / d) - 1, floor(n / d) or ceil(n / d),
+// and two conditional increments reach ceil(n / d).
+__device__ __forceinline__ uint32_t ceil_div_small(uint32_t n, uint32_t d) {
+    uint32_t r = (uint32_t)__fdividef((float)n, (float)d);
+    r += ((unsigned long long)r * d < n) ? 1u : 0u;
+    r += ((unsigned long long)r * d < n) ? 1u : 0u;
+    return r;
+}
+// First job (of a gate/up or down sequence) whose first unit is at or after q, found by the
+// lanes of a warp of which some hold one expert slot each (U <= 32 slots, in any lane order):
+// such a lane holds the slot's index, its first unit lo, its end hi and its units per job jb;
+// `per` jobs per slot, `total` units in all. The slot holding q is the one with lo < q <= hi
+// (slot 0 for q = 0). `start` receives the job's first unit (total past the last job).
+__device__ __forceinline__ int job_at_unit_warp(uint32_t lo, uint32_t hi, uint32_t jb, int slot, bool slot_lane,
+                                                int per, int U, uint32_t q, uint32_t total, uint32_t &start) {
+    const bool holds = slot_lane && (q == 0 ? lo == 0 : (lo < q && q <= hi));
+    const uint32_t m = __ballot_sync(0xffffffffu, holds);
+    const uint32_t r = holds ? ceil_div_small(q - lo, jb) : 0u;
+    const uint32_t st = lo + r * jb;
+    const int j = slot * per + (int)r;
+    if (m == 0) {
+        start = total;
+        return U * per;
+    }
+    const int u = __ffs(m) - 1;
+    start = __shfl_sync(0xffffffffu, st, u);
+    return __shfl_sync(0xffffffffu, j, u);
 }
 
 __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
@@ -400,181 +547,239 @@ __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
     return S.wordpre[w] + __popc(S.selmask[w] & ((1u << (e & 31)) - 1u));
 }
 
-// The plan, by one warp: unique experts in ascending id (slots), each slot's pair list in
-// ascending pair id (token-major, so ascending token), byte prefixes of the gate/up and down
-// job sequences, and this CTA's job ranges. P = 0 (an aborted routing) gives an empty plan.
-__device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
+// Plan for more than 32 pairs (several tokens), out of line: bitmap of the selection in shared
+// memory, per-slot counts and a stable fill of the pair lists 32 slots at a time, and the job
+// ranges by binary search over the slots' unit prefixes.
+__device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
     const int K = a.k, E = a.E, H = a.H, I = a.I;
-    const int G = H / kGroup, GI = I / kGroup;
-    if (P <= 32) {
-        const bool v = lane < P;
-        const int e = v ? S.sel_idx[lane] : 0x7FFFFFFF;
-        const uint32_t same = __match_any_sync(0xffffffffu, e);
-        const bool first = v && (__ffs(same) - 1 == lane);
-        int *tmp = S.cursor;
-        tmp[lane] = first ? e : (v ? -1 - e : 0x7FFFFFFF);    // >= 0: first occurrence of an expert
-        __syncwarp();
-        int slot = 0, before = 0;                             // distinct experts / pairs with a smaller id
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-            const int ej = tmp[j];
-            const int id = ej >= 0 ? ej : -1 - ej;
-            if (ej != 0x7FFFFFFF && id < e) {
-                ++before;
-                slot += ej >= 0 ? 1 : 0;
-            }
-        }
-        const int U = __popc(__ballot_sync(0xffffffffu, first));
-        if (first) {
-            S.ubits[slot] = S.ebits[e];
-            S.uoff[slot] = S.eoff[e];
-            S.pfirst[slot] = before;
-        }
-        if (v) {
-            const int pos = before + __popc(same & ((1u << lane) - 1u));
-            S.ppair[pos] = lane;
-            S.ptok[pos] = lane / K;
-            S.pw[pos] = S.sel_w[lane];
-        }
-        __syncwarp();
-        const uint32_t ts = (lane < U) ? (uint32_t)tile_bytes(S.ubits[lane]) / 64 : 0;   // 64-byte units per tile
-        const uint32_t bg = ts * (uint32_t)(I / 8) * G, bd = ts * (uint32_t)(H / 16) * GI;
-        uint32_t ig = bg, id = bd;
+    const int G = H / kGroup;
+    const int pg = I / 8, pd = H / 16;
+    const uint32_t ug = (uint32_t)pg * (uint32_t)G;
+    int U;
+    uint32_t GUB;
+    // Many pairs: bitmap of the selection in shared memory, per-slot counts and a stable
+    // fill of the pair lists, 32 slots per pass.
+    for (int i = lane; i < kMaxE / 32; i += 32) S.selmask[i] = 0;
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) atomicOr(&S.selmask[S.sel_idx[p] >> 5], 1u << (S.sel_idx[p] & 31));
+    __syncwarp();
+    {
+        const int words = (E + 31) / 32;
+        const int n = (lane < words) ? __popc(S.selmask[lane]) : 0;
+        int incl = n;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t og = __shfl_up_sync(0xffffffffu, ig, off);
-            const uint32_t od = __shfl_up_sync(0xffffffffu, id, off);
-            if (lane >= off) {
-                ig += og;
-                id += od;
-            }
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
         }
-        if (lane < U) {
-            S.cgu[lane] = ig - bg;
-            S.cd[lane] = id - bd;
-        }
-        if (lane == U - 1) {
-            S.cgu[U] = ig;
-            S.cd[U] = id;
-        }
-        if (lane == 0) {
-            S.U = U;
-            S.pfirst[U] = P;
-            if (U == 0) S.cgu[0] = S.cd[0] = 0;
-        }
-        __syncwarp();
-    } else {
-        for (int i = lane; i < kMaxE / 32; i += 32) S.selmask[i] = 0;
-        __syncwarp();
-        for (int p = lane; p < P; p += 32) atomicOr(&S.selmask[S.sel_idx[p] >> 5], 1u << (S.sel_idx[p] & 31));
-        __syncwarp();
-        {
-            const int words = (E + 31) / 32;
-            const int n = (lane < words) ? __popc(S.selmask[lane]) : 0;
-            int incl = n;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            S.wordpre[lane] = incl - n;
-            if (lane == 31) S.U = incl;
-        }
-        __syncwarp();
-        const int U = S.U;
-        for (int u = lane; u < U; u += 32) S.cnt[u] = 0;
-        __syncwarp();
-        for (int p = lane; p < P; p += 32) {
-            const int e = S.sel_idx[p];
-            const int u = slot_of(S, e);
-            S.ubits[u] = S.ebits[e];
-            S.uoff[u] = S.eoff[e];
-            atomicAdd(&S.cnt[u], 1);
-        }
-        __syncwarp();
-        int carry = 0;
-        uint32_t cg = 0, cdd = 0;
-        for (int base = 0; base < U; base += 32) {
-            const int u = base + lane;
-            const int n = (u < U) ? S.cnt[u] : 0;
-            const uint32_t tu = (u < U) ? (uint32_t)tile_bytes(S.ubits[u]) / 64 : 0;
-            const uint32_t bg = tu * (uint32_t)(I / 8) * G, bd = tu * (uint32_t)(H / 16) * GI;
-            int incl = n;
-            uint32_t ig = bg, id = bd;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                const uint32_t og = __shfl_up_sync(0xffffffffu, ig, off);
-                const uint32_t od = __shfl_up_sync(0xffffffffu, id, off);
-                if (lane >= off) {
-                    incl += o;
-                    ig += og;
-                    id += od;
-                }
-            }
-            if (u < U) {
-                S.pfirst[u] = carry + incl - n;
-                S.cursor[u] = carry + incl - n;
-                S.cgu[u] = cg + ig - bg;
-                S.cd[u] = cdd + id - bd;
-            }
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-            cg += __shfl_sync(0xffffffffu, ig, 31);
-            cdd += __shfl_sync(0xffffffffu, id, 31);
-        }
-        if (lane == 0) {
-            S.pfirst[U] = carry;
-            S.cgu[U] = cg;
-            S.cd[U] = cdd;
-        }
-        __syncwarp();
-        // stable fill: pairs in ascending pair id order
-        for (int base = 0; base < P; base += 32) {
-            const int p = base + lane;
-            const int u = (p < P) ? slot_of(S, S.sel_idx[p]) : -1 - lane;
-            const uint32_t peers = __match_any_sync(0xffffffffu, u);
-            const int rank = __popc(peers & ((1u << lane) - 1u));
-            if (p < P) {
-                const int pos = S.cursor[u] + rank;
-                S.ppair[pos] = p;
-                S.ptok[pos] = p / K;
-                S.pw[pos] = S.sel_w[p];
-            }
-            __syncwarp();
-            if (p < P && rank == 0) S.cursor[u] += __popc(peers);
-            __syncwarp();
-        }
+        S.wordpre[lane] = incl - n;
+        if (lane == 31) S.U = incl;
     }
     __syncwarp();
-    // Job ranges: the gate/up sequence is cut at multiples of its bytes / nCTA; the down sequence
-    // is cut so that each CTA's gate/up + down bytes are the layer's bytes / nCTA. That cut is
-    // monotone in the CTA index when every CTA's down share exceeds one gate/up job (plus
-    // rounding); otherwise (tiny layers) the down sequence is cut on its own.
-    // 32-bit arithmetic: floor(X * c / nC) = (X / nC) * c + ((X % nC) * c) / nC
-    const int Uj = S.U;
-    const int pg = I / 8, pd = H / 16;
-    const uint32_t GUB = S.cgu[Uj], DB = S.cd[Uj], B = GUB + DB;
-    auto cut = [&](uint32_t X, int cc) -> uint32_t {
-        return (X / nC) * (uint32_t)cc + ((X % nC) * (uint32_t)cc) / nC;
-    };
-    uint32_t mj = 0;                        // largest gate/up job (64-byte units)
-    for (int u = lane; u < Uj; u += 32) mj = max(mj, (S.cgu[u + 1] - S.cgu[u]) / pg);
+    U = S.U;
+    for (int u = lane; u < U; u += 32) S.cnt[u] = 0;
+    __syncwarp();
+    for (int p = lane; p < P; p += 32) {
+        const int e = S.sel_idx[p];
+        const int u = slot_of(S, e);
+        S.ubits[u] = S.ebits[e];
+        S.uoff[u] = S.eoff[e];
+        atomicAdd(&S.cnt[u], 1);
+    }
+    __syncwarp();
+    int carry = 0;
+    uint32_t cts = 0;
+    for (int base = 0; base < U; base += 32) {
+        const int u = base + lane;
+        const int n = (u < U) ? S.cnt[u] : 0;
+        const uint32_t tu = (u < U) ? (uint32_t)tile_bytes(S.ubits[u]) / 64u : 0u;
+        int incl = n;
+        uint32_t it = tu;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            const uint32_t ot = __shfl_up_sync(0xffffffffu, it, off);
+            if (lane >= off) {
+                incl += o;
+                it += ot;
+            }
+        }
+        if (u < U) {
+            S.pfirst[u] = carry + incl - n;
+            S.cursor[u] = carry + incl - n;
+            S.cgu[u] = (cts + it - tu) * ug;
+            S.cd[u] = (cts + it - tu) * ug / 2u;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        cts += __shfl_sync(0xffffffffu, it, 31);
+    }
+    GUB = cts * ug;
+    if (lane == 0) {
+        S.pfirst[U] = carry;
+        S.cgu[U] = GUB;
+        S.cd[U] = GUB >> 1;
+    }
+    __syncwarp();
+    // stable fill: pairs in ascending pair id order
+    for (int base = 0; base < P; base += 32) {
+        const int p = base + lane;
+        const int u = (p < P) ? slot_of(S, S.sel_idx[p]) : -1 - lane;
+        const uint32_t peers = __match_any_sync(0xffffffffu, u);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        if (p < P) {
+            const int pos = S.cursor[u] + rank;
+            S.ppair[pos] = p;
+            S.ptok[pos] = p / K;
+            S.pw[pos] = S.sel_w[p];
+        }
+        __syncwarp();
+        if (p < P && rank == 0) S.cursor[u] += __popc(peers);
+        __syncwarp();
+    }
+    const uint32_t DB = GUB >> 1, B = GUB + DB;
+    int g0, g1, d0, d1;
+    uint32_t mj = 0;   // largest gate/up job (units)
+    for (int u = lane; u < U; u += 32) mj = max(mj, (S.cgu[u + 1] - S.cgu[u]) / pg);
     mj = __reduce_max_sync(0xffffffffu, mj);
-    const bool mono = (uint64_t)(mj + 2) * nC <= DB;
+    const bool mono = (unsigned long long)(mj + 2u) * (unsigned)nC <= DB;
     int gcut = 0;
     if (lane < 2) {
         const int cc = c + lane;
-        gcut = (cc >= nC) ? Uj * pg : job_at_unit(S.cgu, Uj, pg, cut(GUB, cc));
+        gcut = (cc >= nC) ? U * pg : job_at_unit(S.cgu, U, pg, cut_units(GUB, cc, nC, a.rnC));
     }
-    const int g0 = __shfl_sync(0xffffffffu, gcut, 0), g1 = __shfl_sync(0xffffffffu, gcut, 1);
+    g0 = __shfl_sync(0xffffffffu, gcut, 0);
+    g1 = __shfl_sync(0xffffffffu, gcut, 1);
     int dcut = 0;
     if (lane < 2) {
         const int cc = c + lane;
         const int gj = lane == 0 ? g0 : g1;
-        const uint32_t pos = mono ? cut(B, cc) - job_start_unit(S.cgu, Uj, pg, gj) : cut(DB, cc);
-        dcut = (cc >= nC) ? Uj * pd : job_at_unit(S.cd, Uj, pd, pos);
+        const uint32_t pos = mono ? cut_units(B, cc, nC, a.rnC) - job_start_unit(S.cgu, U, pg, gj)
+                                  : cut_units(DB, cc, nC, a.rnC);
+        dcut = (cc >= nC) ? U * pd : job_at_unit(S.cd, U, pd, pos);
     }
-    const int d0 = __shfl_sync(0xffffffffu, dcut, 0), d1 = __shfl_sync(0xffffffffu, dcut, 1);
+    d0 = __shfl_sync(0xffffffffu, dcut, 0);
+    d1 = __shfl_sync(0xffffffffu, dcut, 1);
+    if (lane == 0) {
+        S.g0 = g0;
+        S.g1 = g1;
+        S.d0 = d0;
+        S.d1 = d1;
+        S.nGU = g1 - g0;
+    }
+    __syncwarp();
+}
+
+// The plan, by one warp: unique experts in ascending id (slots), each slot's pair list in
+// ascending pair id (token-major, so ascending token), unit prefixes of the gate/up and down
+// job sequences, and this CTA's job ranges. P = 0 (an aborted routing) gives an empty plan.
+// A 64-byte unit is the granule of the job sequences: a tile of `bits` is tile_bytes(bits) / 64
+// units, a gate/up job G tiles and a down job GI tiles, so that an expert's down units are
+// exactly half its gate/up units.
+__device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
+    if (P > 32) {
+        make_plan_many(a, S, P, lane, c, nC);
+        return;
+    }
+    const int K = a.k, H = a.H, I = a.I;
+    const int G = H / kGroup, GI = I / kGroup;
+    const int pg = I / 8, pd = H / 16;
+    const uint32_t ug = (uint32_t)pg * (uint32_t)G;   // gate/up units of an expert per unit of tile size
+    int U;
+    uint32_t GUB;                      // gate/up units of all slots
+    uint32_t lo, hi, ts;               // slot lanes: the slot's gate/up units [lo, hi), units per tile
+    int slot;                          // slot of the lane's expert
+    bool slot_lane;                    // the lane holds the first pair of its expert
+    uint32_t mts;                      // largest units per tile over the slots
+    {
+        // One pair per lane. Each lane counts, over a packed list of all pairs {expert, units
+        // per tile, first pair of its expert}, the distinct experts below its own (its slot),
+        // their units and the pairs below it; the totals come out of the same pass.
+        const bool v = lane < P;
+        const int e = v ? S.sel_idx[lane] : 0;
+        const float pw = v ? S.sel_w[lane] : 0.f;
+        const int eb = S.ebits[e];
+        const uint32_t eo = S.eoff[e];
+        const uint32_t tsl = (uint32_t)tile_bytes(eb) / 64u;
+        uint32_t same = 1u << lane;   // one token: its experts are distinct
+        if (a.T > 1) same = __match_any_sync(0xffffffffu, v ? e : -1 - lane);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        const bool first = v && rank == 0;
+        // entries past P: an id above every expert, no units, not first
+        S.plist[lane] = v ? ((uint32_t)e | (tsl << 16) | (first ? 0x80000000u : 0u)) : 0xFFFFu;
+        __syncwarp();
+        uint32_t nsl = 0, units = 0, pbelow = 0, nU = 0, tot = 0;
+        mts = 0;
+        const uint4 *pl = reinterpret_cast<const uint4 *>(S.plist);
+        for (int q4 = 0; q4 < (P + 3) / 4; ++q4) {
+            const uint4 w4 = pl[q4];
+            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t w = ws[j];
+                const bool lt = (w & 0xFFFFu) < (uint32_t)e;
+                const uint32_t tq = (w >> 31) ? (w >> 16) & 0x7FFFu : 0u;   // units of a first entry
+                pbelow += lt ? 1u : 0u;
+                nsl += (lt && tq) ? 1u : 0u;
+                units += lt ? tq : 0u;
+                nU += tq ? 1u : 0u;
+                tot += tq;
+                mts = max(mts, tq);
+            }
+        }
+        U = (int)nU;
+        slot = (int)nsl;
+        slot_lane = first;
+        ts = tsl;
+        lo = units * ug;
+        hi = lo + tsl * ug;
+        GUB = tot * ug;
+        if (first) {
+            S.ubits[slot] = eb;
+            S.uoff[slot] = eo;
+            S.pfirst[slot] = (int)pbelow;
+            S.cgu[slot] = lo;
+            S.cd[slot] = lo >> 1;
+        }
+        if (v) {
+            const int pos = (int)pbelow + rank;
+            S.ppair[pos] = lane;
+            S.ptok[pos] = lane / K;
+            S.pw[pos] = pw;
+        }
+        if (lane == 0) {
+            S.U = U;
+            S.pfirst[U] = P;
+            S.cgu[U] = GUB;
+            S.cd[U] = GUB >> 1;
+        }
+    }
+    // Job ranges. The gate/up sequence is cut at multiples of its units / nCTA; the down
+    // sequence is cut so that each CTA's gate/up + down units are the layer's units / nCTA. That
+    // cut is monotone in the CTA index when every CTA's down share exceeds one gate/up job (plus
+    // rounding); otherwise (tiny layers) the down sequence is cut on its own.
+    const uint32_t DB = GUB >> 1, B = GUB + DB;
+    int g0, g1, d0, d1;
+    {
+        const uint32_t jbg = ts * (uint32_t)G, jbd = ts * (uint32_t)GI;   // units per job of the lane's slot
+        const uint32_t mj = mts * (uint32_t)G;                            // largest gate/up job
+        const bool mono = (unsigned long long)(mj + 2u) * (unsigned)nC <= DB;
+        uint32_t st0, st1, unused;
+        g0 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(GUB, c, nC, a.rnC), GUB, st0);
+        if (c + 1 < nC) {
+            g1 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(GUB, c + 1, nC, a.rnC), GUB, st1);
+        } else {
+            g1 = U * pg;
+            st1 = GUB;
+        }
+        const uint32_t q0 = mono ? cut_units(B, c, nC, a.rnC) - st0 : cut_units(DB, c, nC, a.rnC);
+        d0 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q0, DB, unused);
+        if (c + 1 < nC) {
+            const uint32_t q1 = mono ? cut_units(B, c + 1, nC, a.rnC) - st1 : cut_units(DB, c + 1, nC, a.rnC);
+            d1 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q1, DB, unused);
+        } else {
+            d1 = U * pd;
+        }
+    }
     if (lane == 0) {
         S.g0 = g0;
         S.g1 = g1;
@@ -641,7 +846,7 @@ __device__ __forceinline__ void finalize_down(const DecodeArgs &a, const DecodeS
 
 // ------------------------------------------------------------------------------ kernel
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a, const DecodeLayout L) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a, const DecodeLayout L) {
     extern __shared__ __align__(128) uint8_t dyn[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(dyn);
     uint8_t *act = dyn + L.act;
@@ -715,62 +920,90 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
     const unsigned long long epoch = S.epoch;
     const uint32_t tag = (uint32_t)(epoch + 1ull);
     const uint16_t *xr = xs_on ? xsm : a.x;
-    for (int q = warp; q < ne * T; q += kWarps) {
+    // The CTA's ne * T dot products over H. With fewer of them than warps each is split into
+    // slices of whole 256-element strides, one slice per warp, and the slices' sums are added
+    // in slice order.
+    // Every logit word goes to lrep copies of the T x E block (lstride words apart, spread over
+    // the L2 slices); CTA c polls copy c mod lrep, so that no slice serves all CTAs' polls.
+    auto publish_logit = [&](int t, int e, float l) {
+        const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(l);
+        for (int r = 0; r < a.lrep; ++r) st_relaxed_u64(a.logits + (size_t)r * a.lstride + (size_t)t * E + e, w);
+    };
+    const int nq = ne * T;
+    const int nstr = (H + 255) / 256;
+    const int nsl = (nq > 0 && nq < kWarps) ? min(kWarps / nq, nstr) : 1;
+    for (int it = warp; it < nq * nsl; it += kWarps) {
+        const int q = it / nsl, sl = it - q * nsl;
         const int i = q / T, t = q % T;
         const int e = c + i * nC;
         const float *wrow = wr_on ? wsm + (size_t)i * H : a.wr + (size_t)e * H;
         const uint16_t *xrow = xr + (size_t)t * H;
-        float acc = 0.f;
-        for (int h = lane * 8; h < H; h += 256) {
+        const int h1 = min(H, (sl + 1) * nstr / nsl * 256);
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int h = sl * nstr / nsl * 256 + lane * 8; h < h1; h += 256) {
             const float4 w0 = *reinterpret_cast<const float4 *>(wrow + h);
             const float4 w1 = *reinterpret_cast<const float4 *>(wrow + h + 4);
             const uint4 xv = xs_on ? *reinterpret_cast<const uint4 *>(xrow + h) : __ldcg(reinterpret_cast<const uint4 *>(xrow + h));
-            acc += w0.x * __uint_as_float(xv.x << 16) + w0.y * __uint_as_float(xv.x & 0xFFFF0000u);
-            acc += w0.z * __uint_as_float(xv.y << 16) + w0.w * __uint_as_float(xv.y & 0xFFFF0000u);
-            acc += w1.x * __uint_as_float(xv.z << 16) + w1.y * __uint_as_float(xv.z & 0xFFFF0000u);
-            acc += w1.z * __uint_as_float(xv.w << 16) + w1.w * __uint_as_float(xv.w & 0xFFFF0000u);
+            acc0 += w0.x * __uint_as_float(xv.x << 16) + w0.y * __uint_as_float(xv.x & 0xFFFF0000u);
+            acc1 += w0.z * __uint_as_float(xv.y << 16) + w0.w * __uint_as_float(xv.y & 0xFFFF0000u);
+            acc0 += w1.x * __uint_as_float(xv.z << 16) + w1.y * __uint_as_float(xv.z & 0xFFFF0000u);
+            acc1 += w1.z * __uint_as_float(xv.w << 16) + w1.w * __uint_as_float(xv.w & 0xFFFF0000u);
         }
+        float acc = acc0 + acc1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
-            const float l = acc + (a.bias ? a.bias[e] : 0.f);
-            st_relaxed_u64(a.logits + (size_t)t * E + e,
-                           ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(l));
+            if (nsl == 1) publish_logit(t, e, acc + (a.bias ? a.bias[e] : 0.f));
+            else S.lpart[it] = acc;
         }
     }
-    // per-token sums of x over each group (one warp per group, two values per lane)
-    for (int i = warp; i < T * G; i += kWarps) {
-        const uint32_t v = xs_on ? *reinterpret_cast<const uint32_t *>(xr + (size_t)i * kGroup + 2 * lane)
-                                 : __ldcg(reinterpret_cast<const unsigned int *>(xr + (size_t)i * kGroup + 2 * lane));
-        float s = __uint_as_float(v << 16) + __uint_as_float(v & 0xFFFF0000u);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) Xs[i] = s;
+    if (nsl > 1) {
+        __syncthreads();
+        if (threadIdx.x < nq) {
+            const int q = threadIdx.x, i = q / T, t = q % T;
+            const int e = c + i * nC;
+            float l = 0.f;
+            for (int sl = 0; sl < nsl; ++sl) l += S.lpart[q * nsl + sl];
+            publish_logit(t, e, l + (a.bias ? a.bias[e] : 0.f));
+        }
     }
     grid_dep_launch();
 
-    // ---------------------------------------------------------------- top-k (every CTA)
-    for (int t = warp; t < T; t += kWarps) {
-        int idx = -1;
-        float w = 0.f;
-        bool ok = !S.abort;
-        if (ok) {
-            if (E <= 256) ok = token_topk<8>(a, t, tag, lane, idx, w);
-            else if (E <= 512) ok = token_topk<16>(a, t, tag, lane, idx, w);
-            else ok = token_topk<32>(a, t, tag, lane, idx, w);
+    // per-token sums of x over each group, eight threads per group; with one token they are
+    // formed by the consumer warps while the control warp routes
+    auto group_sums = [&](int tid0, int nthreads) {
+        const int n = T * G * 8;
+        for (int base = tid0 - lane; base < n; base += nthreads) {
+            const int i = base + lane;
+            float s = 0.f;
+            if (i < n) {
+                const uint16_t *src = xr + (size_t)(i >> 3) * kGroup + (i & 7) * 8;
+                const uint4 v = xs_on ? *reinterpret_cast<const uint4 *>(src) : __ldcg(reinterpret_cast<const uint4 *>(src));
+                s = (__uint_as_float(v.x << 16) + __uint_as_float(v.x & 0xFFFF0000u)) +
+                    (__uint_as_float(v.y << 16) + __uint_as_float(v.y & 0xFFFF0000u)) +
+                    (__uint_as_float(v.z << 16) + __uint_as_float(v.z & 0xFFFF0000u)) +
+                    (__uint_as_float(v.w << 16) + __uint_as_float(v.w & 0xFFFF0000u));
+            }
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            if (i < n && (i & 7) == 0) Xs[i >> 3] = s;
         }
-        if (!ok) {
-            if (lane == 0) S.abort = 1;
-        } else if (lane < K) {
-            S.sel_idx[t * K + lane] = idx;
-            S.sel_w[t * K + lane] = w;
-            if (c == 0 && a.idx_out) a.idx_out[t * K + lane] = idx;
-            if (c == 0 && a.w_out) a.w_out[t * K + lane] = w;
-        }
+    };
+    // ---------------------------------------------------------------- top-k (every CTA) + plan
+    auto route_token = [&](int t) {
+        const bool ok = !S.abort && (E <= 256 ? token_topk(a, S, t, tag, lane, c) : token_topk_wide(a, S, t, tag, lane, c));
+        if (!ok && lane == 0) S.abort = 1;
+    };
+    // tokens go to warps from the control warp on, so that with one token the control warp routes
+    // it and makes the plan without a CTA barrier in between
+    for (int t = (warp + 1) % kWarps; t < T; t += kWarps) route_token(t);
+    if (warp != kCW || T > 1) group_sums(threadIdx.x, T > 1 ? kThreads : kCW * 32);
+    if (T > 1) __syncthreads();
+    if (warp == kCW) {
+        __syncwarp();
+        make_plan(a, S, S.abort ? 0 : P, lane, c, nC);
     }
-    __syncthreads();
-    const bool routed = !S.abort;
-    if (warp == kCW) make_plan(a, S, routed ? P : 0, lane, c, nC);
     __syncthreads();
 
     if (warp == kCW) {
@@ -1045,6 +1278,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
     }
 }
 
+// Copies of the exchanged logit words within the fixed logit region (kMaxT x kMaxE words): the
+// T x E block at 4 KB-aligned strides, up to 16 copies.
+void logit_copies(int T, int E, int &rep, int &stride) {
+    stride = (int)align_up((size_t)T * E, 512);
+    rep = 1;
+    while (rep < 16 && (size_t)(rep * 2) * stride <= (size_t)kMaxT * kMaxE) rep *= 2;
+}
+
 template <int NT>
 moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t st) {
     const DecodeLayout L = decode_layout<NT>(a.T, a.H, dev->max_smem_optin);
@@ -1094,6 +1335,8 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     a.h_hi = reinterpret_cast<uint16_t *>(w8 + W.h_hi);
     a.h_lo = reinterpret_cast<uint16_t *>(w8 + W.h_lo);
     a.wait_ns = wait_limit_ns();
+    a.rnC = 1.0 / (double)dev->sms;
+    logit_copies(T, E, a.lrep, a.lstride);
     if (T <= 8) return launch_nt<1>(a, dev, st);
     if (T <= 16) return launch_nt<2>(a, dev, st);
     return launch_nt<4>(a, dev, st);

@@ -77,7 +77,7 @@ constexpr int kDecodeMaxP = 256;   // decode limit on T*k
 
 // Decode workspace, fixed regions first so that one workspace can serve decode calls of any
 // shape: logits, kMaxT x kMaxE 8-byte words {fp32 logit bits (low word), call tag (high word)}
-// (call t writes entry t * E + e); h_ready, finished gate/up row blocks per selected expert;
+// (a call writes entry t * E + e of each of its copies of the T x E block); h_ready, finished gate/up row blocks per selected expert;
 // out_acc, fp32 [T x H] (up to kMaxT x kDecodeMaxH); then h_hi / h_lo, bf16 h of every
 // (token, slot) pair [T*k x I]. h_ready and out_acc are zero between calls: the last CTA of
 // every call clears what the call used.
