@@ -65,9 +65,23 @@ struct DecodeArgs {
     float *out_acc;
     uint32_t *h_ready;
     uint64_t wait_ns;
-    double rnC;     // 1 / number of CTAs
-    int lrep;       // copies of the logit words (a power of two)
-    int lstride;    // words between copies
+    double rnC;                  // 1 / number of CTAs
+    uint32_t cm, cs1, cs2;       // division by the number of CTAs: multiplier and shifts
+    uint32_t kmul;               // ceil(2^16 / k): p / k = (p * kmul) >> 16 for p < 2048
+    int lrep;                    // copies of the logit words (a power of two)
+    int lstride;                 // words between copies
+};
+
+// One ring stage's chunk, written by the producer before it starts the copy: jobs job0 ..
+// job0 + njobs - 1 of one phase and one expert slot u; the first job from its tile k0, the last
+// up to tile k1 (tpj tiles per job); job0's tile 0 lies base_off bytes from the stage start
+// (negative when the chunk begins inside that job). flags: 1 gate/up phase, 2 the CTA's last chunk.
+struct __align__(16) ChunkDesc {
+    int job0, base_off;
+    short njobs, k0, k1, tpj;
+    unsigned short tb;
+    unsigned char bits, flags;
+    short u, pad;
 };
 
 struct __align__(16) DecodeSmem {
@@ -77,9 +91,7 @@ struct __align__(16) DecodeSmem {
     unsigned long long epoch;
     volatile int abort;
     int U, g0, g1, d0, d1, nGU;
-    int gu_done, is_last, hexp, hq;
-    int slot_job[16];
-    int slot_cnt[16];
+    int is_last;
     uint32_t eoff[kMaxE];               // packed offset / 256 of every expert
     uint8_t ebits[kMaxE];               // code width of every expert
     uint32_t selmask[kMaxE / 32];
@@ -97,11 +109,17 @@ struct __align__(16) DecodeSmem {
     int sel_idx[kMaxP];
     float sel_w[kMaxP];
     float lpart[kWarps];                // slice sums of the router dot products
+    ChunkDesc desc[kMaxStages];         // the chunk of each ring stage
     __align__(16) uint32_t plist[32];   // plan scratch: packed pair list
 };
 
 // accumulator slots of NT n-tiles: 16 rows x 8*NT columns fp32, laid out as the MMA fragments
 template <int NT> constexpr int slots_for() { return NT == 4 ? 8 : 16; }
+// A gate/up job's partial sums stay in its slot from the chunk that completes it until the next
+// chunk's barrier; meanwhile that chunk adds into the slots of the jobs it touches. A chunk touching at
+// most (slots - 1) / 2 jobs keeps the two sets apart, so a chunk holds at most that minus one
+// jobs' worth of tiles.
+template <int NT> constexpr int chunk_jobs() { return (slots_for<NT>() - 1) / 2 - 1; }
 template <int NT> constexpr int slot_floats() { return NT * 128; }
 
 struct DecodeLayout {
@@ -127,19 +145,6 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-__device__ __forceinline__ int ld_acquire_cta(const int *p) {
-    int v;
-    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_cta(int *p, int v) {
-    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-__device__ __forceinline__ int atom_add_acq_rel_cta(int *p, int v) {
-    int old;
-    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
-    return old;
-}
 __device__ __forceinline__ void red_shared_f32(float *p, float v) {
     asm volatile("red.relaxed.cta.shared::cta.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
@@ -198,10 +203,10 @@ __device__ __forceinline__ Region region_at(const DecodeSmem &S, const DecodeArg
     r.src = gu ? base + (size_t)r.rb0 * G * r.tb : base + gu_tiles(a.H, a.I) * r.tb + (size_t)r.rb0 * GI * r.tb;
     return r;
 }
-// Chunks of a region: at most one stage; for gate/up regions (split K, accumulator slots) also at
-// most two jobs' worth of tiles, so that one chunk touches at most three jobs.
-__device__ __forceinline__ int region_chunks(const Region &r, bool gu) {
-    const int cap = gu ? min(kStageBytes / r.tb, 2 * r.tpj) : kStageBytes / r.tb;
+// Chunks of a region: at most one stage and at most maxjobs jobs' worth of tiles (gate/up
+// chunks, whose jobs keep partial sums in slots).
+__device__ __forceinline__ int region_chunks(const Region &r, int maxjobs) {
+    const int cap = min(kStageBytes / r.tb, maxjobs * r.tpj);
     return (r.tiles + cap - 1) / cap;
 }
 // tiles [c0, c0 + m) of chunk i of a region (balanced split)
@@ -248,6 +253,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
+}
+// predicated shared-memory store (no branch)
+__device__ __forceinline__ void sts_if(bool p, int *addr, int v) {
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q st.shared.u32 [%1], %2;\n\t}" ::"r"((int)p),
+                 "r"(smem_u32(addr)), "r"(v)
+                 : "memory");
 }
 __device__ __forceinline__ float lds32f(uint32_t a) {
     float v;
@@ -486,7 +497,7 @@ __device__ bool token_topk(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t t
         const bool win = sk[0] == mx;
         const uint32_t b = __ballot_sync(0xffffffffu, win);
         tied |= b & (b - 1u);
-        if (win) sel[r] = lane + 32 * sm_[0];
+        sts_if(win, sel + r, lane + 32 * sm_[0]);
         // the winner shifts its list (selects, no branch)
 #pragma unroll
         for (int m = 0; m < 7; ++m) {
@@ -503,12 +514,18 @@ __device__ bool token_topk(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t t
     return true;
 }
 
-// floor(X * cc / nC) without an integer division: the quotient taken through the double
-// reciprocal of nC (X * cc < 2^53 is exact in double, and the estimate is floor or floor - 1)
-// and corrected once.
-__device__ __forceinline__ uint32_t cut_units(uint32_t X, int cc, int nC, double rnC) {
+// floor(X * cc / nC) without an integer division. Below 2^32 the product is divided by the
+// invariant-divisor method of Granlund and Montgomery (a multiply-high, an add and two shifts
+// with constants set up on the host, exact for every 32-bit dividend); above, the quotient is
+// taken through the double reciprocal of nC (X * cc < 2^53 is exact in double and the estimate
+// is floor or floor - 1) and corrected once.
+__device__ __forceinline__ uint32_t cut_units(const DecodeArgs &a, uint32_t X, int cc, int nC) {
     const unsigned long long n = (unsigned long long)X * (unsigned)cc;
-    unsigned long long q = (unsigned long long)((double)n * rnC);
+    if (n < (1ull << 32)) {
+        const uint32_t n32 = (uint32_t)n, t = __umulhi(a.cm, n32);
+        return (t + ((n32 - t) >> a.cs1)) >> a.cs2;
+    }
+    unsigned long long q = (unsigned long long)((double)n * a.rnC);
     q += ((q + 1ull) * (unsigned)nC <= n) ? 1ull : 0ull;
     return (uint32_t)q;
 }
@@ -551,7 +568,7 @@ __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
 // memory, per-slot counts and a stable fill of the pair lists 32 slots at a time, and the job
 // ranges by binary search over the slots' unit prefixes.
 __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
-    const int K = a.k, E = a.E, H = a.H, I = a.I;
+    const int E = a.E, H = a.H, I = a.I;
     const int G = H / kGroup;
     const int pg = I / 8, pd = H / 16;
     const uint32_t ug = (uint32_t)pg * (uint32_t)G;
@@ -629,7 +646,7 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
         if (p < P) {
             const int pos = S.cursor[u] + rank;
             S.ppair[pos] = p;
-            S.ptok[pos] = p / K;
+            S.ptok[pos] = (int)(((uint32_t)p * a.kmul) >> 16);
             S.pw[pos] = S.sel_w[p];
         }
         __syncwarp();
@@ -645,7 +662,7 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
     int gcut = 0;
     if (lane < 2) {
         const int cc = c + lane;
-        gcut = (cc >= nC) ? U * pg : job_at_unit(S.cgu, U, pg, cut_units(GUB, cc, nC, a.rnC));
+        gcut = (cc >= nC) ? U * pg : job_at_unit(S.cgu, U, pg, cut_units(a, GUB, cc, nC));
     }
     g0 = __shfl_sync(0xffffffffu, gcut, 0);
     g1 = __shfl_sync(0xffffffffu, gcut, 1);
@@ -653,8 +670,8 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
     if (lane < 2) {
         const int cc = c + lane;
         const int gj = lane == 0 ? g0 : g1;
-        const uint32_t pos = mono ? cut_units(B, cc, nC, a.rnC) - job_start_unit(S.cgu, U, pg, gj)
-                                  : cut_units(DB, cc, nC, a.rnC);
+        const uint32_t pos = mono ? cut_units(a, B, cc, nC) - job_start_unit(S.cgu, U, pg, gj)
+                                  : cut_units(a, DB, cc, nC);
         dcut = (cc >= nC) ? U * pd : job_at_unit(S.cd, U, pd, pos);
     }
     d0 = __shfl_sync(0xffffffffu, dcut, 0);
@@ -680,7 +697,7 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
         make_plan_many(a, S, P, lane, c, nC);
         return;
     }
-    const int K = a.k, H = a.H, I = a.I;
+    const int H = a.H, I = a.I;
     const int G = H / kGroup, GI = I / kGroup;
     const int pg = I / 8, pd = H / 16;
     const uint32_t ug = (uint32_t)pg * (uint32_t)G;   // gate/up units of an expert per unit of tile size
@@ -690,6 +707,7 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
     int slot;                          // slot of the lane's expert
     bool slot_lane;                    // the lane holds the first pair of its expert
     uint32_t mts;                      // largest units per tile over the slots
+    bool uniform;                      // every slot has the same tile size (all jobs alike)
     {
         // One pair per lane. Each lane counts, over a packed list of all pairs {expert, units
         // per tile, first pair of its expert}, the distinct experts below its own (its slot),
@@ -707,7 +725,7 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
         // entries past P: an id above every expert, no units, not first
         S.plist[lane] = v ? ((uint32_t)e | (tsl << 16) | (first ? 0x80000000u : 0u)) : 0xFFFFu;
         __syncwarp();
-        uint32_t nsl = 0, units = 0, pbelow = 0, nU = 0, tot = 0;
+        uint32_t nsl = 0, units = 0, pbelow = 0, nU = 0, tot = 0, mtsmin = 0xFFFFu;
         mts = 0;
         const uint4 *pl = reinterpret_cast<const uint4 *>(S.plist);
         for (int q4 = 0; q4 < (P + 3) / 4; ++q4) {
@@ -724,9 +742,11 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
                 nU += tq ? 1u : 0u;
                 tot += tq;
                 mts = max(mts, tq);
+                mtsmin = min(mtsmin, tq ? tq : 0xFFFFu);
             }
         }
         U = (int)nU;
+        uniform = mts == mtsmin;
         slot = (int)nsl;
         slot_lane = first;
         ts = tsl;
@@ -743,7 +763,7 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
         if (v) {
             const int pos = (int)pbelow + rank;
             S.ppair[pos] = lane;
-            S.ptok[pos] = lane / K;
+            S.ptok[pos] = (int)(((uint32_t)lane * a.kmul) >> 16);
             S.pw[pos] = pw;
         }
         if (lane == 0) {
@@ -764,20 +784,32 @@ __device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, i
         const uint32_t mj = mts * (uint32_t)G;                            // largest gate/up job
         const bool mono = (unsigned long long)(mj + 2u) * (unsigned)nC <= DB;
         uint32_t st0, st1, unused;
-        g0 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(GUB, c, nC, a.rnC), GUB, st0);
+        if (uniform && U > 0) {
+            // all jobs of a sequence alike: the first job at or after q is ceil(q / job units)
+            const uint32_t ug1 = mts * (uint32_t)G, ud1 = mts * (uint32_t)GI;
+            const int NG = U * pg, ND = U * pd;
+            g0 = min(NG, (int)ceil_div_small(cut_units(a, GUB, c, nC), ug1));
+            g1 = (c + 1 < nC) ? min(NG, (int)ceil_div_small(cut_units(a, GUB, c + 1, nC), ug1)) : NG;
+            const uint32_t q0 = mono ? cut_units(a, B, c, nC) - (uint32_t)g0 * ug1 : cut_units(a, DB, c, nC);
+            const uint32_t q1 = mono ? cut_units(a, B, c + 1, nC) - (uint32_t)g1 * ug1 : cut_units(a, DB, c + 1, nC);
+            d0 = min(ND, (int)ceil_div_small(q0, ud1));
+            d1 = (c + 1 < nC) ? min(ND, (int)ceil_div_small(q1, ud1)) : ND;
+        } else {
+        g0 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(a, GUB, c, nC), GUB, st0);
         if (c + 1 < nC) {
-            g1 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(GUB, c + 1, nC, a.rnC), GUB, st1);
+            g1 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(a, GUB, c + 1, nC), GUB, st1);
         } else {
             g1 = U * pg;
             st1 = GUB;
         }
-        const uint32_t q0 = mono ? cut_units(B, c, nC, a.rnC) - st0 : cut_units(DB, c, nC, a.rnC);
+        const uint32_t q0 = mono ? cut_units(a, B, c, nC) - st0 : cut_units(a, DB, c, nC);
         d0 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q0, DB, unused);
         if (c + 1 < nC) {
-            const uint32_t q1 = mono ? cut_units(B, c + 1, nC, a.rnC) - st1 : cut_units(DB, c + 1, nC, a.rnC);
+            const uint32_t q1 = mono ? cut_units(a, B, c + 1, nC) - st1 : cut_units(a, DB, c + 1, nC);
             d1 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q1, DB, unused);
         } else {
             d1 = U * pd;
+        }
         }
     }
     if (lane == 0) {
@@ -818,9 +850,11 @@ __device__ __forceinline__ void finalize_gu(const DecodeArgs &a, const DecodeSme
             }
         }
     }
+
 }
 // Down job dj, computed whole by one warp: w * y of rows 16 rb + g and 16 rb + g + 8 added into
 // the fp32 output accumulator.
+// Down job dj, summed in one warp's registers: w * y added into the fp32 output accumulator.
 template <int NT>
 __device__ __forceinline__ void finalize_down(const DecodeArgs &a, const DecodeSmem &S, int dj, const float (&acc)[NT][4],
                                               const float (&acc2)[NT][4], int lane) {
@@ -877,7 +911,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         mbar_init(smem_u32(&S.xbar), 1);
         fence_barrier_init();
         S.abort = 0;
-        S.gu_done = 0;
         S.is_last = 0;
         if (wr_on && ne > 0) {
             const uint32_t rowb = (uint32_t)H * 4;
@@ -897,10 +930,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
     }
     for (int i = threadIdx.x; i < NSLOT * SF; i += kThreads) accs[i] = 0.f;
-    if (threadIdx.x < NSLOT) {
-        S.slot_job[threadIdx.x] = threadIdx.x;
-        S.slot_cnt[threadIdx.x] = 0;
-    }
     __syncthreads();
     // Everything below may read data that the previous launch in the stream produces.
     grid_dep_wait();
@@ -1011,12 +1040,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (lane != 0) return;
         uint32_t cc = 0;
         bool ok = true;
+        const bool has_down = S.d1 > S.d0;
         for (int ph = 0; ph < 2 && ok; ++ph) {
             const bool gu = ph == 0;
             const int jend = gu ? S.g1 : S.d1;
             for (int j = gu ? S.g0 : S.d0; j < jend && ok;) {
                 const Region r = region_at(S, a, gu, j);
-                const int nch = region_chunks(r, gu);
+                const int nch = region_chunks(r, gu ? chunk_jobs<NT>() : kStageBytes);
+                const int jnext = j + r.tiles / r.tpj;
                 for (int ch = 0; ch < nch; ++ch) {
                     int c0, m;
                     chunk_range(r, nch, ch, c0, m);
@@ -1027,13 +1058,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         ok = false;
                         break;
                     }
+                    // the chunk's descriptor, published to the consumers by the barrier's arrival
+                    const int jlo = c0 / r.tpj, jhi = (c0 + m - 1) / r.tpj;
+                    ChunkDesc dd;
+                    dd.job0 = r.jg0 + jlo;
+                    dd.base_off = (jlo * r.tpj - c0) * r.tb;
+                    dd.njobs = (short)(jhi - jlo + 1);
+                    dd.k0 = (short)(c0 - jlo * r.tpj);
+                    dd.k1 = (short)(c0 + m - jhi * r.tpj);
+                    dd.tpj = (short)r.tpj;
+                    dd.tb = (unsigned short)r.tb;
+                    dd.bits = (unsigned char)r.bits;
+                    const bool last = ch == nch - 1 && jnext >= jend && (!gu || !has_down);
+                    dd.flags = (unsigned char)((gu ? 1 : 0) | (last ? 2 : 0));
+                    dd.u = (short)r.u;
+                    dd.pad = 0;
+                    S.desc[s] = dd;
                     const uint32_t bytes = (uint32_t)(m * r.tb);
                     const uint32_t fb = smem_u32(&S.full[s]);
                     mbar_expect_tx(fb, bytes);
                     bulk_g2s(smem_u32(ring + (size_t)s * kStageBytes), r.src + (size_t)c0 * r.tb, bytes, fb);
                     ++cc;
                 }
-                j += r.tiles / r.tpj;
+                j = jnext;
             }
         }
         // copies still in flight land before the CTA may exit
@@ -1052,17 +1099,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             acc2[i][0] = acc2[i][1] = acc2[i][2] = acc2[i][3] = 0.f;
         }
     };
-    auto aborted = [&]() -> bool { return __shfl_sync(0xffffffffu, (int)S.abort, 0) != 0; };
     JobCtx<NT> jc;
-    int cur_hexp = -1;
     bool hfit = true;
     const uint16_t *hh = nullptr, *hl = nullptr;
     const float *hs = nullptr;
 
     // h of expert slot u into shared memory (with its per-group sums), after the expert's
     // gate/up rows are published by every CTA that computed some; all consumer warps take part.
+    // This CTA's gate/up rows are all stored (their finalisers passed a consumer barrier since):
+    // one fence makes them visible GPU-wide, then each expert's counter grows by the CTA's jobs.
+    bool published = false;
+    auto publish_h = [&]() {
+        if (threadIdx.x == 0 && !published && S.g1 > S.g0) {
+            __threadfence();
+            const int pg = I / 8;
+            const int u0 = S.g0 / pg, u1 = (S.g1 - 1) / pg;
+            for (int u = u0; u <= u1; ++u)
+                atomicAdd(&a.h_ready[u], (uint32_t)(min(S.g1, (u + 1) * pg) - max(S.g0, u * pg)));
+        }
+        published = true;
+    };
     auto load_h = [&](int u) {
         consumer_sync();   // nobody still reads the previous contents of act
+        if (!S.abort) publish_h();
         if (threadIdx.x == 0 && !S.abort &&
             !wait_counter(&a.h_ready[u], (uint32_t)(I / 8), a.wait_ns, status))
             S.abort = 1;
@@ -1137,120 +1196,88 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         jc.bg = gu ? !xs_on : !hfit;
     };
-    // this warp's partial of CTA-local job jl into its accumulator slot; the job's last warp
-    // finalises it, and the warp that finalises the CTA's last gate/up job publishes them all
-    auto flush = [&](int jl, int gj, bool gu, int target) {
-        if (aborted()) return;
-        const int slot = jl % NSLOT;
-        float *sp = accs + slot * SF;
-        if (lane == 0 && ld_acquire_cta(&S.slot_job[slot]) != jl) {
-            const uint64_t t0 = global_timer();
-            while (ld_acquire_cta(&S.slot_job[slot]) != jl) {
-                if (global_timer() - t0 > a.wait_ns) {
-                    atomicOr(status, kStatusTimeout);
-                    S.abort = 1;
-                    break;
-                }
-            }
-        }
-        __syncwarp();
-        if (aborted()) return;
+    // Gate/up jobs are split along K: tile k of a job goes to warp k % 8, which adds its partial
+    // sums into the job's slot (CTA-local job q uses slot q % NSLOT) after its last tile of the
+    // job. A down job (a few tiles) belongs to one warp and is finalised from its registers.
+    auto add_partial = [&](int q) {
+        float *sp = accs + (q % NSLOT) * SF;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) red_shared_f32(sp + (nt * 4 + i) * 32 + lane, acc[nt][i] + acc2[nt][i]);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atom_add_acq_rel_cta(&S.slot_cnt[slot], 1) == target - 1) ? 1 : 0;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) return;
-        __syncwarp();
-        finalize_gu<NT>(a, S, gj, sp, lane);
-        __syncwarp();
-        if (lane == 0) {
-            S.slot_cnt[slot] = 0;
-            st_release_cta(&S.slot_job[slot], jl + NSLOT);
+        zero_acc();
+    };
+    // Gate/up jobs fj0 .. fj0 + fn - 1 have all their partials in their slots (after the barrier
+    // that follows the chunk that completed them); warp gj % 8 finalises job gj.
+    int fj0 = 0, fn = 0;
+    auto finalize_pending = [&]() {
+        for (int i = 0; i < fn; ++i) {
+            const int gj = fj0 + i;
+            if ((gj & (kCW - 1)) == warp) finalize_gu<NT>(a, S, gj, accs + ((gj - S.g0) % NSLOT) * SF, lane);
         }
-        if (gu) {
-            int pub = 0;
-            if (lane == 0) pub = (atom_add_acq_rel_cta(&S.gu_done, 1) + 1 == S.nGU) ? 1 : 0;
-            pub = __shfl_sync(0xffffffffu, pub, 0);
-            if (pub) {
-                // every h row of this CTA is stored (the other warps released them through
-                // gu_done); make them visible GPU-wide before the counters say so
-                __syncwarp();
-                __threadfence();
-                const int pg = I / 8;
-                const int u0 = S.g0 / pg, u1 = (S.g1 - 1) / pg;
-                for (int u = u0 + lane; u <= u1; u += 32) {
-                    const int n = min(S.g1, (u + 1) * pg) - max(S.g0, u * pg);
-                    atomicAdd(&a.h_ready[u], (uint32_t)n);
-                }
-            }
-        }
+        fn = 0;
     };
 
     zero_acc();
-    uint32_t cc = 0;
-    for (int ph = 0; ph < 2; ++ph) {
-        const bool gu = ph == 0;
-        const int jend = gu ? S.g1 : S.d1;
-        for (int j = gu ? S.g0 : S.d0; j < jend;) {
-            const Region r = region_at(S, a, gu, j);
-            if (!gu && r.u != cur_hexp) {
-                load_h(r.u);
-                cur_hexp = r.u;
-            }
-            set_ctx(r.u, gu);
-            const int tpj = r.tpj;
-            const int target = tpj < kCW ? tpj : kCW;   // warps that add into a gate/up job
-            const int kl = (warp < tpj) ? warp + kCW * ((tpj - 1 - warp) / kCW) : -1;   // this warp's last k-tile
-            const int nch = region_chunks(r, gu);
-            for (int ch = 0; ch < nch; ++ch) {
-                int c0, m;
-                chunk_range(r, nch, ch, c0, m);
-                const int s = cc % NS;
-                const uint32_t use = cc / NS;
-                bool live = !aborted();
-                if (live) {
-                    const bool got = mbar_wait(smem_u32(&S.full[s]), use & 1u, a.wait_ns, status);
-                    live = __all_sync(0xffffffffu, got);
-                    if (!live && lane == 0) S.abort = 1;
+    int s = 0;
+    uint32_t par = 0;
+    int cur_u = -1, cur_gu = -1, tpj = 1, kl = -1;
+    bool more = S.g1 > S.g0 || S.d1 > S.d0;
+    while (more) {
+        const bool got = !S.abort && mbar_wait(smem_u32(&S.full[s]), par, a.wait_ns, status);
+        if (!got && lane == 0) S.abort = 1;
+        // One barrier per chunk: every warp's partials of the previous chunk are in, and all
+        // warps agree on an abort.
+        consumer_sync();
+        if (S.abort) break;
+        finalize_pending();
+        const ChunkDesc d = S.desc[s];
+        const bool gu = d.flags & 1;
+        if (d.u != cur_u || (int)gu != cur_gu) {
+            if (!gu) load_h(d.u);
+            set_ctx(d.u, gu);
+            cur_u = d.u;
+            cur_gu = gu;
+            tpj = d.tpj;
+            kl = (warp < tpj) ? warp + kCW * ((tpj - 1 - warp) / kCW) : -1;   // this warp's last tile of a job
+        }
+        const uint8_t *sb = ring + (size_t)s * kStageBytes + d.base_off;
+        for (int i = 0; i < d.njobs; ++i) {
+            const int k0 = i == 0 ? d.k0 : 0, k1 = i == d.njobs - 1 ? d.k1 : tpj;
+            const uint8_t *job_base = sb + (size_t)i * tpj * d.tb;
+            const int gj = d.job0 + i;
+            if (gu) {
+                if (d.bits == 4) run_tiles<4, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
+                else if (d.bits == 6) run_tiles<6, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
+                else run_tiles<8, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
+                if (kl >= k0 && kl < k1) add_partial(gj - S.g0);
+            } else if (((gj - S.d0) & (kCW - 1)) == warp) {
+                if (d.bits == 4) run_tiles_seq<4, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
+                else if (d.bits == 6) run_tiles_seq<6, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
+                else run_tiles_seq<8, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
+                if (k1 == tpj) {
+                    finalize_down<NT>(a, S, gj, acc, acc2, lane);
+                    zero_acc();
                 }
-                const uint8_t *sb = ring + (size_t)s * kStageBytes;
-                const int jlo = c0 / tpj, jhi = (c0 + m - 1) / tpj;
-                for (int jb = jlo; jb <= jhi; ++jb) {
-                    const int k0 = max(c0, jb * tpj) - jb * tpj, k1 = min(c0 + m, (jb + 1) * tpj) - jb * tpj;
-                    const uint8_t *job_base = sb + ((long long)jb * tpj - c0) * r.tb;
-                    const int gj = r.jg0 + jb;
-                    if (gu) {
-                        if (live) {
-                            if (r.bits == 4) run_tiles<4, NT, true>(job_base, r.tb, k0, k1, warp, jc, lane, acc, acc2);
-                            else if (r.bits == 6) run_tiles<6, NT, true>(job_base, r.tb, k0, k1, warp, jc, lane, acc, acc2);
-                            else run_tiles<8, NT, true>(job_base, r.tb, k0, k1, warp, jc, lane, acc, acc2);
-                        }
-                        if (kl >= k0 && kl < k1) {
-                            flush(gj - S.g0, gj, true, target);
-                            zero_acc();
-                        }
-                    } else if ((gj - S.d0) % kCW == warp) {
-                        // down jobs: the whole job in one warp, no cross-warp reduction
-                        if (live) {
-                            if (r.bits == 4) run_tiles_seq<4, NT>(job_base, r.tb, k0, k1, jc, lane, acc, acc2);
-                            else if (r.bits == 6) run_tiles_seq<6, NT>(job_base, r.tb, k0, k1, jc, lane, acc, acc2);
-                            else run_tiles_seq<8, NT>(job_base, r.tb, k0, k1, jc, lane, acc, acc2);
-                        }
-                        if (k1 == tpj) {
-                            if (live && !aborted()) finalize_down<NT>(a, S, gj, acc, acc2, lane);
-                            zero_acc();
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
-                ++cc;
             }
-            j += r.tiles / r.tpj;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
+        fj0 = d.job0;
+        fn = gu ? d.njobs - (d.k1 < tpj ? 1 : 0) : 0;
+        more = !(d.flags & 2);
+        if (++s == NS) {
+            s = 0;
+            par ^= 1u;
+        }
+    }
+    consumer_sync();
+    if (!S.abort) {
+        finalize_pending();
+        if (!published) {
+            // no down job here: the gate/up rows are published after their finalisers are done
+            consumer_sync();
+            publish_h();
         }
     }
 
@@ -1336,6 +1363,16 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     a.h_lo = reinterpret_cast<uint16_t *>(w8 + W.h_lo);
     a.wait_ns = wait_limit_ns();
     a.rnC = 1.0 / (double)dev->sms;
+    {
+        // Granlund-Montgomery constants for division by the number of CTAs
+        const uint32_t d = (uint32_t)dev->sms;
+        uint32_t l = 0;
+        while ((1ull << l) < d) ++l;   // ceil(log2 d)
+        a.cm = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1ull);
+        a.cs1 = l < 1 ? l : 1u;
+        a.cs2 = l > 0 ? l - 1u : 0u;
+    }
+    a.kmul = (uint32_t)((65536 + k - 1) / k);
     logit_copies(T, E, a.lrep, a.lstride);
     if (T <= 8) return launch_nt<1>(a, dev, st);
     if (T <= 16) return launch_nt<2>(a, dev, st);
