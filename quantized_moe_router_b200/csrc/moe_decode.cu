@@ -49,6 +49,7 @@ constexpr int kMaxStages = 8;
 constexpr int kActBytes = 65536;            // x (routing + gate/up), then h of one expert (down)
 constexpr int kMaxP = kDecodeMaxP;
 constexpr int kSmemBudget = 232448;         // 227 KB opt-in shared memory per CTA
+constexpr int kBiasRows = 32;               // router bias values kept in shared memory
 
 struct DecodeArgs {
     const uint16_t *x;
@@ -110,6 +111,7 @@ struct __align__(16) DecodeSmem {
     float sel_w[kMaxP];
     float lpart[kWarps];                // slice sums of the router dot products
     ChunkDesc desc[kMaxStages];         // the chunk of each ring stage
+    float bias[kBiasRows];              // router bias of the CTA's rows c, c + nCTA, ...
     __align__(16) uint32_t plist[32];   // plan scratch: packed pair list
 };
 
@@ -930,18 +932,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
     }
     for (int i = threadIdx.x; i < NSLOT * SF; i += kThreads) accs[i] = 0.f;
+    // the router bias of this CTA's rows (a weight), off the logits' critical path
+    if (threadIdx.x < ne && threadIdx.x < kBiasRows) S.bias[threadIdx.x] = a.bias ? a.bias[c + threadIdx.x * nC] : 0.f;
     __syncthreads();
     // Everything below may read data that the previous launch in the stream produces.
     grid_dep_wait();
 
     // ---------------------------------------------------------------- logits
     if (threadIdx.x == 0) {
-        S.epoch = *reinterpret_cast<volatile unsigned long long *>(&a.ctl->done) / (unsigned long long)nC;
+        // the copy of x first: the read of the call counter overlaps it
         if (xs_on) {
             const uint32_t bytes = (uint32_t)(T * H * 2);
             mbar_expect_tx(smem_u32(&S.xbar), bytes);
             bulk_g2s(smem_u32(act), a.x, bytes, smem_u32(&S.xbar));
         }
+        S.epoch = *reinterpret_cast<volatile unsigned long long *>(&a.ctl->done) / (unsigned long long)nC;
     }
     if (xs_on && !mbar_wait(smem_u32(&S.xbar), 0, a.wait_ns, status)) S.abort = 1;
     if (wr_on && ne > 0 && !mbar_wait(smem_u32(&S.wbar), 0, a.wait_ns, status)) S.abort = 1;
@@ -954,6 +959,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // in slice order.
     // Every logit word goes to lrep copies of the T x E block (lstride words apart, spread over
     // the L2 slices); CTA c polls copy c mod lrep, so that no slice serves all CTAs' polls.
+    auto row_bias = [&](int i, int e) -> float { return i < kBiasRows ? S.bias[i] : (a.bias ? a.bias[e] : 0.f); };
     auto publish_logit = [&](int t, int e, float l) {
         const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(l);
         for (int r = 0; r < a.lrep; ++r) st_relaxed_u64(a.logits + (size_t)r * a.lstride + (size_t)t * E + e, w);
@@ -982,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
-            if (nsl == 1) publish_logit(t, e, acc + (a.bias ? a.bias[e] : 0.f));
+            if (nsl == 1) publish_logit(t, e, acc + row_bias(i, e));
             else S.lpart[it] = acc;
         }
     }
@@ -993,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int e = c + i * nC;
             float l = 0.f;
             for (int sl = 0; sl < nsl; ++sl) l += S.lpart[q * nsl + sl];
-            publish_logit(t, e, l + (a.bias ? a.bias[e] : 0.f));
+            publish_logit(t, e, l + row_bias(i, e));
         }
     }
     grid_dep_launch();
@@ -1132,33 +1138,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         float *hsw = reinterpret_cast<float *>(act);
         uint16_t *hhw = reinterpret_cast<uint16_t *>(act + hsb), *hlw = hhw + (size_t)nu * I;
         if (!S.abort) {
-            for (int item = threadIdx.x; item < nu * GI; item += kCW * 32) {
-                const int q = item / GI, grp = item % GI;
-                const size_t o = (size_t)S.ppair[pf + q] * I + (size_t)grp * kGroup;
-                const uint4 *sh = reinterpret_cast<const uint4 *>(a.h_hi + o);
-                const uint4 *sl = reinterpret_cast<const uint4 *>(a.h_lo + o);
-                uint4 vh[8], vl[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    vh[i] = __ldcg(sh + i);
-                    vl[i] = __ldcg(sl + i);
+            // eight threads per group of 64 values: one 16-byte piece of h hi and of h lo each,
+            // the group's sum over a 3-step shuffle
+            const int n8 = nu * GI * 8;
+            for (int base = threadIdx.x - lane; base < n8; base += kCW * 32) {
+                const int i8 = base + lane;
+                const bool v = i8 < n8;
+                const int item = i8 >> 3, part = i8 & 7;
+                const int q = item / GI, grp = item - q * GI;
+                uint4 vh = make_uint4(0, 0, 0, 0), vl = make_uint4(0, 0, 0, 0);
+                if (v) {
+                    const size_t o = (size_t)S.ppair[pf + q] * I + (size_t)grp * kGroup + part * 8;
+                    vh = __ldcg(reinterpret_cast<const uint4 *>(a.h_hi + o));
+                    vl = __ldcg(reinterpret_cast<const uint4 *>(a.h_lo + o));
                 }
+                const uint32_t w8[8] = {vh.x, vh.y, vh.z, vh.w, vl.x, vl.y, vl.z, vl.w};
                 float sum = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t w8[8] = {vh[i].x, vh[i].y, vh[i].z, vh[i].w, vl[i].x, vl[i].y, vl[i].z, vl[i].w};
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) sum += __uint_as_float(w8[j] << 16) + __uint_as_float(w8[j] & 0xFFFF0000u);
-                }
-                hsw[item] = sum;
-                if (hfit) {
-                    uint4 *dh = reinterpret_cast<uint4 *>(hhw + (size_t)q * I + (size_t)grp * kGroup);
-                    uint4 *dl = reinterpret_cast<uint4 *>(hlw + (size_t)q * I + (size_t)grp * kGroup);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        dh[i] = vh[i];
-                        dl[i] = vl[i];
-                    }
+                for (int j = 0; j < 8; ++j) sum += __uint_as_float(w8[j] << 16) + __uint_as_float(w8[j] & 0xFFFF0000u);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                if (v && part == 0) hsw[item] = sum;
+                if (v && hfit) {
+                    const size_t d = (size_t)q * I + (size_t)grp * kGroup + part * 8;
+                    *reinterpret_cast<uint4 *>(hhw + d) = vh;
+                    *reinterpret_cast<uint4 *>(hlw + d) = vl;
                 }
             }
         }
