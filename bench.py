@@ -485,7 +485,13 @@ def run_prefill(args, w, world, rank):
         "value": world * w.T * nsteps / (ms * 1e-3), "unit": "tokens/s", "steps": nsteps,
         "ms_per_step": ms / nsteps, "ms_per_layer": ms / nsteps / w.layers,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                     "frac": achieved / bf16, "traffic": None, "peak_source": peak_src,
+                     "frac": achieved / bf16,
+                     "traffic": recorded_traffic("prefill_tc_grouped_prefill_t4096_h2048.txt",
+                                                 ["quantized_moe_router_b200/csrc/moe_prefill_tc.cu",
+                                                  "quantized_moe_router_b200/csrc/moe_prefill.cu",
+                                                  "quantized_moe_router_b200/csrc/moe_internal.cuh"])
+                     if w.name == "prefill_t4096_l8_h2048_e256_k8_i512_int4" else None,
+                     "peak_source": peak_src,
                      "flops_per_launch": prefill_flops(w),
                      "kernel": "expert phase (moe_prefill_experts: grouped gate/up + down GEMMs, combine)",
                      "kernel_ms_per_launch": gemm_ms},
