@@ -147,6 +147,15 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// named barrier 2: the control warp arrives when the plan is in shared memory, the consumer
+// warps wait for it (and for each other's group sums)
+__device__ __forceinline__ void plan_ready_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory"); }
+__device__ __forceinline__ void plan_ready_wait() { asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory"); }
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long *p, unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+    return old;
+}
 __device__ __forceinline__ void red_shared_f32(float *p, float v) {
     asm volatile("red.relaxed.cta.shared::cta.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
@@ -1038,10 +1047,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (warp == kCW) {
         __syncwarp();
         make_plan(a, S, S.abort ? 0 : P, lane, c, nC);
-    }
-    __syncthreads();
-
-    if (warp == kCW) {
+        __syncwarp();
+        // hand the plan to the consumer warps and start streaming without waiting for them
+        plan_ready_arrive();
         // ------------------------------------------------------------ producer (one thread)
         if (lane != 0) return;
         uint32_t cc = 0;
@@ -1096,6 +1104,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
 
     // ---------------------------------------------------------------- consumers
+    plan_ready_wait();
     const int g = lane >> 2, t = lane & 3;
     float acc[NT][4], acc2[NT][4];
     auto zero_acc = [&]() {
@@ -1289,15 +1298,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // ---------------------------------------------------------------- completion
     consumer_sync();
     if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned long long old = atomicAdd(&a.ctl->done, 1ull);
+        // release (this CTA's additions, ordered before it by the barrier) and acquire (the
+        // other CTAs' additions, for the last CTA) in one step
+        const unsigned long long old = atom_add_acq_rel_u64(&a.ctl->done, 1ull);
         S.is_last = (old + 1ull == (epoch + 1ull) * (unsigned long long)nC) ? 1 : 0;
     }
     consumer_sync();
     if (S.is_last) {
         // every CTA's additions are complete: convert, then leave the accumulator and the
         // readiness counters zero for the next call
-        __threadfence();
         float4 *acc4 = reinterpret_cast<float4 *>(a.out_acc);
         uint2 *out4 = reinterpret_cast<uint2 *>(a.out);
         for (int i = threadIdx.x; i < T * H / 4; i += kCW * 32) {
