@@ -373,30 +373,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     if (warp < kDqWarps) {
         // ------------------------------------------------------------ dequantisers
         const int b = warp;
-        uint32_t j = 0;
         bool ok = run;
         const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
+        // step counters kept incrementally (no division in the loop): position jk in the K
+        // chunk, raw slot rs and its phase, A/B stage slot and its phase
+        int jk = 0, rs = 0, slot = 0;
+        uint32_t rpar = 0, apar = 0;
+        bool first_pass = true;
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
             // per unit: the expert's width and whether this warp's row block exists
             const int bits = __ldg(&pe[U.e].bits);
             const int tb = tile_bytes(bits);
             const bool have = 8 * U.mt + b < G.nrb;
-            for (int kg = 0; kg < G.KG; ++kg, ++j) {
-                const uint32_t chunk = j / KC;
-                const uint32_t rs = chunk % R;
-                if (j % KC == 0 && !tc_wait(S, a, &S.raw_full[rs], (chunk / R) & 1u)) {
+            for (int kg = 0; kg < G.KG; ++kg) {
+                if (jk == 0 && !tc_wait(S, a, &S.raw_full[rs], rpar)) {
                     ok = false;
                     break;
                 }
-                const int slot = j % kABStages;
-                const uint32_t use = j / kABStages;
-                if (use > 0 && !tc_wait(S, a, &S.ab_empty[slot], (use - 1) & 1u)) {
+                if (!first_pass && !tc_wait(S, a, &S.ab_empty[slot], apar ^ 1u)) {
                     ok = false;
                     break;
                 }
                 uint8_t *As = ring + (size_t)slot * stage_bytes;
-                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + (int)(j % KC)) * tb;
+                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + jk) * tb;
                 if (!have) {
                     // row block past the matrix: zero rows (the epilogue skips them)
                     const uint4 z = make_uint4(0, 0, 0, 0);
@@ -416,7 +416,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(smem_u32(&S.ab_full[slot]));
-                    if (j % KC == (uint32_t)KC - 1) mbar_arrive(smem_u32(&S.raw_empty[rs]));
+                    if (jk == KC - 1) mbar_arrive(smem_u32(&S.raw_empty[rs]));
+                }
+                if (++jk == KC) {
+                    jk = 0;
+                    if (++rs == R) {
+                        rs = 0;
+                        rpar ^= 1u;
+                    }
+                }
+                if (++slot == kABStages) {
+                    slot = 0;
+                    apar ^= 1u;
+                    first_pass = false;
                 }
             }
         }
