@@ -9,27 +9,28 @@
 //     layer): mbarrier set-up, this CTA's router rows copied into shared memory, the packed
 //     layer's expert table read. Both are weights, never produced by the previous launch.
 //   * Routing. x is copied into shared memory; each CTA computes the fp32 logits of its
-//     E / nCTA experts and stores each as one 8-byte word {logit, call tag}. Every CTA then
-//     polls the T x E words until all carry this call's tag (the tag is derived from a
-//     completion counter that grows by nCTA per call, so no barrier and no reset is needed)
-//     and runs the same warp-per-token top-k + softmax in registers; all CTAs agree on the
-//     selection without a second exchange.
-//   * Plan (control warp). Unique experts in ascending id, their pair lists (ascending
-//     token) and two job sequences: gate/up jobs (8 intermediate rows x all of H) and down
-//     jobs (16 output rows x all of I). Each CTA takes a contiguous range of each, cut so that
-//     every CTA streams the same number of bytes as a few long contiguous regions.
-//   * Streaming. The control warp streams the CTA's regions with bulk copies of up to 24 KB
-//     (on B200 one SM completes roughly one bulk copy per 250 ns whatever its size, so copies
-//     must be large) into a ring of 4-6 stages. Tile kg of a job goes to consumer warp kg % 8
-//     (split K), which multiplies it with mma.sync on bf16 operands made from the codes by one
-//     LOP3 per register (exact integers 128 + q) and applies the group's scale and zero in fp32.
-//   * A warp adds its partial of a job into a shared-memory accumulator slot when it has done
-//     its last tile of that job; the last of the job's warps finalises it: SiLU-GLU and the
-//     bf16 hi/lo split of h for gate/up jobs (stored to global), w * y added into the fp32
-//     output accumulator for down jobs. When a CTA has finalised all its gate/up jobs it
-//     publishes them (one fence, one counter add per expert); a down job waits only for the
-//     counter of its own expert, so the second exchange costs no grid-wide barrier, and the
-//     down tiles are already streaming while it waits.
+//     E / nCTA experts (the dot products split over all warps) and publishes each as one 8-byte
+//     word {logit, call tag} into up to 16 copies of the T x E block, so that the CTAs' polls
+//     spread over the L2 slices. Every CTA polls its copy until all words carry this call's tag
+//     (derived from a completion counter that grows by nCTA per call: no barrier, no reset) and
+//     runs the same top-k + softmax: all CTAs agree on the selection without a second exchange.
+//   * Plan (control warp). Unique experts in ascending id, their pair lists (ascending token)
+//     and two job sequences: gate/up jobs (8 intermediate rows x all of H) and down jobs (16
+//     output rows x all of I). Each CTA takes a contiguous range of each, cut so that every CTA
+//     streams the same number of bytes as a few long contiguous regions.
+//   * Streaming. The control warp streams the CTA's regions with bulk copies of up to 48 KB
+//     (on B200 one SM completes roughly one bulk copy per 250 ns whatever its size, and every
+//     chunk costs the consumers one barrier, so chunks are large) into a ring of 2-3 stages,
+//     writing each chunk's job range into a descriptor next to it.
+//   * Gate/up: tile kg of a job goes to consumer warp kg % 8 (split K), which multiplies it with
+//     mma.sync on bf16 operands made from the codes by one LOP3 per register (exact integers
+//     128 + q) and applies the group's scale and zero in fp32; after its last tile of a job a
+//     warp adds its partial into the job's shared-memory slot. One consumer barrier per chunk
+//     marks the previous chunk's jobs complete; each is finalised (SiLU-GLU, h as a bf16 hi/lo
+//     pair) by one warp while the others run on. The CTA publishes its h rows once (counter adds
+//     per expert after a fence); a down job waits only for the counter of its own expert.
+//   * Down: a whole job in one warp (its few tiles in a row), w * y added into the fp32 output
+//     accumulator.
 //   * The last CTA to finish (completion counter) converts the accumulator to bf16 and clears
 //     the accumulator and the counters for the next call.
 // Every wait is bounded; on expiry the kernel records MOE_ERR_TIMEOUT in the workspace, the
@@ -44,7 +45,7 @@ namespace {
 constexpr int kCW = 8;                      // consumer warps
 constexpr int kWarps = kCW + 1;             // + the control warp (routing plan, bulk copies)
 constexpr int kThreads = kWarps * 32;
-constexpr int kStageBytes = 24576;          // bytes per bulk copy / ring stage
+constexpr int kStageBytes = 49152;          // bytes per bulk copy / ring stage
 constexpr int kMaxStages = 8;
 constexpr int kActBytes = 65536;            // x (routing + gate/up), then h of one expert (down)
 constexpr int kMaxP = kDecodeMaxP;
