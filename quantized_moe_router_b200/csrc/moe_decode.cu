@@ -10,7 +10,7 @@
 //     layer's expert table read. Both are weights, never produced by the previous launch.
 //   * Routing. x is copied into shared memory; each CTA computes the fp32 logits of its
 //     E / nCTA experts (the dot products split over all warps) and publishes each as one 8-byte
-//     word {logit, call tag} into up to 16 copies of the T x E block, so that the CTAs' polls
+//     word {logit, call tag} into up to 32 copies of the T x E block, so that the CTAs' polls
 //     spread over the L2 slices. Every CTA polls its copy until all words carry this call's tag
 //     (derived from a completion counter that grows by nCTA per call: no barrier, no reset) and
 //     runs the same top-k + softmax: all CTAs agree on the selection without a second exchange.
@@ -147,7 +147,7 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
     return L;
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory"); }
 // named barrier 2: the control warp arrives when the plan is in shared memory, the consumer
 // warps wait for it (and for each other's group sums)
 __device__ __forceinline__ void plan_ready_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory"); }
@@ -341,15 +341,15 @@ __device__ __forceinline__ void run_tiles_seq(const uint8_t *job_base, int tb, i
 }
 
 // The warp's tiles of job `jb` (region-local) inside a chunk: k-tiles kg in [k0, k1) with
-// kg % 8 == warp, two at a time so that their MMA chains interleave.
+// kg % kCW == warp, two at a time so that their MMA chains interleave.
 template <int BITS, int NT, bool GU>
 __device__ __forceinline__ void run_tiles(const uint8_t *job_base, int tb, int k0, int k1, int warp,
                                           const JobCtx<NT> &jc, int lane, float (&acc)[NT][4],
                                           float (&acc2)[NT][4]) {
-    int kg = k0 + ((warp - k0) & 7);
-    for (; kg < k1; kg += 16) {
-        const bool two = kg + 8 < k1;
-        const int kg2 = two ? kg + 8 : kg;
+    int kg = k0 + ((warp - k0) % kCW + kCW) % kCW;   // first tile >= k0 with kg % kCW == warp
+    for (; kg < k1; kg += 2 * kCW) {
+        const bool two = kg + kCW < k1;
+        const int kg2 = two ? kg + kCW : kg;
         consume_tile<BITS, NT, GU>(job_base + (size_t)kg * tb, kg, jc, lane, acc);
         consume_tile<BITS, NT, GU>(job_base + (size_t)kg2 * tb, kg2, jc, lane, acc2, two ? 1.f : 0.f);
     }
@@ -1211,7 +1211,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         jc.bg = gu ? !xs_on : !hfit;
     };
-    // Gate/up jobs are split along K: tile k of a job goes to warp k % 8, which adds its partial
+    // Gate/up jobs are split along K: tile k of a job goes to warp k % kCW, which adds its partial
     // sums into the job's slot (CTA-local job q uses slot q % NSLOT) after its last tile of the
     // job. A down job (a few tiles) belongs to one warp and is finalised from its registers.
     auto add_partial = [&](int q) {
@@ -1223,12 +1223,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         zero_acc();
     };
     // Gate/up jobs fj0 .. fj0 + fn - 1 have all their partials in their slots (after the barrier
-    // that follows the chunk that completed them); warp gj % 8 finalises job gj.
+    // that follows the chunk that completed them); warp gj % kCW finalises job gj.
     int fj0 = 0, fn = 0;
     auto finalize_pending = [&]() {
         for (int i = 0; i < fn; ++i) {
             const int gj = fj0 + i;
-            if ((gj & (kCW - 1)) == warp) finalize_gu<NT>(a, S, gj, accs + ((gj - S.g0) % NSLOT) * SF, lane);
+            if (gj % kCW == warp) finalize_gu<NT>(a, S, gj, accs + ((gj - S.g0) % NSLOT) * SF, lane);
         }
         fn = 0;
     };
@@ -1266,7 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 else if (d.bits == 6) run_tiles<6, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
                 else run_tiles<8, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
                 if (kl >= k0 && kl < k1) add_partial(gj - S.g0);
-            } else if (((gj - S.d0) & (kCW - 1)) == warp) {
+            } else if ((gj - S.d0) % kCW == warp) {
                 if (d.bits == 4) run_tiles_seq<4, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
                 else if (d.bits == 6) run_tiles_seq<6, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
                 else run_tiles_seq<8, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
@@ -1321,11 +1321,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 }
 
 // Copies of the exchanged logit words within the fixed logit region (kMaxT x kMaxE words): the
-// T x E block at 4 KB-aligned strides, up to 16 copies.
+// T x E block at 4 KB-aligned strides, up to 32 copies.
 void logit_copies(int T, int E, int &rep, int &stride) {
     stride = (int)align_up((size_t)T * E, 512);
     rep = 1;
-    while (rep < 16 && (size_t)(rep * 2) * stride <= (size_t)kMaxT * kMaxE) rep *= 2;
+    while (rep < 32 && (size_t)(rep * 2) * stride <= (size_t)kMaxT * kMaxE) rep *= 2;
 }
 
 template <int NT>
