@@ -280,7 +280,7 @@ __device__ __forceinline__ float lds32f(uint32_t a) {
 
 template <int BITS, int NT, bool GU>
 __device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const JobCtx<NT> &jc, int lane,
-                                             float (&acc)[NT][4], float keep = 1.f) {
+                                             float (&acc)[NT][4]) {
     const int g = lane >> 2, t = lane & 3;
     const uint4 lo = *reinterpret_cast<const uint4 *>(tile + 16 * lane);
     uint4 hi8 = make_uint4(0, 0, 0, 0);
@@ -288,9 +288,7 @@ __device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const 
     if (BITS == 8) hi8 = *reinterpret_cast<const uint4 *>(tile + kLoBytes + 16 * lane);
     if (BITS == 6) hi6 = *reinterpret_cast<const uint2 *>(tile + kLoBytes + 8 * lane);
     const uint2 sz = *reinterpret_cast<const uint2 *>(tile + kLoBytes + hi_bytes(BITS) + 8 * g);
-    // keep = 0 turns the tile into a no-op (scales zeroed), so that pairs of tiles run without a
-    // branch and their MMA chains interleave
-    const float sA = keep * half_lo(sz.x), zA = half_hi(sz.x), sB = keep * half_lo(sz.y), zB = half_hi(sz.y);
+    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         // Up to two n-tiles every lane loads: a column without a token reads a valid row (the
@@ -332,12 +330,12 @@ __device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const 
 template <int BITS, int NT>
 __device__ __forceinline__ void run_tiles_seq(const uint8_t *job_base, int tb, int k0, int k1, const JobCtx<NT> &jc,
                                               int lane, float (&acc)[NT][4], float (&acc2)[NT][4]) {
-    for (int kg = k0; kg < k1; kg += 2) {
-        const bool two = kg + 1 < k1;
-        const int kg2 = two ? kg + 1 : kg;
+    int kg = k0;
+    for (; kg + 1 < k1; kg += 2) {
         consume_tile<BITS, NT, false>(job_base + (size_t)kg * tb, kg, jc, lane, acc);
-        consume_tile<BITS, NT, false>(job_base + (size_t)kg2 * tb, kg2, jc, lane, acc2, two ? 1.f : 0.f);
+        consume_tile<BITS, NT, false>(job_base + (size_t)(kg + 1) * tb, kg + 1, jc, lane, acc2);
     }
+    if (kg < k1) consume_tile<BITS, NT, false>(job_base + (size_t)kg * tb, kg, jc, lane, acc);   // odd tail
 }
 
 // The warp's tiles of job `jb` (region-local) inside a chunk: k-tiles kg in [k0, k1) with
@@ -347,12 +345,11 @@ __device__ __forceinline__ void run_tiles(const uint8_t *job_base, int tb, int k
                                           const JobCtx<NT> &jc, int lane, float (&acc)[NT][4],
                                           float (&acc2)[NT][4]) {
     int kg = k0 + ((warp - k0) % kCW + kCW) % kCW;   // first tile >= k0 with kg % kCW == warp
-    for (; kg < k1; kg += 2 * kCW) {
-        const bool two = kg + kCW < k1;
-        const int kg2 = two ? kg + kCW : kg;
+    for (; kg + kCW < k1; kg += 2 * kCW) {
         consume_tile<BITS, NT, GU>(job_base + (size_t)kg * tb, kg, jc, lane, acc);
-        consume_tile<BITS, NT, GU>(job_base + (size_t)kg2 * tb, kg2, jc, lane, acc2, two ? 1.f : 0.f);
+        consume_tile<BITS, NT, GU>(job_base + (size_t)(kg + kCW) * tb, kg + kCW, jc, lane, acc2);
     }
+    if (kg < k1) consume_tile<BITS, NT, GU>(job_base + (size_t)kg * tb, kg, jc, lane, acc);   // odd tail
 }
 
 // ------------------------------------------------------------------------------ routing
