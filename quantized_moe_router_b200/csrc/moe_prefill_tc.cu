@@ -8,9 +8,10 @@
 //   * 1 producer warp streams the unit's packed tiles from HBM into a ring of raw slots with 1-D
 //     bulk copies (one per row block and K chunk of up to 4 tiles; the copy engine, not the
 //     load/store path, so the token-row loads below do not queue behind the weight stream);
-//   * 8 dequantiser warps, one per packed 16x64 tile of the unit's 8 row blocks, read their tile
-//     from the raw slot and write w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile
-//     A [128 x 64];
+//   * 4 dequantiser warps, each taking two of the unit's 8 row blocks per K step (the two tiles'
+//     work interleaves; measured faster than 8 warps of one tile, which compete for issue slots
+//     with the rest of the SM), read their packed 16x64 tiles from the raw slot and write
+//     w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile A [128 x 64];
 //   * 1 loader thread brings the unit's token rows into a swizzled tile B [N x 64] with 2-D tensor
 //     copies (TMA, 64 rows each, the 128-byte swizzle applied by the copy engine): gate/up reads
 //     x16, the pairs' hidden states in bucket order as fp16 (scaled per token by a power of two
@@ -40,7 +41,7 @@ constexpr int kMaxN = 256;                        // tokens per unit (UMMA N lim
 constexpr int kABStages = 3;
 constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
 constexpr int kMaxRaw = 8;                        // raw ring slots (K chunks) at most
-constexpr int kDqWarps = 8, kLdWarps = 1;
+constexpr int kDqWarps = 4, kLdWarps = 1;
 constexpr int kRowBox = 64;                       // token rows per tensor copy
 constexpr int kMmaWarp = kDqWarps + kLdWarps;
 constexpr int kEpiWarp0 = kMmaWarp + 1;
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
 
     if (warp < kDqWarps) {
         // ------------------------------------------------------------ dequantisers
-        const int b = warp;
+        const int b0 = warp, b1 = warp + 4;
         bool ok = run;
         const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
         // step counters kept incrementally (no division in the loop): position jk in the K
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
             // per unit: the expert's width and whether this warp's row block exists
             const int bits = __ldg(&pe[U.e].bits);
             const int tb = tile_bytes(bits);
-            const bool have = 8 * U.mt + b < G.nrb;
+            const bool have0 = 8 * U.mt + b0 < G.nrb, have1 = 8 * U.mt + b1 < G.nrb;
             for (int kg = 0; kg < G.KG; ++kg) {
                 if (jk == 0 && !tc_wait(S, a, &S.raw_full[rs], rpar)) {
                     ok = false;
@@ -396,21 +397,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 uint8_t *As = ring + (size_t)slot * stage_bytes;
-                const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + jk) * tb;
-                if (!have) {
-                    // row block past the matrix: zero rows (the epilogue skips them)
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    const int g = lane >> 2, t = lane & 3;
-                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t)) = z;
-                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t + 1)) = z;
-                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t)) = z;
-                    *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t + 1)) = z;
-                } else if (bits == 4) {
-                    dequant_fragment<4>(rawt, lane, As, b);
-                } else if (bits == 8) {
-                    dequant_fragment<8>(rawt, lane, As, b);
+                const uint8_t *rawt0 = raw + (size_t)rs * slot_bytes + (size_t)(b0 * KC + jk) * tb;
+                const uint8_t *rawt1 = raw + (size_t)rs * slot_bytes + (size_t)(b1 * KC + jk) * tb;
+                if (have0 && have1 && bits == 4) {
+                    dequant_fragment<4>(rawt0, lane, As, b0);
+                    dequant_fragment<4>(rawt1, lane, As, b1);
                 } else {
-                    dequant_fragment<6>(rawt, lane, As, b);
+#pragma unroll 1
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const int b = bb ? b1 : b0;
+                        const bool have = bb ? have1 : have0;
+                        const uint8_t *rawt = bb ? rawt1 : rawt0;
+                        if (!have) {
+                            const uint4 z = make_uint4(0, 0, 0, 0);
+                            const int g = lane >> 2, t = lane & 3;
+                            *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t)) = z;
+                            *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t + 1)) = z;
+                            *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t)) = z;
+                            *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t + 1)) = z;
+                        } else if (bits == 4) {
+                            dequant_fragment<4>(rawt, lane, As, b);
+                        } else if (bits == 8) {
+                            dequant_fragment<8>(rawt, lane, As, b);
+                        } else {
+                            dequant_fragment<6>(rawt, lane, As, b);
+                        }
+                    }
                 }
                 fence_proxy_async();  // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
