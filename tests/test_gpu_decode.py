@@ -127,3 +127,24 @@ def test_decode_workspace_shared_across_shapes():
         x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
         out, idx, w = decode_call(layer, x, I, E, k, ws)
         check_block(oracle.get(), x, layer.wr_np, layer.bias_np, layer.expert_fn, E, H, I, k, out, idx, w)
+
+
+@pytest.mark.parametrize("E,k,dups", [
+    (16, 16, [(2, 5), (0, 15)]),      # one expert per lane: ties between lanes (the exact fallback)
+    (40, 32, [(3, 35), (10, 20)])])   # a tie inside a lane (3, 35) and one between lanes (10, 20)
+def test_decode_exact_ties_take_lower_index(E, k, dups):
+    rng = np.random.default_rng(E * 31 + k)
+    T, H, I = 5, 128, 64
+    layer0 = hand_layer(rng, E, H, I, [4], bias=False)
+    wr = layer0.wr_np.copy()
+    for lo, hi in dups:
+        wr[hi] = wr[lo]            # identical logits in every precision
+    layer = HandLayer(layer0.experts_np, wr, None, H, I)
+    x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
+    out, idx, w = decode_call(layer, x, I, E, k)
+    for t in range(T):
+        pos = {int(e): i for i, e in enumerate(idx[t])}
+        for lo, hi in dups:
+            if lo in pos and hi in pos:
+                assert pos[lo] < pos[hi], (t, lo, hi, idx[t])   # equal logits: lower index first
+    check_block(oracle.get(), x, layer.wr_np, layer.bias_np, layer.expert_fn, E, H, I, k, out, idx, w)
