@@ -94,5 +94,15 @@ def test_host_validation_before_any_launch(L):
     src = (qm.ExpertSrc * 1)()
     src[0].bits = 5
     assert L.moe_pack_layer(C.cast(src, C.c_void_p), 1, 128, 64, fake, 1 << 20, None) == qm.MOE_ERR_INVALID_ARG
+    # the two halves of prefill: workspace too small, null or misaligned pointers, bad shape
+    big = 1 << 30
+    assert L.moe_prefill_route(fake, fake, None, 4, 2048, 512, 256, 8, None, None, fake, ws_small, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_route(fake, None, None, 4, 2048, 512, 256, 8, None, None, fake, big, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_route(fake + 2, fake, None, 4, 2048, 512, 256, 8, None, None, fake, big, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_route(fake, fake, None, 4, 2048, 512, 256, 33, None, None, fake, big, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_experts(fake, fake, 4, 2048, 512, 256, 8, fake, fake, ws_small, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_experts(fake, None, 4, 2048, 512, 256, 8, fake, fake, big, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_experts(fake, fake, 4, 2048, 512, 256, 8, fake + 8, fake, big, None) == qm.MOE_ERR_INVALID_ARG
+    assert L.moe_prefill_experts(fake, fake, 4, 2000, 512, 256, 8, fake, fake, big, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_workspace_init(None, 1024, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_status(None, None) == qm.MOE_ERR_INVALID_ARG
