@@ -202,6 +202,17 @@ def oracle_decode_sample(w, steps, layers, threads=None):
     return total, steps * w.T, o.threads()
 
 
+def metric_name(w):
+    return ("decode" if w.mode == "decode" else "prefill") + " tokens/s (MoE expert block, all layers)"
+
+
+def base_config(w, world):
+    """The workload keys of the config object, the same on both arms."""
+    return {"workload": w.name, "tokens_per_step": w.T, "layers": w.layers, "H": w.H, "E": w.E, "k": w.k,
+            "I": w.I, "weights": "mixed 4/6/8-bit" if w.mixed_bits else f"int{w.bits} group-64 affine",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, w):
     """--impl reference: the fp64 oracle on the host cores, one step = one decode token through
     `layers_per_step` layers of the workload (a bounded sample), rank 0 only."""
@@ -218,12 +229,13 @@ def run_reference(args, w):
     per_step = statistics.mean(times)
     # tokens/s of the full workload: one token needs all w.layers layers
     value = w.T / (per_step * w.layers / layers)
-    sample = f"{args.steps} steps, each 1 decode token through {layers} of {w.layers} layers (fp64), scaled to all layers"
+    sample = (f"{args.steps} steps, each 1 token through {layers} of {w.layers} layers (fp64; tokens are "
+              f"independent in this block), scaled to all layers")
     line = {
-        "impl": "reference", "metric": "decode tokens/s", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_name(w), "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * w.layers / layers * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name},
+        "config": base_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -265,14 +277,13 @@ def run_ours(args, w):
     rank, world, local = dist_setup(args.gpus)
     if w.mode == "prefill":
         res = run_prefill(args, w, world, rank)
+        res.pop("workload")
         line = {"metric": res.pop("metric"), "value": res.pop("value"), "unit": res.pop("unit"), "n_gpus": world,
                 "steps": res.pop("steps"), "warmup": max(args.warmup, 3), "ms_per_step": res.pop("ms_per_step"),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic",
-                "config": {"workload": res.pop("workload"), "tokens_per_step": w.T, "layers": w.layers, "H": w.H,
-                           "E": w.E, "k": w.k, "I": w.I, "weights": f"int{w.bits} group-64 affine",
-                           "l2": "no flush: each layer streams ~453 MB of expert weights (> 126 MB L2)",
-                           "parallelism": f"replicas x{world}"},
+                "config": dict(base_config(w, world),
+                               l2="no flush: each layer streams the weights of all its experts (> 126 MB L2)"),
                 "gpu_launches": res["steps_launches"], **{k: v for k, v in res.items() if k != "steps_launches"}}
         if rank == 0:
             print(json.dumps(line), flush=True)
@@ -365,7 +376,7 @@ def run_ours(args, w):
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
 
     line = {
-        "metric": "decode tokens/s (MoE expert block, all layers)",
+        "metric": metric_name(w),
         "value": world * w.T * args.steps / (ms * 1e-3),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -377,11 +388,9 @@ def run_ours(args, w):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "tokens_per_step": w.T, "layers": w.layers, "H": w.H, "E": w.E, "k": w.k,
-                   "I": w.I, "weights": "mixed 4/6/8-bit" if w.mixed_bits else f"int{w.bits} group-64 affine",
-                   "l2": "no flush: each step streams ~%.0f MB of expert weights (> 126 MB L2); %.1f GB resident"
-                         % (expert_b * w.layers / 1e6, sum(lw.packed.numel() for lw in layers) / 1e9),
-                   "parallelism": f"replicas x{world}"},
+        "config": dict(base_config(w, world),
+                       l2="no flush: each step streams ~%.0f MB of expert weights (> 126 MB L2); %.1f GB resident"
+                          % (expert_b * w.layers / 1e6, sum(lw.packed.numel() for lw in layers) / 1e9)),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": traffic, "peak_source": peak_src,
                      "bytes_per_launch": layer_bytes, "kernel_ms_per_launch": kern_ms,
@@ -481,7 +490,7 @@ def run_prefill(args, w, world, rank):
     _, bf16, peak_src = measured_peaks()
     achieved = prefill_flops(w) / (gemm_ms * 1e-3) / 1e12
     res = {
-        "workload": w.name, "metric": "prefill tokens/s (MoE expert block, all layers)",
+        "workload": w.name, "metric": metric_name(w),
         "value": world * w.T * nsteps / (ms * 1e-3), "unit": "tokens/s", "steps": nsteps,
         "ms_per_step": ms / nsteps, "ms_per_layer": ms / nsteps / w.layers,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
