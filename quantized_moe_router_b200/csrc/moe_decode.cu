@@ -148,6 +148,18 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory"); }
+// The same barrier, returning the OR of `flag` over the consumer threads: a decision that all
+// consumer warps take identically (S.abort can change at any time, so reading it after a plain
+// barrier could split the warps).
+__device__ __forceinline__ bool consumer_sync_or(bool flag) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag), "n"(kCW * 32)
+        : "memory");
+    return r != 0;
+}
 // named barrier 2: the control warp arrives when the plan is in shared memory, the consumer
 // warps wait for it (and for each other's group sums)
 __device__ __forceinline__ void plan_ready_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory"); }
@@ -1237,11 +1249,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool more = S.g1 > S.g0 || S.d1 > S.d0;
     while (more) {
         const bool got = !S.abort && mbar_wait(smem_u32(&S.full[s]), par, a.wait_ns, status);
-        if (!got && lane == 0) S.abort = 1;
         // One barrier per chunk: every warp's partials of the previous chunk are in, and all
-        // warps agree on an abort.
-        consumer_sync();
-        if (S.abort) break;
+        // warps take the same abort decision.
+        if (consumer_sync_or(!got || S.abort)) {
+            if (lane == 0) S.abort = 1;
+            break;
+        }
         finalize_pending();
         const ChunkDesc d = S.desc[s];
         const bool gu = d.flags & 1;
@@ -1283,8 +1296,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             par ^= 1u;
         }
     }
-    consumer_sync();
-    if (!S.abort) {
+    if (!consumer_sync_or(S.abort)) {
         finalize_pending();
         if (!published) {
             // no down job here: the gate/up rows are published after their finalisers are done
