@@ -31,6 +31,11 @@ def build(src: str = SRC, out: str = LIB, extra: Sequence[str] = ()) -> str:
     return out
 
 
+# Published defaults of the HQQ zero-point optimiser (l_p norm, initial beta, beta growth
+# per iteration, iteration cap).
+HQQ_P, HQQ_BETA, HQQ_KAPPA, HQQ_ITERS = 0.7, 10.0, 1.01, 20
+
+
 class _Expert(C.Structure):
     _fields_ = [("codes", C.c_void_p * 3), ("scale", C.c_void_p * 3), ("zero", C.c_void_p * 3),
                 ("bits", C.c_int32)]
@@ -59,6 +64,14 @@ class Oracle:
         L.oracle_weight.restype = C.c_double
         L.oracle_max_threads.restype = C.c_int
         L.oracle_set_threads.argtypes = [C.c_int]
+        f64 = C.c_double
+        L.oracle_f64_to_f16.argtypes = [f64]
+        L.oracle_f64_to_f16.restype = C.c_uint16
+        L.oracle_hqq_shrink.argtypes = [f64, f64, f64]
+        L.oracle_hqq_shrink.restype = f64
+        L.oracle_hqq_group.argtypes = [vp, i32, f64, f64, f64, i32, vp, vp, vp, vp, vp, vp]
+        L.oracle_hqq_quantize.argtypes = [vp, i32, i32, i32, f64, f64, f64, i32, vp, vp, vp, vp]
+        L.oracle_hqq_codes.argtypes = [vp, i32, i32, i32, vp, vp, vp]
 
     # -------------------------------------------------------------- marshalling helpers
     @staticmethod
@@ -147,6 +160,55 @@ class Oracle:
         idx, w = self.topk(logits, k)
         out = self.combine(x_bf16, experts, H, I, idx, w)
         return out, idx, w, logits
+
+    # -------------------------------------------------------------- quantiser
+    def f64_to_f16(self, v: float) -> int:
+        """IEEE binary16 bits of v, round to nearest even."""
+        return int(self.lib.oracle_f64_to_f16(float(v)))
+
+    def hqq_shrink(self, x: float, beta: float, p: float) -> float:
+        """The generalised soft threshold of the zero-point iteration."""
+        return float(self.lib.oracle_hqq_shrink(float(x), float(beta), float(p)))
+
+    def hqq_group(self, w: np.ndarray, bits: int, p: float = HQQ_P, beta: float = HQQ_BETA,
+                  kappa: float = HQQ_KAPPA, iters: int = HQQ_ITERS):
+        """One group of 64 fp64 weights: (s16 bits, z16 bits, codes [64], z trace, err trace)."""
+        w = np.ascontiguousarray(w, dtype=np.float64).reshape(64)
+        s16, z16 = C.c_uint16(), C.c_uint16()
+        q = np.empty(64, np.uint8)
+        zt = np.empty(max(iters, 1), np.float64)
+        et = np.empty(max(iters, 1), np.float64)
+        ran = C.c_int()
+        self.lib.oracle_hqq_group(_ptr(w), bits, p, beta, kappa, iters, C.addressof(s16),
+                                  C.addressof(z16), _ptr(q), _ptr(zt), _ptr(et),
+                                  C.addressof(ran))
+        return s16.value, z16.value, q, zt[:ran.value].copy(), et[:ran.value].copy()
+
+    def hqq_quantize(self, w_bf16: np.ndarray, bits: int, p: float = HQQ_P,
+                     beta: float = HQQ_BETA, kappa: float = HQQ_KAPPA, iters: int = HQQ_ITERS):
+        """bf16 bits [rows x cols] -> (codes uint8 [rows x cols], s16 bits, z16 bits
+        [rows x cols/64], iterations run per group [rows x cols/64])."""
+        w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+        rows, cols = w.shape
+        if cols % 64 or bits not in (4, 6, 8) or iters < 0:
+            raise ValueError("cols must be a multiple of 64, bits 4/6/8, iters >= 0")
+        q = np.empty((rows, cols), np.uint8)
+        s16 = np.empty((rows, cols // 64), np.uint16)
+        z16 = np.empty((rows, cols // 64), np.uint16)
+        ran = np.empty((rows, cols // 64), np.int32)
+        self.lib.oracle_hqq_quantize(_ptr(w), rows, cols, bits, p, beta, kappa, iters, _ptr(q),
+                                     _ptr(s16), _ptr(z16), _ptr(ran))
+        return q, s16, z16, ran
+
+    def hqq_codes(self, w_bf16: np.ndarray, bits: int, s16: np.ndarray, z16: np.ndarray):
+        """Nearest codes of bf16 weights on the grid of the given fp16 scale and zero bits."""
+        w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+        rows, cols = w.shape
+        s = np.ascontiguousarray(s16, dtype=np.uint16).reshape(rows, cols // 64)
+        z = np.ascontiguousarray(z16, dtype=np.uint16).reshape(rows, cols // 64)
+        q = np.empty((rows, cols), np.uint8)
+        self.lib.oracle_hqq_codes(_ptr(w), rows, cols, bits, _ptr(s), _ptr(z), _ptr(q))
+        return q
 
 
 _default: Optional[Oracle] = None

@@ -200,3 +200,159 @@ void oracle_moe_forward(const uint16_t *x, const float *wr, const float *bias,
     oracle_combine(x, experts, T, H, I, E, k, idx, w, out);
     if (!logits) free(l);
 }
+
+/* ============================================================================= quantiser
+ *
+ * HQQ-style group quantiser: bf16 weights -> the canonical (codes, fp16 scale, fp16 zero)
+ * format read above. The page "Krasis update" (list of the v1.0 results, the item on 4/6/8-bit
+ * sensitivity-aware HQQ) names Half-Quadratic Quantization at 4, 6 and 8 bits, built from the
+ * weights alone with no calibration run, but prints no steps. The steps below restate the published method
+ * (H. Badri and A. Shaji, "Half-Quadratic Quantization of Large Machine Learning Models",
+ * 2023): the min-max scale of each group is kept, and only the zero point is optimised. It
+ * minimises an l_p norm (p < 1) of the reconstruction error by half-quadratic splitting, which
+ * alternates a closed-form shrinkage of the error with a closed-form least-squares zero.
+ *
+ * One group w_0..w_63 (fp64, exact from bf16), Q = 2^b - 1, all arithmetic in fp64:
+ *   1. lo = min w, hi = max w; a constant group c is widened to [min(c, 0), max(c, 0)], and
+ *      an all-zero group to [0, Q].
+ *      s = fp16((hi - lo) / Q), at least the smallest positive fp16 and at most 65504;
+ *      z_0 = -lo / s (s is the stored fp16 value from here on).
+ *   2. For i = 0 .. iters-1, with beta_0 = beta and beta_{i+1} = kappa * beta_i:
+ *        q_j = clamp(rint(w_j / s + z_i), 0, Q),   r_j = (q_j - z_i) * s
+ *        err_i = sum_j |w_j - r_j|; if err_i is not below the best so far, stop;
+ *               otherwise z_i becomes the best zero
+ *        e_j = shrink_p(w_j - r_j, beta_i)
+ *        z_{i+1} = (1/64) * sum_j (q_j - (w_j - e_j) / s)
+ *      with the generalised soft threshold
+ *      shrink_p(x, beta) = sign(x) * max(|x| - |x|^(p-1) / beta, 0), and shrink_p(0) = 0.
+ *      For p = 1 this is the proximal map of |x| / beta (the soft threshold).
+ *   3. z = fp16(best zero), clamped to +-65504; q_j = clamp(rint(w_j / s + z), 0, Q) with the
+ *      stored fp16 s and z. These are the nearest points of the stored grid.
+ * The readings this takes where the published text leaves room: the stop rule and the best
+ * zero are per group (the objective is a sum of independent group terms); the codes are
+ * recomputed from the stored fp16 scale and zero; iters = 0 is plain min-max rounding.
+ */
+
+/* double -> IEEE binary16 bits, round to nearest, ties to even (from the format's definition:
+ * 11 significant bits for normal values, a fixed quantum of 2^-24 below 2^-14, and infinity
+ * from 65520 = 65504 + half a unit in the last place up) */
+uint16_t oracle_f64_to_f16(double v) {
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isnan(v)) return 0x7E00;
+    if (a >= 65520.0) return (uint16_t)(sign | 0x7C00);
+    int e;
+    (void)frexp(a, &e);                       /* a in [2^(e-1), 2^e) */
+    int qe = e - 11;                          /* quantum of an 11-bit significand */
+    if (qe < -24) qe = -24;                   /* subnormal spacing */
+    double n = rint(ldexp(a, -qe));           /* exact power-of-two scaling, then RNE */
+    double r = ldexp(n, qe);
+    if (r == 0.0) return sign;
+    if (r < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)n);
+    int re;
+    double m = frexp(r, &re);                 /* r = m * 2^re, m in [0.5, 1) */
+    uint16_t ex = (uint16_t)(re - 1 + 15);
+    uint16_t man = (uint16_t)((2.0 * m - 1.0) * 1024.0);
+    return (uint16_t)(sign | (uint16_t)(ex << 10) | man);
+}
+
+double oracle_hqq_shrink(double x, double beta, double p) {
+    if (x == 0.0) return 0.0;
+    double a = fabs(x);
+    double t = a - pow(a, p - 1.0) / beta;
+    return t > 0.0 ? copysign(t, x) : 0.0;
+}
+
+static double hqq_code(double w, double s, double z, double qmax) {
+    double q = rint(w / s + z);
+    return fmin(fmax(q, 0.0), qmax);
+}
+
+/* One group of ORACLE_GROUP weights. Outputs the stored scale/zero bits and the codes; the
+ * optional traces receive z_i and err_i of every iteration that ran (at most iters entries),
+ * *n_iter how many ran. */
+void oracle_hqq_group(const double *w, int bits, double p, double beta, double kappa,
+                      int iters, uint16_t *s16, uint16_t *z16, uint8_t *q_out,
+                      double *z_trace, double *err_trace, int *n_iter) {
+    const int n = ORACLE_GROUP;
+    double qmax = (double)((1 << bits) - 1);
+    double lo = w[0], hi = w[0];
+    for (int j = 1; j < n; j++) {
+        if (w[j] < lo) lo = w[j];
+        if (w[j] > hi) hi = w[j];
+    }
+    if (lo == hi) {
+        if (lo == 0.0) {
+            hi = qmax;
+        } else {
+            lo = fmin(lo, 0.0);
+            hi = fmax(hi, 0.0);
+        }
+    }
+    uint16_t sb = oracle_f64_to_f16(fmin((hi - lo) / qmax, 65504.0));
+    if (sb == 0) sb = 1;
+    double s = f16_to_f64(sb);
+    double z = -lo / s;
+    double zbest = z, best = INFINITY;
+    double q[ORACLE_GROUP], r[ORACLE_GROUP];
+    int ran = 0;
+    for (int i = 0; i < iters; i++) {
+        double err = 0.0;
+        for (int j = 0; j < n; j++) {
+            q[j] = hqq_code(w[j], s, z, qmax);
+            r[j] = (q[j] - z) * s;
+            err += fabs(w[j] - r[j]);
+        }
+        if (z_trace) z_trace[i] = z;
+        if (err_trace) err_trace[i] = err;
+        ran = i + 1;
+        if (!(err < best)) break;
+        best = err;
+        zbest = z;
+        double acc = 0.0;
+        for (int j = 0; j < n; j++) {
+            double e = oracle_hqq_shrink(w[j] - r[j], beta, p);
+            acc += q[j] - (w[j] - e) / s;
+        }
+        z = acc / (double)n;
+        beta *= kappa;
+    }
+    uint16_t zb = oracle_f64_to_f16(fmin(fmax(zbest, -65504.0), 65504.0));
+    double zs = f16_to_f64(zb);
+    for (int j = 0; j < n; j++) q_out[j] = (uint8_t)hqq_code(w[j], s, zs, qmax);
+    *s16 = sb;
+    *z16 = zb;
+    if (n_iter) *n_iter = ran;
+}
+
+/* A bf16 matrix [rows x cols] (cols a multiple of 64), one group per 64 columns of a row:
+ * codes q [rows x cols] (one byte each, unpacked), scale and zero bits [rows x cols/64],
+ * iterations run per group (nullable). */
+void oracle_hqq_quantize(const uint16_t *w_bf16, int rows, int cols, int bits, double p,
+                         double beta, double kappa, int iters, uint8_t *q, uint16_t *s16,
+                         uint16_t *z16, int32_t *iters_used) {
+    int gpr = cols / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (long g = 0; g < (long)rows * gpr; g++) {
+        long r = g / gpr, c0 = (g % gpr) * ORACLE_GROUP;
+        double w[ORACLE_GROUP];
+        for (int j = 0; j < ORACLE_GROUP; j++) w[j] = bf16_to_f64(w_bf16[r * cols + c0 + j]);
+        int ran = 0;
+        oracle_hqq_group(w, bits, p, beta, kappa, iters, &s16[g], &z16[g], &q[r * cols + c0],
+                         NULL, NULL, &ran);
+        if (iters_used) iters_used[g] = ran;
+    }
+}
+
+/* Step 3 alone: the nearest codes of bf16 weights for given fp16 scale and zero bits. */
+void oracle_hqq_codes(const uint16_t *w_bf16, int rows, int cols, int bits,
+                      const uint16_t *s16, const uint16_t *z16, uint8_t *q) {
+    int gpr = cols / ORACLE_GROUP;
+    double qmax = (double)((1 << bits) - 1);
+    for (long r = 0; r < rows; r++)
+        for (long c = 0; c < cols; c++) {
+            long g = r * gpr + c / ORACLE_GROUP;
+            q[r * cols + c] = (uint8_t)hqq_code(bf16_to_f64(w_bf16[r * cols + c]),
+                                                f16_to_f64(s16[g]), f16_to_f64(z16[g]), qmax);
+        }
+}

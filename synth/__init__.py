@@ -24,8 +24,8 @@ Generator (identical on the host, here, and on the device, ``synth/csrc/synth.cu
 * Storage rounding: double -> fp32 round-to-nearest-even (RNE); fp32 -> bf16 RNE;
   fp32 -> fp16 RNE. (fp16/bf16 values are therefore rounded twice, by definition.)
 
-Workload recipes (the synthetic configurations; the readings of the recipe text are listed
-in DESIGN.md):
+Workload recipes (the synthetic configurations, with the readings taken where the recipe
+text is open):
 
 * x ~ N(0, 1) rounded to bf16, a fresh draw per (step, layer).
 * router weights W_r ~ N(0, 1/H) (second argument = variance), fp32, [E x H] row-major.

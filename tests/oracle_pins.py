@@ -295,6 +295,239 @@ def pin_onehot_x(o):
             assert np.array_equal(g, dense[0][:, j]) and np.array_equal(u, dense[1][:, j])
 
 
+# ----------------------------------------------------------------------------- quantiser pins
+
+def grid_distances(w, s, z, Q):
+    """|w_j - (q - z) * s| for every weight j and every code q in 0..Q (brute force)."""
+    cand = (np.arange(Q + 1, dtype=np.float64) - z) * s
+    return np.abs(np.asarray(w, np.float64)[:, None] - cand[None, :])
+
+
+def check_nearest(w, q, s, z, Q, what=""):
+    """Every code is a nearest point of the grid (q - z) * s, q in 0..Q."""
+    d = grid_distances(w, s, z, Q)
+    chosen = d[np.arange(len(w)), np.asarray(q, np.int64)]
+    assert np.all(chosen <= d.min(1) + 1e-12 * s), what
+
+
+def f16_of(v):
+    """numpy's binary16 rounding of a double (round to nearest even), as bits."""
+    with np.errstate(over="ignore"):
+        return int(np.array([v], np.float64).astype(np.float16).view(np.uint16)[0])
+
+
+def pin_f16_conversion(o):
+    """The oracle's double -> binary16 rounding equals numpy's, ties, subnormals and overflow
+    included."""
+    rng = np.random.default_rng(30)
+    vals = list(rng.normal(0, 1, 400) * 10.0 ** rng.integers(-9, 6, 400))
+    h = np.arange(0, 0x7BFF, 37, dtype=np.uint16)
+    hv = h.view(np.float16).astype(np.float64)
+    nv = (h + 1).view(np.float16).astype(np.float64)
+    mid = (hv + nv) / 2                                     # exact in fp64: ties
+    vals += list(hv) + list(mid) + list(np.nextafter(mid, 0)) + list(np.nextafter(mid, 1e9))
+    vals += [0.0, 65504.0, 65519.99, 65520.0, 1e6, 2.0 ** -24, 2.0 ** -25, 2.0 ** -25 * 1.001,
+             2.0 ** -26, 3 * 2.0 ** -25, 2.0 ** -14 - 2.0 ** -25, 1e-300]
+    for v in vals:
+        for sg in (1.0, -1.0):
+            assert o.f64_to_f16(sg * v) == f16_of(sg * v), (sg * v, hex(o.f64_to_f16(sg * v)))
+
+
+def pin_hqq_minmax_rounding(o):
+    """iters = 0 is min-max rounding: s = fp16((max - min) / Q) and z = fp16(-min / s) as numpy
+    rounds them, and every code is a nearest grid point (brute force over all 2^b codes)."""
+    rng = np.random.default_rng(31)
+    for bits in (4, 6, 8):
+        Q = (1 << bits) - 1
+        wb = synth.to_bf16_bits(rng.normal(0, 0.05, (6, 256)) + rng.normal(0, 0.03, (6, 1)))
+        q, s16, z16, ran = o.hqq_quantize(wb, bits, iters=0)
+        assert np.all(ran == 0)
+        w = xf(wb)
+        for r in range(6):
+            for g in range(4):
+                wg = w[r, G * g:G * (g + 1)]
+                lo, hi = wg.min(), wg.max()
+                assert s16[r, g] == f16_of((hi - lo) / Q), bits
+                s = f16(s16[r, g])
+                assert z16[r, g] == f16_of(-lo / s), bits
+                check_nearest(wg, q[r, G * g:G * (g + 1)], s, f16(z16[r, g]), Q, bits)
+
+
+def pin_hqq_codes_nearest(o):
+    """After the zero-point iteration, and for arbitrary given scales and zeros, every code is a
+    nearest point of the stored fp16 grid."""
+    rng = np.random.default_rng(32)
+    for bits, p, beta in ((4, 0.7, 10.0), (6, 0.7, 1e4), (8, 1.0, 1e3), (4, 0.5, 1e5)):
+        Q = (1 << bits) - 1
+        wb = synth.to_bf16_bits(rng.standard_t(3, (5, 192)) * 0.03)
+        q, s16, z16, _ = o.hqq_quantize(wb, bits, p=p, beta=beta)
+        w = xf(wb)
+        for r in range(5):
+            for g in range(3):
+                sl = slice(G * g, G * (g + 1))
+                check_nearest(w[r, sl], q[r, sl], f16(s16[r, g]), f16(z16[r, g]), Q, bits)
+        s_any = synth.to_f16_bits(np.abs(rng.normal(0, 0.01, (5, 3))) + 1e-4)
+        z_any = synth.to_f16_bits(rng.uniform(-5, Q + 5, (5, 3)))
+        q2 = o.hqq_codes(wb, bits, s_any, z_any)
+        for r in range(5):
+            for g in range(3):
+                sl = slice(G * g, G * (g + 1))
+                check_nearest(w[r, sl], q2[r, sl], f16(s_any[r, g]), f16(z_any[r, g]), Q, bits)
+
+
+def pin_hqq_exact_grid(o):
+    """Weights that already lie on a b-bit grid spanning codes 0..Q come back exactly (scale,
+    zero and codes), with and without the zero-point iteration."""
+    rng = np.random.default_rng(33)
+    for bits in (4, 6, 8):
+        Q = (1 << bits) - 1
+        rows = 8
+        q = rng.integers(0, Q + 1, (rows, 2 * G))
+        q[:, 0], q[:, G - 1], q[:, G], q[:, 2 * G - 1] = 0, Q, Q, 0
+        s = 2.0 ** rng.integers(-9, -3, (rows, 2)).astype(np.float64)
+        z = rng.integers(0, Q + 1, (rows, 2)).astype(np.float64)
+        w = (q - np.repeat(z, G, 1)) * np.repeat(s, G, 1)
+        wb = synth.to_bf16_bits(w)
+        assert np.array_equal(xf(wb), w)
+        for iters in (0, 20):
+            qq, s16, z16, _ = o.hqq_quantize(wb, bits, iters=iters)
+            assert np.array_equal(qq, q) and np.array_equal(f16(s16), s), (bits, iters)
+            assert np.array_equal(f16(z16), z), (bits, iters)
+
+
+TRACE_CASES = ((4, 0.7, 10.0, 1.01, 1.0), (4, 0.7, 1e4, 1.01, 0.05), (6, 1.0, 1e3, 1.05, 0.5),
+               (8, 0.5, 1e5, 1.2, 0.02), (4, 1.0, 30.0, 1.01, 2.0))
+
+
+def pin_hqq_trace(o):
+    """Each iteration's error is the brute-force L1 distance of the group to its nearest grid
+    points at that iteration's zero; errors fall strictly until the iteration that stops; the
+    stored zero is the fp16 value of the zero with the least error."""
+    rng = np.random.default_rng(34)
+    for bits, p, beta, kappa, scale in TRACE_CASES:
+        Q = (1 << bits) - 1
+        for _ in range(12):
+            wg = xf(synth.to_bf16_bits(rng.standard_t(3, G) * scale))
+            s16, z16, q, zt, et = o.hqq_group(wg, bits, p=p, beta=beta, kappa=kappa, iters=20)
+            s = f16(s16)
+            assert 1 <= len(et) <= 20
+            for i in range(len(et)):
+                err = grid_distances(wg, s, zt[i], Q).min(1).sum()
+                assert abs(et[i] - err) <= 1e-12 * max(err, s), (bits, i)
+            assert np.all(np.diff(et[:-1]) < 0)
+            if len(et) < 20:
+                assert et[-1] >= et[-2]
+            best = int(np.argmin(et))
+            assert z16 == f16_of(zt[best]), (bits, best)
+
+
+def pin_hqq_zero_update(o):
+    """Each new zero is the least-squares solution (numpy lstsq) of q - z = (w - e) / s, with q
+    the nearest codes at the previous zero, e the shrunk residual and beta_i = beta * kappa^i."""
+    rng = np.random.default_rng(35)
+    for bits, p, beta, kappa, scale in TRACE_CASES:
+        Q = (1 << bits) - 1
+        for _ in range(8):
+            wg = xf(synth.to_bf16_bits(rng.standard_t(3, G) * scale))
+            s16, _, _, zt, _ = o.hqq_group(wg, bits, p=p, beta=beta, kappa=kappa, iters=20)
+            s = f16(s16)
+            for i in range(len(zt) - 1):
+                qn = grid_distances(wg, s, zt[i], Q).argmin(1)
+                res = wg - (qn - zt[i]) * s
+                e = np.array([o.hqq_shrink(x, beta * kappa ** i, p) for x in res])
+                rhs = qn - (wg - e) / s
+                z_ls = np.linalg.lstsq(np.ones((G, 1)), rhs, rcond=None)[0][0]
+                assert abs(zt[i + 1] - z_ls) <= 1e-10 * max(1.0, abs(z_ls)), (bits, i)
+
+
+def pin_hqq_shrink(o):
+    """p = 1: the shrink is the proximal map of |y| / beta (brute-force minimisation). p < 1: an
+    odd map toward 0 that is exactly 0 up to |x| = beta^(-1/(2-p)) and nonzero beyond, grows
+    with beta, and tends to the p = 1 map as p -> 1."""
+    from scipy.optimize import minimize_scalar
+    rng = np.random.default_rng(36)
+    for beta in (0.5, 3.0, 40.0):
+        for x in rng.normal(0, 2.0 / beta, 25):
+            f = lambda y, x=x: 0.5 * (y - x) ** 2 + abs(y) / beta  # noqa: E731
+            r = minimize_scalar(f, bounds=(-abs(x) - 1, abs(x) + 1), method="bounded",
+                                options={"xatol": 1e-13})
+            assert abs(o.hqq_shrink(x, beta, 1.0) - r.x) < 1e-7, (beta, x)
+    for p in (0.5, 0.7, 0.9):
+        for beta in (10.0, 1e3):
+            thr = beta ** (-1.0 / (2.0 - p))
+            for m in (0.1, 0.5, 0.99, 0.9999, 1.0001, 1.01, 2.0, 10.0):
+                for x in (m * thr, -m * thr):
+                    e = o.hqq_shrink(x, beta, p)
+                    assert o.hqq_shrink(-x, beta, p) == -e
+                    if m < 1:
+                        assert e == 0.0, (p, beta, m)
+                    else:
+                        assert e != 0 and np.sign(e) == np.sign(x) and abs(e) < abs(x), (p, m)
+                        assert abs(o.hqq_shrink(x, 2 * beta, p)) > abs(e)
+            x = 3 * thr
+            assert abs(o.hqq_shrink(x, beta, 1 - 1e-9) - o.hqq_shrink(x, beta, 1.0)) < 1e-6 * x
+    assert o.hqq_shrink(0.0, 10.0, 0.7) == 0.0
+
+
+def pin_hqq_constant_groups(o):
+    """An all-zero group is stored exactly; a constant group c is reproduced to fp16 precision."""
+    for bits in (4, 6, 8):
+        Q = (1 << bits) - 1
+        for c in (0.0, 0.75, -0.0390625, 3.0e-3, -7.5):
+            wb = synth.to_bf16_bits(np.full((1, G), c))
+            cv = float(xf(wb)[0, 0])
+            q, s16, z16, _ = o.hqq_quantize(wb, bits)
+            rec = (q[0].astype(np.float64) - f16(z16[0, 0])) * f16(s16[0, 0])
+            if cv == 0.0:
+                assert np.all(rec == 0.0), bits
+            else:
+                assert np.all(np.abs(rec - cv) <= abs(cv) * 2.0 ** -10), (bits, c)
+            assert np.all(q <= Q)
+
+
+def pin_hqq_power_of_two_scaling(o):
+    """p = 1: scaling the weights by 2^k and beta by 2^-k scales the stored scale by 2^k and
+    leaves zeros, codes and iteration counts unchanged (exact in binary arithmetic)."""
+    rng = np.random.default_rng(37)
+    wb = synth.to_bf16_bits(rng.standard_t(3, (4, 128)) * 0.02)
+    w = xf(wb)
+    for bits, beta in ((4, 300.0), (6, 3000.0), (8, 30.0)):
+        q0, s0, z0, r0 = o.hqq_quantize(wb, bits, p=1.0, beta=beta, kappa=1.03)
+        for k in (-3, 2, 5):
+            wk = synth.to_bf16_bits(w * 2.0 ** k)
+            q1, s1, z1, r1 = o.hqq_quantize(wk, bits, p=1.0, beta=beta * 2.0 ** -k, kappa=1.03)
+            assert np.array_equal(q1, q0) and np.array_equal(z1, z0) and np.array_equal(r1, r0)
+            assert np.array_equal(f16(s1), f16(s0) * 2.0 ** k), (bits, k)
+
+
+def pin_hqq_matrix_layout(o):
+    """The matrix call quantises group g of row r from columns 64g..64g+63 of that row."""
+    rng = np.random.default_rng(38)
+    wb = synth.to_bf16_bits(rng.normal(0, 0.04, (3, 320)))
+    q, s16, z16, ran = o.hqq_quantize(wb, 6, beta=1e4)
+    w = xf(wb)
+    for r in range(3):
+        for g in range(5):
+            sg, zg, qg, zt, _ = o.hqq_group(w[r, G * g:G * (g + 1)], 6, beta=1e4)
+            assert (sg, zg, len(zt)) == (s16[r, g], z16[r, g], ran[r, g])
+            assert np.array_equal(qg, q[r, G * g:G * (g + 1)])
+
+
+def pin_hqq_beats_minmax(o):
+    """Summed over many groups, the stored result has less L1 reconstruction error than plain
+    min-max rounding (the iteration starts there and only keeps improvements)."""
+    rng = np.random.default_rng(39)
+    for bits in (4, 6, 8):
+        wb = synth.to_bf16_bits(rng.standard_t(4, (16, 512)) * 0.02)
+        w = xf(wb)
+        errs = []
+        for iters in (0, 20):
+            q, s16, z16, _ = o.hqq_quantize(wb, bits, iters=iters)
+            rec = (q - np.repeat(f16(z16), G, 1)) * np.repeat(f16(s16), G, 1)
+            errs.append(np.abs(rec - w).sum())
+        assert errs[1] < errs[0], (bits, errs)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]
 
 

@@ -29,6 +29,23 @@ MUTANTS = {
     "f16_exponent_bias": ("ex - 25)", "ex - 24)"),
     "f16_subnormal_scale": ("ldexp((double)man, -24)", "ldexp((double)man, -14)"),
     "router_reads_transposed": ("(double)wr[(size_t)e * H + h]", "(double)wr[(size_t)h * E + e]"),
+    # quantiser
+    "f16_round_truncates": ("double n = rint(ldexp(a, -qe));", "double n = floor(ldexp(a, -qe));"),
+    "f16_subnormal_quantum": ("if (qe < -24) qe = -24;", "if (qe < -14) qe = -14;"),
+    "hqq_levels_not_minus_one": ("double qmax = (double)((1 << bits) - 1);\n    double lo",
+                                 "double qmax = (double)(1 << bits);\n    double lo"),
+    "hqq_zero_from_max": ("double z = -lo / s;", "double z = -hi / s;"),
+    "hqq_no_clamp": ("return fmin(fmax(q, 0.0), qmax);", "return q;"),
+    "hqq_err_signed": ("err += fabs(w[j] - r[j]);", "err += w[j] - r[j];"),
+    "hqq_shrink_exponent": ("pow(a, p - 1.0) / beta", "pow(a, p) / beta"),
+    "hqq_shrink_beta_inverted": ("pow(a, p - 1.0) / beta", "pow(a, p - 1.0) * beta"),
+    "hqq_zero_update_sign": ("acc += q[j] - (w[j] - e) / s;", "acc += q[j] + (w[j] - e) / s;"),
+    "hqq_shrink_ignored": ("acc += q[j] - (w[j] - e) / s;", "acc += q[j] - w[j] / s;"),
+    "hqq_beta_not_grown": ("beta *= kappa;", ""),
+    "hqq_keeps_last_zero": ("oracle_f64_to_f16(fmin(fmax(zbest,", "oracle_f64_to_f16(fmin(fmax(z,"),
+    "hqq_no_stop": ("if (!(err < best)) break;", "if (!(err < best)) continue;"),
+    "hqq_codes_unrounded_zero": ("hqq_code(w[j], s, zs, qmax)", "hqq_code(w[j], s, zbest, qmax)"),
+    "hqq_matrix_group_column": ("c0 = (g % gpr) * ORACLE_GROUP;", "c0 = (g / rows) * ORACLE_GROUP;"),
 }
 
 
