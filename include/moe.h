@@ -91,6 +91,47 @@ moe_status_t moe_pack_layer(const moe_expert_src_t *src, int E, int H, int I, vo
                             size_t packed_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Quantiser: bf16 weights -> the canonical format above.
+ *
+ * HQQ-style group quantisation (Half-Quadratic Quantization, H. Badri and A. Shaji, 2023; the
+ * page "Krasis update", list of the v1.0 results, names it at 4, 6 and 8 bits, built from the
+ * weights alone). For each 64-wide group of a row, Q = 2^bits - 1:
+ *   1. s = fp16((max - min) / Q), kept within [least positive fp16, 65504]; z = -min / s.
+ *      A constant group c is quantised over [min(c, 0), max(c, 0)], an all-zero group with
+ *      scale 1.
+ *   2. Up to `iters` half-quadratic steps on the zero point: with q = clamp(rint(w/s + z), 0, Q)
+ *      and r = (q - z) * s, stop if sum |w - r| did not fall below (1 - 2^-40) times the best
+ *      so far (which keeps its zero; the margin exceeds the sum's rounding, so ties on the flat
+ *      stretches of the L1 error stop as in exact arithmetic); otherwise e = shrink(w - r) with
+ *      shrink(x) = sign(x) * max(|x| - |x|^(lp_norm - 1) / beta, 0), z = mean(q - (w - e)/s),
+ *      beta = beta * kappa.
+ *   3. zero = fp16(best z), clamped to +-65504; codes = the nearest points of the stored fp16
+ *      grid, clamp(rint(w/scale + zero), 0, Q).
+ * Arithmetic is IEEE fp64, each operation correctly rounded and unfused, and the two sums over
+ * a group run in index order, so results are those of the definition evaluated in that order
+ * (the power function of the shrink, accurate to a few units in the last place, aside).
+ *   w (device, 16-byte aligned) bf16 [rows x cols], row-major, cols % 64 == 0, rows >= 0.
+ *   params (host) or NULL for the published defaults {0.7, 10.0, 1.01, 20}; required:
+ *     0 < lp_norm <= 1, beta > 0 and finite, kappa >= 1 and finite, 0 <= iters <= 1000
+ *     (iters = 0 is plain min-max rounding).
+ *   codes (device, 4-byte aligned): rows x (cols*bits/8) bytes in the canonical layout.
+ *   scale, zero (device, 2-byte aligned): fp16 [rows x cols/64].
+ *   iters_used (device, 4-byte aligned) int32 [rows x cols/64] or NULL: steps run per group,
+ *     counting the one that stopped.
+ * rows == 0 launches nothing. Asynchronous on `stream`.
+ * ------------------------------------------------------------------------------------- */
+typedef struct moe_hqq_params {
+    double lp_norm;
+    double beta;
+    double kappa;
+    int32_t iters;
+} moe_hqq_params_t;
+
+moe_status_t moe_quantize_hqq(const uint16_t *w, int rows, int cols, int bits,
+                              const moe_hqq_params_t *params, void *codes, uint16_t *scale,
+                              uint16_t *zero, int32_t *iters_used, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * Routing alone.
  *
  * x (device) bf16 [T x H]; w_router (device) fp32 [E x H]; bias (device) fp32 [E] or NULL.

@@ -219,8 +219,8 @@ void oracle_moe_forward(const uint16_t *x, const float *wr, const float *bias,
  *      z_0 = -lo / s (s is the stored fp16 value from here on).
  *   2. For i = 0 .. iters-1, with beta_0 = beta and beta_{i+1} = kappa * beta_i:
  *        q_j = clamp(rint(w_j / s + z_i), 0, Q),   r_j = (q_j - z_i) * s
- *        err_i = sum_j |w_j - r_j|; if err_i is not below the best so far, stop;
- *               otherwise z_i becomes the best zero
+ *        err_i = sum_j |w_j - r_j|; if err_i is not below (1 - 2^-40) times the best so far,
+ *               stop; otherwise z_i becomes the best zero
  *        e_j = shrink_p(w_j - r_j, beta_i)
  *        z_{i+1} = (1/64) * sum_j (q_j - (w_j - e_j) / s)
  *      with the generalised soft threshold
@@ -230,8 +230,15 @@ void oracle_moe_forward(const uint16_t *x, const float *wr, const float *bias,
  *      stored fp16 s and z. These are the nearest points of the stored grid.
  * The readings this takes where the published text leaves room: the stop rule and the best
  * zero are per group (the objective is a sum of independent group terms); the codes are
- * recomputed from the stored fp16 scale and zero; iters = 0 is plain min-max rounding.
+ * recomputed from the stored fp16 scale and zero; iters = 0 is plain min-max rounding; and
+ * the stop test is the one exact arithmetic takes. Near its optimum the L1 error is flat in
+ * the zero (the residual signs balance), so successive iterates often have equal error, and a
+ * strict comparison of two rounded 64-term sums would decide those ties by rounding. A fall
+ * counts only if it exceeds 2^-40 of the error; the rounding of such a sum, in any order, is
+ * below 2^-46 of it.
  */
+
+#define HQQ_FALL (1.0 - 0x1p-40)   /* an error must fall below HQQ_FALL * best to count */
 
 /* double -> IEEE binary16 bits, round to nearest, ties to even (from the format's definition:
  * 11 significant bits for normal values, a fixed quantum of 2^-24 below 2^-14, and infinity
@@ -306,7 +313,7 @@ void oracle_hqq_group(const double *w, int bits, double p, double beta, double k
         if (z_trace) z_trace[i] = z;
         if (err_trace) err_trace[i] = err;
         ran = i + 1;
-        if (!(err < best)) break;
+        if (!(err < best * HQQ_FALL)) break;
         best = err;
         zbest = z;
         double acc = 0.0;

@@ -36,7 +36,14 @@ SIGNATURES = {
     "moe_prefill_experts": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_set_wait_limit_ns": (None, [_u64]),
+    "moe_quantize_hqq": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
+
+
+class HqqParams(C.Structure):
+    """moe_hqq_params_t"""
+    _fields_ = [("lp_norm", C.c_double), ("beta", C.c_double), ("kappa", C.c_double),
+                ("iters", C.c_int32)]
 
 
 class ExpertSrc(C.Structure):
@@ -119,6 +126,28 @@ def pack_layer(experts: Sequence[dict], H: int, I: int, out: Optional[torch.Tens
     _check(lib().moe_pack_layer(C.cast(src, C.c_void_p), E, H, I, out.data_ptr(), out.numel(), _stream(stream)),
            "moe_pack_layer")
     return out
+
+
+HQQ_DEFAULTS = {"lp_norm": 0.7, "beta": 10.0, "kappa": 1.01, "iters": 20}
+
+
+def quantize_hqq(w: torch.Tensor, bits: int, lp_norm: float = 0.7, beta: float = 10.0,
+                 kappa: float = 1.01, iters: int = 20, with_iters: bool = False, stream=None):
+    """HQQ-style quantisation of bf16 weights [rows, cols] (CUDA, contiguous) into the canonical
+    format: returns (codes uint8 [rows, cols*bits//8], scale fp16 [rows, cols//64],
+    zero fp16 [rows, cols//64]) and, with ``with_iters``, the int32 steps run per group."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous 2-D bf16 tensor")
+    rows, cols = w.shape
+    dev = w.device
+    codes = torch.empty((rows, cols * bits // 8), dtype=torch.uint8, device=dev)
+    scale = torch.empty((rows, cols // 64), dtype=torch.float16, device=dev)
+    zero = torch.empty((rows, cols // 64), dtype=torch.float16, device=dev)
+    it = torch.empty((rows, cols // 64), dtype=torch.int32, device=dev) if with_iters else None
+    prm = HqqParams(float(lp_norm), float(beta), float(kappa), int(iters))
+    _check(lib().moe_quantize_hqq(_p(w), rows, cols, bits, C.addressof(prm), _p(codes), _p(scale), _p(zero),
+                                  _p(it), _stream(stream)), "moe_quantize_hqq")
+    return (codes, scale, zero, it) if with_iters else (codes, scale, zero)
 
 
 # ------------------------------------------------------------------------------ routing

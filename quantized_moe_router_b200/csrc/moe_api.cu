@@ -1,6 +1,7 @@
 // moe_api.cu -- the extern "C" entry points of include/moe.h: argument validation, workspace
 // sizing and dispatch to the kernels. Nothing here allocates device memory.
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -21,6 +22,9 @@ moe_status_t launch_prefill_route(const uint16_t *x, const float *wr, const floa
 moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T, int H, int I, int E, int k,
                                     uint16_t *out, void *ws, cudaStream_t st);
 moe_status_t launch_pack(const moe_expert_src_t *src, int E, int H, int I, void *packed, cudaStream_t st);
+moe_status_t launch_quantize_hqq(const uint16_t *w, int rows, int cols, int bits, double p, double beta,
+                                 double kappa, int iters, void *codes, uint16_t *scale, uint16_t *zero,
+                                 int32_t *iters_used, cudaStream_t st);
 size_t packed_layer_bytes(int E, int H, int I, const int32_t *bits);
 
 static std::atomic<uint64_t> g_wait_ns{2000000000ull};
@@ -136,6 +140,26 @@ moe_status_t moe_pack_layer(const moe_expert_src_t *src, int E, int H, int I, vo
     const moe_status_t d = check_device();
     if (d != MOE_OK) return d;
     return launch_pack(src, E, H, I, packed, (cudaStream_t)stream);
+}
+
+moe_status_t moe_quantize_hqq(const uint16_t *w, int rows, int cols, int bits, const moe_hqq_params_t *params,
+                              void *codes, uint16_t *scale, uint16_t *zero, int32_t *iters_used,
+                              moe_stream_t stream) {
+    if (rows < 0 || cols < kGroup || cols % kGroup || (bits != 4 && bits != 6 && bits != 8))
+        return MOE_ERR_INVALID_ARG;
+    const moe_hqq_params_t p = params ? *params : moe_hqq_params_t{0.7, 10.0, 1.01, 20};
+    if (!(p.lp_norm > 0.0 && p.lp_norm <= 1.0) || !(p.beta > 0.0 && p.beta < HUGE_VAL) ||
+        !(p.kappa >= 1.0 && p.kappa < HUGE_VAL) || p.iters < 0 || p.iters > 1000)
+        return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!w || !codes || !scale || !zero) return MOE_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(codes, 4) || !aligned(scale, 2) || !aligned(zero, 2) ||
+        (iters_used && !aligned(iters_used, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = check_device();
+    if (d != MOE_OK) return d;
+    return launch_quantize_hqq(w, rows, cols, bits, p.lp_norm, p.beta, p.kappa, p.iters, codes, scale, zero,
+                               iters_used, (cudaStream_t)stream);
 }
 
 moe_status_t moe_route_topk(const uint16_t *x, const float *w_router, const float *bias, int T, int H, int E, int k,

@@ -399,10 +399,14 @@ TRACE_CASES = ((4, 0.7, 10.0, 1.01, 1.0), (4, 0.7, 1e4, 1.01, 0.05), (6, 1.0, 1e
                (8, 0.5, 1e5, 1.2, 0.02), (4, 1.0, 30.0, 1.01, 2.0))
 
 
+HQQ_FALL = 1.0 - 2.0 ** -40
+
+
 def pin_hqq_trace(o):
     """Each iteration's error is the brute-force L1 distance of the group to its nearest grid
-    points at that iteration's zero; errors fall strictly until the iteration that stops; the
-    stored zero is the fp16 value of the zero with the least error."""
+    points at that iteration's zero; each step that continues has an error below 1 - 2^-40
+    times the one before; only the last step run may fail that (the stop); the stored zero is
+    the fp16 value of the zero with the least error."""
     rng = np.random.default_rng(34)
     for bits, p, beta, kappa, scale in TRACE_CASES:
         Q = (1 << bits) - 1
@@ -414,10 +418,11 @@ def pin_hqq_trace(o):
             for i in range(len(et)):
                 err = grid_distances(wg, s, zt[i], Q).min(1).sum()
                 assert abs(et[i] - err) <= 1e-12 * max(err, s), (bits, i)
-            assert np.all(np.diff(et[:-1]) < 0)
+            assert np.all(et[1:-1] < et[:-2] * HQQ_FALL)
             if len(et) < 20:
-                assert et[-1] >= et[-2]
-            best = int(np.argmin(et))
+                assert len(et) >= 2 and not et[-1] < et[-2] * HQQ_FALL
+            last_fell = len(et) == 1 or et[-1] < et[-2] * HQQ_FALL
+            best = len(et) - 1 if last_fell else len(et) - 2
             assert z16 == f16_of(zt[best]), (bits, best)
 
 

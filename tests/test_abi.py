@@ -106,3 +106,30 @@ def test_host_validation_before_any_launch(L):
     assert L.moe_prefill_experts(fake, fake, 4, 2000, 512, 256, 8, fake, fake, big, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_workspace_init(None, 1024, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_status(None, None) == qm.MOE_ERR_INVALID_ARG
+
+
+def test_quantizer_host_validation(L):
+    fake = 1 << 20
+    P = qm.HqqParams
+
+    def q(w=fake, rows=4, cols=128, bits=4, prm=None, codes=fake, s=fake, z=fake, it=None):
+        pp = None if prm is None else C.addressof(prm)
+        return L.moe_quantize_hqq(w, rows, cols, bits, pp, codes, s, z, it, None)
+
+    assert q(rows=0) == qm.MOE_OK                 # nothing to do: nothing launched
+    assert q(cols=100) == qm.MOE_ERR_INVALID_ARG
+    assert q(cols=0) == qm.MOE_ERR_INVALID_ARG
+    assert q(rows=-1) == qm.MOE_ERR_INVALID_ARG
+    assert q(bits=5) == qm.MOE_ERR_INVALID_ARG
+    assert q(w=None) == qm.MOE_ERR_INVALID_ARG
+    assert q(codes=None) == qm.MOE_ERR_INVALID_ARG
+    assert q(s=None) == qm.MOE_ERR_INVALID_ARG
+    assert q(w=fake + 8) == qm.MOE_ERR_INVALID_ARG       # w not 16-byte aligned
+    assert q(codes=fake + 2) == qm.MOE_ERR_INVALID_ARG
+    assert q(z=fake + 1) == qm.MOE_ERR_INVALID_ARG
+    assert q(it=fake + 2) == qm.MOE_ERR_INVALID_ARG
+    for bad in (P(0.0, 10.0, 1.01, 20), P(1.5, 10.0, 1.01, 20), P(0.7, 0.0, 1.01, 20),
+                P(0.7, float("inf"), 1.01, 20), P(0.7, 10.0, 0.9, 20), P(0.7, 10.0, float("nan"), 20),
+                P(0.7, 10.0, 1.01, -1), P(0.7, 10.0, 1.01, 1001)):
+        assert q(prm=bad) == qm.MOE_ERR_INVALID_ARG, (bad.lp_norm, bad.beta, bad.kappa, bad.iters)
+    assert q(rows=0, prm=P(0.7, 10.0, 1.01, 2000)) == qm.MOE_ERR_INVALID_ARG   # params checked first

@@ -43,7 +43,8 @@ MUTANTS = {
     "hqq_shrink_ignored": ("acc += q[j] - (w[j] - e) / s;", "acc += q[j] - w[j] / s;"),
     "hqq_beta_not_grown": ("beta *= kappa;", ""),
     "hqq_keeps_last_zero": ("oracle_f64_to_f16(fmin(fmax(zbest,", "oracle_f64_to_f16(fmin(fmax(z,"),
-    "hqq_no_stop": ("if (!(err < best)) break;", "if (!(err < best)) continue;"),
+    "hqq_no_stop": ("if (!(err < best * HQQ_FALL)) break;", "if (!(err < best * HQQ_FALL)) continue;"),
+    "hqq_strict_stop": ("if (!(err < best * HQQ_FALL)) break;", "if (!(err < best)) break;"),
     "hqq_codes_unrounded_zero": ("hqq_code(w[j], s, zs, qmax)", "hqq_code(w[j], s, zbest, qmax)"),
     "hqq_matrix_group_column": ("c0 = (g % gpr) * ORACLE_GROUP;", "c0 = (g / rows) * ORACLE_GROUP;"),
 }
