@@ -96,6 +96,48 @@ def _p(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _dev(t: Optional[torch.Tensor], name: str, dtype, shape=None, optional: bool = False) -> None:
+    """Checks that a tensor handed to the library is a contiguous CUDA tensor of the expected
+    dtype (and shape) on the current device. The C ABI takes raw device pointers, so a host
+    tensor, another GPU's tensor or a strided view must be refused here, before any launch."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} must have dtype {dtype}, not {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+
+
+_F16 = (torch.float16, torch.int16, torch.uint16) if hasattr(torch, "uint16") else (torch.float16, torch.int16)
+
+
+def _x_shape(x: torch.Tensor, name: str = "x"):
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D [T, H] tensor")
+    return x.shape
+
+
+def _check_block_args(x, w_router, bias, k, idx_out, w_out):
+    T, H = _x_shape(x)
+    _dev(x, "x", torch.bfloat16)
+    if not isinstance(w_router, torch.Tensor) or w_router.dim() != 2:
+        raise ValueError("w_router must be a 2-D [E, H] tensor")
+    E = w_router.shape[0]
+    _dev(w_router, "w_router", torch.float32, (E, H))
+    _dev(bias, "bias", torch.float32, (E,), optional=True)
+    _dev(idx_out, "idx_out", torch.int32, (T, k), optional=True)
+    _dev(w_out, "w_out", torch.float32, (T, k), optional=True)
+    return T, H, E
+
+
 # ------------------------------------------------------------------------------ weights
 
 def packed_layer_bytes(E: int, H: int, I: int, bits: Sequence[int]) -> int:
@@ -113,9 +155,17 @@ def pack_layer(experts: Sequence[dict], H: int, I: int, out: Optional[torch.Tens
     E = len(experts)
     bits = [int(ex["bits"]) for ex in experts]
     nbytes = packed_layer_bytes(E, H, I, bits)
+    for e, ex in enumerate(experts):
+        for m, (rows, cols) in enumerate(((I, H), (I, H), (H, I))):
+            _dev(ex["codes"][m], f"experts[{e}].codes[{m}]", torch.uint8, (rows, cols * bits[e] // 8))
+            _dev(ex["scale"][m], f"experts[{e}].scale[{m}]", _F16, (rows, cols // 64))
+            _dev(ex["zero"][m], f"experts[{e}].zero[{m}]", _F16, (rows, cols // 64))
     dev = experts[0]["codes"][0].device
     if out is None:
         out = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _dev(out, "out", torch.uint8)
+    if out.numel() < nbytes:
+        raise ValueError(f"out holds {out.numel()} bytes, the packed layer needs {nbytes}")
     src = (ExpertSrc * E)()
     for e, ex in enumerate(experts):
         for m in range(3):
@@ -136,9 +186,8 @@ def quantize_hqq(w: torch.Tensor, bits: int, lp_norm: float = 0.7, beta: float =
     """HQQ-style quantisation of bf16 weights [rows, cols] (CUDA, contiguous) into the canonical
     format: returns (codes uint8 [rows, cols*bits//8], scale fp16 [rows, cols//64],
     zero fp16 [rows, cols//64]) and, with ``with_iters``, the int32 steps run per group."""
-    if w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_contiguous():
-        raise ValueError("w must be a contiguous 2-D bf16 tensor")
-    rows, cols = w.shape
+    rows, cols = _x_shape(w, "w")
+    _dev(w, "w", torch.bfloat16)
     dev = w.device
     codes = torch.empty((rows, cols * bits // 8), dtype=torch.uint8, device=dev)
     scale = torch.empty((rows, cols // 64), dtype=torch.float16, device=dev)
@@ -154,8 +203,7 @@ def quantize_hqq(w: torch.Tensor, bits: int, lp_norm: float = 0.7, beta: float =
 
 def route_topk(x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Tensor], k: int,
                idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None, stream=None):
-    T, H = x.shape
-    E = w_router.shape[0]
+    T, H, E = _check_block_args(x, w_router, bias, k, idx_out, w_out)
     if idx_out is None:
         idx_out = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if w_out is None:
@@ -181,7 +229,12 @@ def workspace(T: int, H: int, I: int, E: int, k: int, mode: int, device="cuda", 
 
 
 def _forward(fn, what, x, w_router, bias, packed, I, E, k, ws, out, idx_out, w_out, stream):
-    T, H = x.shape
+    T, H, E_r = _check_block_args(x, w_router, bias, k, idx_out, w_out)
+    if E_r != E:
+        raise ValueError(f"w_router has {E_r} rows, E = {E}")
+    _dev(packed, "packed", torch.uint8)
+    _dev(ws, "ws", torch.uint8)
+    _dev(out, "out", torch.bfloat16, (T, H), optional=True)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(fn(_p(x), _p(w_router), _p(bias), _p(packed), T, H, I, E, k, _p(out), _p(idx_out), _p(w_out),
@@ -203,14 +256,21 @@ def forward_prefill(x, w_router, bias, packed, I, E, k, ws, out=None, idx_out=No
 
 def prefill_route(x, w_router, bias, I, E, k, ws, idx_out=None, w_out=None, stream=None):
     """Routing and bucketing of the prefill path into the workspace `ws`."""
-    T, H = x.shape
+    T, H, E_r = _check_block_args(x, w_router, bias, k, idx_out, w_out)
+    if E_r != E:
+        raise ValueError(f"w_router has {E_r} rows, E = {E}")
+    _dev(ws, "ws", torch.uint8)
     _check(lib().moe_prefill_route(_p(x), _p(w_router), _p(bias), T, H, I, E, k, _p(idx_out), _p(w_out), _p(ws),
                                    ws.numel(), _stream(stream)), "moe_prefill_route")
 
 
 def prefill_experts(x, packed, I, E, k, ws, out=None, stream=None):
     """Expert GEMMs and combine over the buckets of the last prefill_route on `ws`; returns out."""
-    T, H = x.shape
+    T, H = _x_shape(x)
+    _dev(x, "x", torch.bfloat16)
+    _dev(packed, "packed", torch.uint8)
+    _dev(ws, "ws", torch.uint8)
+    _dev(out, "out", torch.bfloat16, (T, H), optional=True)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_prefill_experts(_p(x), _p(packed), T, H, I, E, k, _p(out), _p(ws), ws.numel(), _stream(stream)),
@@ -220,7 +280,11 @@ def prefill_experts(x, packed, I, E, k, ws, out=None, stream=None):
 
 def forward_decode_noalloc(x, w_router, bias, packed, I, E, k, out=None, idx_out=None, w_out=None, stream=None):
     """Decode-path expert block using the library's fixed device scratch (no workspace)."""
-    T, H = x.shape
+    T, H, E_r = _check_block_args(x, w_router, bias, k, idx_out, w_out)
+    if E_r != E:
+        raise ValueError(f"w_router has {E_r} rows, E = {E}")
+    _dev(packed, "packed", torch.uint8)
+    _dev(out, "out", torch.bfloat16, (T, H), optional=True)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_expert_forward_decode_noalloc(_p(x), _p(w_router), _p(bias), _p(packed), T, H, I, E, k,
@@ -231,6 +295,7 @@ def forward_decode_noalloc(x, w_router, bias, packed, I, E, k, out=None, idx_out
 
 def device_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronises the stream and returns (and clears) the workspace's device status."""
+    _dev(ws, "ws", torch.uint8)
     return lib().moe_get_device_status(ws.data_ptr(), _stream(stream))
 
 

@@ -133,3 +133,51 @@ def test_quantizer_host_validation(L):
                 P(0.7, 10.0, 1.01, -1), P(0.7, 10.0, 1.01, 1001)):
         assert q(prm=bad) == qm.MOE_ERR_INVALID_ARG, (bad.lp_norm, bad.beta, bad.kappa, bad.iters)
     assert q(rows=0, prm=P(0.7, 10.0, 1.01, 2000)) == qm.MOE_ERR_INVALID_ARG   # params checked first
+
+
+def test_binding_refuses_tensors_the_library_cannot_take(L):
+    """The C ABI takes raw device pointers; the binding refuses host tensors, wrong dtypes,
+    wrong shapes and strided views before anything reaches the library (CPU only)."""
+    import torch
+    T, H, E, I, k = 2, 128, 4, 64, 2
+    x = torch.zeros((T, H), dtype=torch.bfloat16)
+    wr = torch.zeros((E, H), dtype=torch.float32)
+    packed = torch.zeros(1 << 16, dtype=torch.uint8)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.forward_decode(x, wr, None, packed, I, E, k, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.forward_prefill(x, wr, None, packed, I, E, k, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.route_topk(x, wr, None, k)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.prefill_route(x, wr, None, I, E, k, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.prefill_experts(x, packed, I, E, k, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.forward_decode_noalloc(x, wr, None, packed, I, E, k)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.quantize_hqq(torch.zeros((4, 128), dtype=torch.bfloat16), 4)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.device_status(ws)
+    ex = {"bits": 4, "codes": [torch.zeros((I, H // 2), dtype=torch.uint8)] * 2 + [torch.zeros((H, I // 2), dtype=torch.uint8)],
+          "scale": [torch.zeros((I, H // 64), dtype=torch.float16)] * 2 + [torch.zeros((H, I // 64), dtype=torch.float16)],
+          "zero": [torch.zeros((I, H // 64), dtype=torch.float16)] * 2 + [torch.zeros((H, I // 64), dtype=torch.float16)]}
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm.pack_layer([ex], H, I)
+    # dtype, shape and layout checks come from the same helper
+    with pytest.raises(ValueError, match="2-D"):
+        qm.quantize_hqq(torch.zeros(128, dtype=torch.bfloat16), 4)
+    with pytest.raises(ValueError, match="2-D"):
+        qm.forward_decode(torch.zeros(H, dtype=torch.bfloat16), wr, None, packed, I, E, k, ws)
+
+
+def test_tensor_check_helper():
+    import torch
+    qm._dev(None, "bias", torch.float32, optional=True)
+    with pytest.raises(ValueError, match="required"):
+        qm._dev(None, "x", torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm._dev(torch.zeros(3), "x", torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        qm._dev(object(), "x", torch.float32)
