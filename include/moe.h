@@ -91,6 +91,84 @@ moe_status_t moe_pack_layer(const moe_expert_src_t *src, int E, int H, int I, vo
                             size_t packed_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Expert cache: packed layers kept in host memory, the experts a call needs streamed into a
+ * fixed pool of device slots.
+ *
+ * The pages run models whose experts do not fit in GPU memory: "Krasis update" (overview)
+ * streams the model from system RAM to VRAM; "RTX 3060 12GB ... --moe-direct-io" loads the
+ * selected experts on demand into a fixed number of slots per layer (72), without dropping
+ * experts and with output bit-identical to the stock engine; the Qwen-tin news page (memory
+ * placement and performance) keeps the expert weights on SSD and caches part of them in RAM
+ * and VRAM, about 96% of a token's expert bytes being resident already. Here each layer's
+ * packed form (as written by moe_pack_layer) stays in host memory, ideally page-locked, and a
+ * device pool holds one header per layer and `slots` expert-sized slots shared by all layers
+ * (a per-layer limit is one cache per layer). The forward calls read the same packed bytes
+ * either way, so a call through the cache computes what the resident call computes; the
+ * forward kernels add partial sums in arrival order, so either may differ from a repeat of
+ * itself in the last bit of an output.
+ *   [header of layer 0] ... [header of layer L-1] [slot 0] ... [slot slots-1]
+ * A layer's header has the packed format's layout; its entries point into the slots, so the
+ * header's address is a packed layer that the forward calls accept unchanged, as long as every
+ * expert the call selects is resident. Entries of experts that are not resident still point
+ * inside the pool (they read another expert's bytes, never memory outside it).
+ *
+ * Use per layer call: route (moe_route_topk, or the caller's own prediction), read the selected
+ * experts on the host, moe_cache_request (which experts are missing and where they go: host work
+ * only), moe_cache_commit (the copies and the header rewrite, on `stream`), then the forward
+ * call with the returned header. The forward call's idx_out shows which experts it used; a
+ * selection outside the request (possible only at a near-tie between the two routings) is
+ * requested and the call repeated.
+ *
+ * Eviction: a missing expert takes a free slot, else the slot of the least recently requested
+ * expert that none of the last `keep_recent` requests (this one included) named. keep_recent = 2
+ * lets the copies of one layer run while the previous layer's call still reads its experts,
+ * provided the caller orders the copies after the previous request's commit. A cache object is
+ * not thread-safe. Calls that read the pool must be ordered with the commits that overwrite it
+ * (one stream, or events).
+ * ------------------------------------------------------------------------------------- */
+typedef struct moe_expert_cache moe_expert_cache_t;
+
+/* Device bytes of the pool for L host layers (host_layers[l]: host pointer to layer l's packed
+ * form; all layers with the same E, H, I) and `slots` slots; 0 if an argument is invalid. */
+size_t moe_cache_pool_bytes(int L, const void *const *host_layers, const size_t *host_bytes,
+                            int slots);
+
+/* Creates the cache: host_layers / host_bytes (host arrays [L]) give each layer's packed form in
+ * host memory and its size, checked against the headers; pool (device, 256-byte aligned) holds
+ * pool_bytes >= moe_cache_pool_bytes. 1 <= slots, 1 <= keep_recent <= 8. The host layers must
+ * stay valid and unchanged while the cache exists. Host work only: no device memory is touched
+ * until the first commit. */
+moe_status_t moe_cache_create(int L, const void *const *host_layers, const size_t *host_bytes,
+                              int slots, int keep_recent, void *pool, size_t pool_bytes,
+                              moe_expert_cache_t **cache);
+
+void moe_cache_destroy(moe_expert_cache_t *cache);
+
+/* Makes experts[0..n) of `layer` (host array; duplicates allowed) the current request: counts
+ * hits and misses, gives every missing expert a slot (evicting as described above) and writes
+ * the missing experts and their slots to load_experts / load_slots (host arrays of at least n
+ * entries; either may be NULL) and their number to *n_load. Host work only. Fails with
+ * MOE_ERR_UNSUPPORTED, changing nothing, if the slots that may be evicted are too few. A
+ * request replaces an earlier request that was not committed. */
+moe_status_t moe_cache_request(moe_expert_cache_t *cache, int layer, const int32_t *experts,
+                               int n, int32_t *load_experts, int32_t *load_slots, int *n_load);
+
+/* Enqueues on `stream` the host -> device copies of the current request's missing experts and
+ * the rewrite of its layer's header (a copy from pageable host memory, so the call returns once
+ * the stream has drained up to it), and returns in *packed the device address of that layer's
+ * packed header. If a copy cannot be enqueued the missing experts are marked absent again and
+ * MOE_ERR_CUDA is returned. */
+moe_status_t moe_cache_commit(moe_expert_cache_t *cache, moe_stream_t stream, const void **packed);
+
+/* Slot that holds (layer, expert), or -1 (also for invalid arguments). */
+int moe_cache_slot_of(const moe_expert_cache_t *cache, int layer, int expert);
+
+/* Counters since creation: experts requested that were resident (hits), that had to be loaded
+ * (misses), and resident experts that lost their slot (evictions). */
+moe_status_t moe_cache_stats(const moe_expert_cache_t *cache, uint64_t *hits, uint64_t *misses,
+                             uint64_t *evictions);
+
+/* ---------------------------------------------------------------------------------------
  * Quantiser: bf16 weights -> the canonical format above.
  *
  * HQQ-style group quantisation (Half-Quadratic Quantization, H. Badri and A. Shaji, 2023; the

@@ -37,6 +37,13 @@ SIGNATURES = {
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_set_wait_limit_ns": (None, [_u64]),
     "moe_quantize_hqq": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_cache_pool_bytes": (_sz, [_i, _vp, _vp, _i]),
+    "moe_cache_create": (_i, [_i, _vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "moe_cache_destroy": (None, [_vp]),
+    "moe_cache_request": (_i, [_vp, _i, _vp, _i, _vp, _vp, _vp]),
+    "moe_cache_commit": (_i, [_vp, _vp, _vp]),
+    "moe_cache_slot_of": (_i, [_vp, _i, _i]),
+    "moe_cache_stats": (_i, [_vp, _vp, _vp, _vp]),
 }
 
 
@@ -197,6 +204,74 @@ def quantize_hqq(w: torch.Tensor, bits: int, lp_norm: float = 0.7, beta: float =
     _check(lib().moe_quantize_hqq(_p(w), rows, cols, bits, C.addressof(prm), _p(codes), _p(scale), _p(zero),
                                   _p(it), _stream(stream)), "moe_quantize_hqq")
     return (codes, scale, zero, it) if with_iters else (codes, scale, zero)
+
+
+class ExpertCache:
+    """Expert cache of include/moe.h (moe_cache_*): the packed layers stay in host memory
+    (``host_layers``: 1-D uint8 CPU tensors as moe_pack_layer wrote them, ideally pinned) and a
+    device pool of ``slots`` expert slots holds the experts that calls need, behind one packed
+    header per layer. Marshalling only; the policy and the copies are the library's."""
+
+    def __init__(self, host_layers: Sequence[torch.Tensor], slots: int, keep_recent: int = 1,
+                 device="cuda"):
+        for l, t in enumerate(host_layers):
+            if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.uint8 or t.dim() != 1 \
+                    or not t.is_contiguous():
+                raise ValueError(f"host_layers[{l}] must be a contiguous 1-D uint8 CPU tensor")
+        self.host_layers = list(host_layers)   # kept alive: the library reads them at every commit
+        L = len(self.host_layers)
+        self._ptrs = (C.c_void_p * L)(*[t.data_ptr() for t in self.host_layers])
+        self._sizes = (C.c_size_t * L)(*[t.numel() for t in self.host_layers])
+        n = lib().moe_cache_pool_bytes(L, C.cast(self._ptrs, C.c_void_p), C.cast(self._sizes, C.c_void_p), slots)
+        if n == 0:
+            raise MoeError("moe_cache_pool_bytes", MOE_ERR_INVALID_ARG)
+        self.pool = torch.empty(n, dtype=torch.uint8, device=device)
+        h = C.c_void_p()
+        _check(lib().moe_cache_create(L, C.cast(self._ptrs, C.c_void_p), C.cast(self._sizes, C.c_void_p), slots,
+                                      keep_recent, self.pool.data_ptr(), n, C.byref(h)), "moe_cache_create")
+        self._h = h
+        self.slots = slots
+
+    def request(self, layer: int, experts: Sequence[int]):
+        """Host work only: returns (missing experts, their slots) of this request."""
+        ids = [int(e) for e in experts]
+        arr = (C.c_int32 * max(1, len(ids)))(*ids)
+        le = (C.c_int32 * max(1, len(ids)))()
+        ls = (C.c_int32 * max(1, len(ids)))()
+        nl = C.c_int()
+        _check(lib().moe_cache_request(self._h, layer, C.cast(arr, C.c_void_p), len(ids), C.cast(le, C.c_void_p),
+                                       C.cast(ls, C.c_void_p), C.byref(nl)), "moe_cache_request")
+        return list(le[:nl.value]), list(ls[:nl.value])
+
+    def commit(self, stream=None) -> torch.Tensor:
+        """Copies of the current request and its layer's header, on `stream`; returns the layer's
+        packed header as a uint8 view of the pool, for the forward calls."""
+        out = C.c_void_p()
+        _check(lib().moe_cache_commit(self._h, _stream(stream), C.byref(out)), "moe_cache_commit")
+        return self.pool[out.value - self.pool.data_ptr():]
+
+    def prepare(self, layer: int, experts: Sequence[int], stream=None) -> torch.Tensor:
+        self.request(layer, experts)
+        return self.commit(stream)
+
+    def slot_of(self, layer: int, expert: int) -> int:
+        return lib().moe_cache_slot_of(self._h, layer, expert)
+
+    def stats(self):
+        h, m, e = C.c_uint64(), C.c_uint64(), C.c_uint64()
+        _check(lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(e)), "moe_cache_stats")
+        return {"hits": h.value, "misses": m.value, "evictions": e.value}
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().moe_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
 
 
 # ------------------------------------------------------------------------------ routing

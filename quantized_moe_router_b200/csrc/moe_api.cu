@@ -27,6 +27,13 @@ moe_status_t launch_quantize_hqq(const uint16_t *w, int rows, int cols, int bits
                                  int32_t *iters_used, cudaStream_t st);
 size_t packed_layer_bytes(int E, int H, int I, const int32_t *bits);
 
+moe_status_t require_sm100() {
+    const DeviceInfo *d = device_info();
+    if (!d) return MOE_ERR_CUDA;
+    if (d->cc_major != 10 || d->cc_minor != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
 static std::atomic<uint64_t> g_wait_ns{2000000000ull};
 uint64_t wait_limit_ns() { return g_wait_ns.load(); }
 
@@ -57,12 +64,7 @@ namespace {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-moe_status_t check_device() {
-    const DeviceInfo *d = device_info();
-    if (!d) return MOE_ERR_CUDA;
-    if (d->cc_major != 10 || d->cc_minor != 0) return MOE_ERR_UNSUPPORTED;
-    return MOE_OK;
-}
+moe_status_t check_device() { return require_sm100(); }
 
 bool shape_ok(int T, int H, int I, int E, int k) {
     return T >= 1 && H >= 64 && H % kGroup == 0 && I >= 64 && I % kGroup == 0 && E >= 1 && E <= kMaxE &&

@@ -319,6 +319,8 @@ struct DeviceInfo {
     int max_smem_optin;
 };
 const DeviceInfo *device_info();
+// MOE_OK on an sm_100 device, MOE_ERR_UNSUPPORTED on another, MOE_ERR_CUDA without one
+moe_status_t require_sm100();
 uint64_t wait_limit_ns();
 
 }  // namespace moe

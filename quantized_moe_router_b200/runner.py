@@ -78,3 +78,34 @@ class PrefillStack:
         for l, lw in enumerate(self.layers):
             forward_prefill(self.x_in[l], lw.wr, lw.bias, lw.packed, self.I, self.E, self.k, self.ws,
                             out=self.out[l], stream=stream)
+
+
+def forward_through_cache(cache, layer: int, x: torch.Tensor, w_router: torch.Tensor,
+                          bias: Optional[torch.Tensor], I: int, E: int, k: int, ws: torch.Tensor,
+                          mode: int = MODE_DECODE, retries: int = 2):
+    """One layer call whose experts come through an ExpertCache, on the current stream.
+
+    Prefill: routing and bucketing first (prefill_route), then exactly the experts the buckets
+    name are made resident and the grouped GEMMs read them through the layer's cache header.
+    Decode: the fused kernel routes again inside; the experts of a separate routing call are made
+    resident, and the call's own idx_out is checked against them. An expert outside them (the two
+    routings can differ only where two logits tie to fp32 rounding) is loaded and the call
+    repeated. Returns (out, idx, w). Plumbing only: every step runs in the library."""
+    from . import prefill_experts, prefill_route, route_topk
+    T, H = x.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    wts = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    if mode == MODE_PREFILL:
+        prefill_route(x, w_router, bias, I, E, k, ws, idx_out=idx, w_out=wts)
+        packed = cache.prepare(layer, sorted(set(idx.cpu().flatten().tolist())))
+        return prefill_experts(x, packed, I, E, k, ws), idx, wts
+    route_topk(x, w_router, bias, k, idx_out=idx, w_out=wts)
+    want = set(idx.cpu().flatten().tolist())
+    for _ in range(retries + 1):
+        packed = cache.prepare(layer, sorted(want))
+        out = forward_decode(x, w_router, bias, packed, I, E, k, ws, idx_out=idx, w_out=wts)
+        used = set(idx.cpu().flatten().tolist())
+        if used <= want:
+            return out, idx, wts
+        want |= used
+    raise RuntimeError("the decode call kept selecting experts outside the cache request")
