@@ -27,9 +27,9 @@
 // moves to its next group when the current one stops; a warp runs in lockstep only within a
 // step. The group's 64 weights sit in shared memory, element-major across the block's threads
 // (conflict-free), loaded with eight 16-byte reads per thread.
-// The kernel is bound by the fp64 pipe and the power function of the shrink, not by memory:
-// 2 bytes read and b/8 + 1/16 bytes written per weight, against roughly 40 fp64 operations and
-// three divisions per weight and step.
+// The kernel is bound by the fp64 pipe, not by memory: 2 bytes read and b/8 + 1/16 bytes written
+// per weight, against roughly 40 fp64 operations and three divisions per weight and step, plus
+// the power function of the shrink for the weights outside its dead zone.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -49,9 +49,20 @@ __device__ __forceinline__ double grid_code(double w, double s, double z, double
     return fmin(fmax(q, 0.0), qmax);
 }
 
-__device__ __forceinline__ double shrink_lp(double x, double beta, double p) {
+// The shrink is 0 on its dead zone |x| <= beta^(-1/(2-p)). `dead` is that bound lowered by a
+// relative 2^-20: below it the exact |x| - |x|^(p-1)/beta is negative by more than 2^-20 of |x|,
+// a million times the error of the power function and the division, so the formula evaluated in
+// fp64 is negative too and the result is the same 0 -- without the power function, which is
+// most of the step's cost when the shrink is inactive (as for LLM-like weights at the published
+// defaults).
+__device__ __forceinline__ double dead_zone(double beta, double p) {
+    return p < 1.0 ? __dmul_rn(pow(beta, -1.0 / (2.0 - p)), 1.0 - 0x1p-20) : 0.0;
+}
+
+__device__ __forceinline__ double shrink_lp(double x, double beta, double p, double dead) {
     if (x == 0.0) return 0.0;
     const double a = fabs(x);
+    if (a < dead) return 0.0;
     const double pw = p == 1.0 ? 1.0 : pow(a, p - 1.0);   // pow(a, 0) is exactly 1
     const double t = __dsub_rn(a, __ddiv_rn(pw, beta));
     return t > 0.0 ? copysign(t, x) : 0.0;
@@ -140,11 +151,12 @@ __global__ void __launch_bounds__(kQuantThreads)
             } else {
                 best = err;
                 zbest = z;
+                const double dead = dead_zone(beta, a.p);
                 double acc = 0.0;
                 for (int j = 0; j < kGroup; ++j) {
                     const double v = wt(sw, j);
                     const double q = grid_code(v, s, z, qmax);
-                    const double e = shrink_lp(__dsub_rn(v, __dmul_rn(__dsub_rn(q, z), s)), beta, a.p);
+                    const double e = shrink_lp(__dsub_rn(v, __dmul_rn(__dsub_rn(q, z), s)), beta, a.p, dead);
                     acc = __dadd_rn(acc, __dsub_rn(q, __ddiv_rn(__dsub_rn(v, e), s)));
                 }
                 z = __ddiv_rn(acc, (double)kGroup);
