@@ -181,3 +181,23 @@ def test_tensor_check_helper():
         qm._dev(torch.zeros(3), "x", torch.float32)
     with pytest.raises(ValueError, match="CUDA tensor"):
         qm._dev(object(), "x", torch.float32)
+
+
+def test_header_is_plain_c_and_links(tmp_path, L):
+    """A C11 translation unit can include include/moe.h and take every entry point's address, and
+    links against the library (the ABI is C, not C++)."""
+    import subprocess
+    names = declared_functions()
+    src = tmp_path / "abi_check.c"
+    body = "\n".join(f"    p[{i}] = (void (*)(void)){n};" for i, n in enumerate(names))
+    src.write_text('#include "moe.h"\n#include <stdio.h>\n\nint main(void) {\n'
+                   f'    void (*p[{len(names)}])(void);\n{body}\n'
+                   f'    for (int i = 0; i < {len(names)}; ++i) if (!p[i]) return 1;\n'
+                   '    printf("%s\\n", moe_status_str(MOE_OK));\n    return 0;\n}\n')
+    libdir = os.path.dirname(qm.LIB_PATH)
+    exe = tmp_path / "abi_check"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lmoe_b200", "-Wl,-rpath," + libdir,
+                    "-Wl,-rpath,/usr/local/cuda/lib64", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and out.stdout.strip() == "MOE_OK", out
