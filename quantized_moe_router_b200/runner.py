@@ -63,6 +63,61 @@ class DecodeStack:
         self.graph.replay()
 
 
+class DecodeRun:
+    """S decode steps through L layers of the same shape, replayed as one CUDA graph of S * L
+    launches (step-major: every layer of step 0, then step 1, ...).
+
+    x is the caller's device tensor [S, L, T, H] bf16 that the graph reads in place (copy new
+    hidden states into it between replays); out [S, L, T, H], idx [S, L, T, k] and
+    wts [S, L, T, k] hold every call's results after a replay. One workspace serves all calls,
+    so the calls are ordered, as the layers of a model are.
+    """
+
+    def __init__(self, layers: Sequence[LayerWeights], x: torch.Tensor, I: int, E: int, k: int,
+                 with_routing_outputs: bool = True):
+        S, L, T, H = x.shape
+        if L != len(layers):
+            raise ValueError(f"x has {L} layers, {len(layers)} layer weights given")
+        self.layers = list(layers)
+        self.x = x
+        self.S, self.L, self.T, self.H, self.I, self.E, self.k = S, L, T, H, I, E, k
+        dev = x.device
+        self.ws = workspace(T, H, I, E, k, MODE_DECODE, dev)
+        self.out = torch.zeros((S, L, T, H), dtype=torch.bfloat16, device=dev)
+        self.idx = torch.zeros((S, L, T, k), dtype=torch.int32, device=dev) if with_routing_outputs else None
+        self.wts = torch.zeros((S, L, T, k), dtype=torch.float32, device=dev) if with_routing_outputs else None
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+
+    def launch(self, stream=None):
+        for s in range(self.S):
+            for l, lw in enumerate(self.layers):
+                forward_decode(self.x[s, l], lw.wr, lw.bias, lw.packed, self.I, self.E, self.k, self.ws,
+                               out=self.out[s, l], idx_out=None if self.idx is None else self.idx[s, l],
+                               w_out=None if self.wts is None else self.wts[s, l], stream=stream)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.launch()          # warm-up outside the graph (also sets kernel attributes)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.launch()
+        self.graph = g
+        return g
+
+    def replay(self):
+        if self.graph is None:
+            self.capture()
+        self.graph.replay()
+
+    @property
+    def launches(self) -> int:
+        return self.S * self.L
+
+
 class PrefillStack:
     """L prefill layers of the same shape sharing one workspace, launched back to back."""
 
@@ -74,10 +129,12 @@ class PrefillStack:
         self.x_in = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
         self.out = torch.zeros((L, T, H), dtype=torch.bfloat16, device=device)
 
-    def launch(self, stream=None):
+    def launch(self, stream=None, idx_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None):
+        """idx_out / w_out: optional [L, T, k] tensors that receive every layer's routing."""
         for l, lw in enumerate(self.layers):
             forward_prefill(self.x_in[l], lw.wr, lw.bias, lw.packed, self.I, self.E, self.k, self.ws,
-                            out=self.out[l], stream=stream)
+                            out=self.out[l], idx_out=None if idx_out is None else idx_out[l],
+                            w_out=None if w_out is None else w_out[l], stream=stream)
 
 
 def forward_through_cache(cache, layer: int, x: torch.Tensor, w_router: torch.Tensor,

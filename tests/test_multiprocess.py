@@ -31,7 +31,7 @@ def test_max_over_ranks_single_rank_is_identity():
 
 
 class Args:
-    gpus, steps, warmup = 2, 1, 0
+    gpus, steps, warmup, seq = 2, 1, 0, 0
 
 
 def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
