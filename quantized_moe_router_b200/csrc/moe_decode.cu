@@ -3,51 +3,50 @@
 //
 // This is the "MoE megakernel" of the page "Raon-1-mini ... RTX 5070 Ti" (table row: one
 // persistent kernel for each layer's expert block) with the "pipelined megakernel" row's
-// overlap (the next expert's tiles are in flight while the current one is multiplied), laid
-// out for sm_100a. One CTA per SM: 8 consumer warps and one control warp.
+// overlap (the next weights are in flight while the current ones are multiplied), laid out for
+// sm_100a. One CTA per SM: 16 consumer warps and one control warp.
 //   * Prologue, before the programmatic-dependent-launch wait (it overlaps the previous
 //     layer): mbarrier set-up, this CTA's router rows copied into shared memory, the packed
 //     layer's expert table read. Both are weights, never produced by the previous launch.
 //   * Routing. x is copied into shared memory; each CTA computes the fp32 logits of its
-//     E / nCTA experts (the dot products split over all warps) and publishes each as one 8-byte
-//     word {logit, call tag} into up to 32 copies of the T x E block, so that the CTAs' polls
-//     spread over the L2 slices. Every CTA polls its copy until all words carry this call's tag
-//     (derived from a completion counter that grows by nCTA per call: no barrier, no reset) and
-//     runs the same top-k + softmax: all CTAs agree on the selection without a second exchange.
-//   * Plan (control warp). Unique experts in ascending id, their pair lists (ascending token)
-//     and two job sequences: gate/up jobs (8 intermediate rows x all of H) and down jobs (16
-//     output rows x all of I). Each CTA takes a contiguous range of each, cut so that every CTA
-//     streams the same number of bytes as a few long contiguous regions.
-//   * Streaming. The control warp streams the CTA's regions with bulk copies of up to 48 KB
-//     (on B200 one SM completes roughly one bulk copy per 250 ns whatever its size, and every
-//     chunk costs the consumers one barrier, so chunks are large) into a ring of 2-3 stages,
-//     writing each chunk's job range into a descriptor next to it.
-//   * Gate/up: tile kg of a job goes to consumer warp kg % 8 (split K), which multiplies it with
+//     E / nCTA experts and publishes each as one 8-byte word {logit, call tag} into up to 32
+//     copies of the T x E block, so that the CTAs' polls spread over the L2 slices. Every CTA
+//     polls its copy until all words carry this call's tag (derived from a completion counter
+//     that grows by nCTA per call: no barrier, no reset) and runs the same top-k + softmax, so
+//     all CTAs agree on the selection without a second exchange.
+//   * Work units. A unit is (selected expert, 16 consecutive intermediate rows): the unit's
+//     gate/up rows (two 8-row blocks over all of H), SiLU-GLU of those 16 rows, and the matching
+//     16 columns of the down matrix over all H output rows. Everything a unit needs is on the
+//     CTA that runs it, so no intermediate leaves the SM; the units (expert-major) are cut into
+//     one contiguous range per CTA with equal bytes.
+//   * Streaming. The control warp issues the bulk copies of its range's weights (a unit is three
+//     contiguous pieces: gate/up tiles, the down quarter, the down scale/zero entries) into a ring
+//     of 32 KB stages as soon as the selection is known; consumers free stages as they go.
+//   * Gate/up: tile kg of the unit goes to consumer warp kg % 16 (split K), multiplied with
 //     mma.sync on bf16 operands made from the codes by one LOP3 per register (exact integers
-//     128 + q) and applies the group's scale and zero in fp32; after its last tile of a job a
-//     warp adds its partial into the job's shared-memory slot. One consumer barrier per chunk
-//     marks the previous chunk's jobs complete; each is finalised (SiLU-GLU, h as a bf16 hi/lo
-//     pair) by one warp while the others run on. The CTA publishes its h rows once (counter adds
-//     per expert after a fence); a down job waits only for the counter of its own expert.
-//   * Down: a whole job in one warp (its few tiles in a row), w * y added into the fp32 output
-//     accumulator.
-//   * The last CTA to finish (completion counter) converts the accumulator to bf16 and clears
-//     the accumulator and the counters for the next call.
+//     128 + q), the group's scale and zero applied in fp32; the warps' partial sums meet in shared
+//     memory, and one warp per 8 tokens forms h = silu(g) * u as a bf16 hi + lo pair.
+//   * Down: super-tile st (64 output rows) of the unit's quarter goes to warp st % 16; w * y is
+//     accumulated in registers across the CTA's units (one token: all of them; several tokens: the
+//     units of one expert) and added into the fp32 output accumulator once.
+//   * Completion: one counter per 256 output rows; the CTA that completes a row group converts it
+//     to bf16 and clears it for the next call.
 // Every wait is bounded; on expiry the kernel records MOE_ERR_TIMEOUT in the workspace, the
 // warps skip the remaining work in lock step, and the call still leaves the workspace clean.
-// The kernel is instantiated for 1, 2 and 4 MMA n-tiles (up to 8, 16 and 32 tokens per expert).
+#include <atomic>
+
 #include "moe_internal.cuh"
 #include "moe_topk.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kCW = 8;                      // consumer warps
-constexpr int kWarps = kCW + 1;             // + the control warp (routing plan, bulk copies)
-constexpr int kThreads = kWarps * 32;
-constexpr int kStageBytes = 49152;          // bytes per bulk copy / ring stage
+constexpr int kMaxCW = 16;                  // consumer warps at most (+ one control warp)
+constexpr int kMaxWarps = kMaxCW + 1;
+constexpr int kSlice = 16;                  // intermediate rows per work unit
+constexpr int kStageBytes = 32768;          // bytes per ring stage
 constexpr int kMaxStages = 8;
-constexpr int kActBytes = 65536;            // x (routing + gate/up), then h of one expert (down)
+constexpr int kActBytes = 65536;            // x of all tokens in shared memory (more: read through L2)
 constexpr int kMaxP = kDecodeMaxP;
 constexpr int kSmemBudget = 232448;         // 227 KB opt-in shared memory per CTA
 constexpr int kBiasRows = 32;               // router bias values kept in shared memory
@@ -63,27 +62,12 @@ struct DecodeArgs {
     float *w_out;
     Control *ctl;
     unsigned long long *logits;
-    uint16_t *h_hi, *h_lo;
+    unsigned long long *rowcnt;
     float *out_acc;
-    uint32_t *h_ready;
     uint64_t wait_ns;
-    double rnC;                  // 1 / number of CTAs
-    uint32_t cm, cs1, cs2;       // division by the number of CTAs: multiplier and shifts
     uint32_t kmul;               // ceil(2^16 / k): p / k = (p * kmul) >> 16 for p < 2048
     int lrep;                    // copies of the logit words (a power of two)
     int lstride;                 // words between copies
-};
-
-// One ring stage's chunk, written by the producer before it starts the copy: jobs job0 ..
-// job0 + njobs - 1 of one phase and one expert slot u; the first job from its tile k0, the last
-// up to tile k1 (tpj tiles per job); job0's tile 0 lies base_off bytes from the stage start
-// (negative when the chunk begins inside that job). flags: 1 gate/up phase, 2 the CTA's last chunk.
-struct __align__(16) ChunkDesc {
-    int job0, base_off;
-    short njobs, k0, k1, tpj;
-    unsigned short tb;
-    unsigned char bits, flags;
-    short u, pad;
 };
 
 struct __align__(16) DecodeSmem {
@@ -91,9 +75,9 @@ struct __align__(16) DecodeSmem {
     uint64_t empty[kMaxStages];
     uint64_t xbar, wbar;
     unsigned long long epoch;
+    unsigned long long ccost[kMaxP + 1];   // bytes of the units of expert slots < j
     volatile int abort;
-    int U, g0, g1, d0, d1, nGU;
-    int is_last;
+    int U, u0, u1;
     uint32_t eoff[kMaxE];               // packed offset / 256 of every expert
     uint8_t ebits[kMaxE];               // code width of every expert
     uint32_t selmask[kMaxE / 32];
@@ -103,42 +87,35 @@ struct __align__(16) DecodeSmem {
     int cnt[kMaxP];
     int pfirst[kMaxP + 1];
     int cursor[kMaxP];
-    uint32_t cgu[kMaxP + 1];            // 64-byte units of all gate/up jobs of expert slots < u
-    uint32_t cd[kMaxP + 1];             // 64-byte units of all down jobs of expert slots < u
     int ptok[kMaxP];
-    int ppair[kMaxP];
     float pw[kMaxP];
     int sel_idx[kMaxP];
     float sel_w[kMaxP];
-    float lpart[kWarps];                // slice sums of the router dot products
-    ChunkDesc desc[kMaxStages];         // the chunk of each ring stage
+    float lpart[kMaxWarps];             // slice sums of the router dot products
     float bias[kBiasRows];              // router bias of the CTA's rows c, c + nCTA, ...
-    __align__(16) uint32_t plist[32];   // plan scratch: packed pair list
 };
 
-// accumulator slots of NT n-tiles: 16 rows x 8*NT columns fp32, laid out as the MMA fragments
-template <int NT> constexpr int slots_for() { return NT == 4 ? 8 : 16; }
-// A gate/up job's partial sums stay in its slot from the chunk that completes it until the next
-// chunk's barrier; meanwhile that chunk adds into the slots of the jobs it touches. A chunk touching at
-// most (slots - 1) / 2 jobs keeps the two sets apart, so a chunk holds at most that minus one
-// jobs' worth of tiles.
-template <int NT> constexpr int chunk_jobs() { return (slots_for<NT>() - 1) / 2 - 1; }
-template <int NT> constexpr int slot_floats() { return NT * 128; }
-
+// Shared-memory regions after DecodeSmem. NT: MMA n-tiles (8 tokens each) of a unit.
 struct DecodeLayout {
-    size_t ring, act, accs, xs, total;
+    size_t xs, xsum, gred, hbuf, hcol, ycta, ring, total;
     int stages;
 };
 template <int NT>
 DecodeLayout decode_layout(int T, int H, int smem_limit) {
     DecodeLayout L;
     size_t o = align_up(sizeof(DecodeSmem), 128);
-    L.act = o;
-    o += kActBytes;
-    L.accs = o;
-    o += (size_t)slots_for<NT>() * slot_floats<NT>() * 4;
     L.xs = o;
+    if ((size_t)T * H * 2 <= (size_t)kActBytes) o += align_up((size_t)T * H * 2, 128);
+    L.xsum = o;                                   // x group sums [T x H/64] fp32
     o += align_up((size_t)T * (H / kGroup) * 4, 128);
+    L.gred = o;                                   // gate/up partial sums [2][NT][4][32] fp32
+    o += (size_t)2 * NT * 4 * 32 * 4;
+    L.hbuf = o;                                   // h hi / lo [2][NT][8 pairs][16] bf16
+    o += (size_t)2 * NT * 8 * 16 * 2;
+    L.hcol = o;                                   // per pair column: X = sum h [NT x 8], weight [NT x 8]
+    o += (size_t)2 * NT * 8 * 4;
+    L.ycta = o;                                   // one token: the CTA's output rows [H] fp32
+    if (T == 1) o += align_up((size_t)H * 4, 128);
     L.ring = align_up(o, 128);
     const long long room = (long long)min(smem_limit, kSmemBudget) - (long long)L.ring;
     L.stages = room > 0 ? (int)(room / kStageBytes) : 0;
@@ -147,23 +124,27 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
     return L;
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory"); }
+template <int CW>
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(CW * 32) : "memory"); }
 // The same barrier, returning the OR of `flag` over the consumer threads: a decision that all
 // consumer warps take identically (S.abort can change at any time, so reading it after a plain
 // barrier could split the warps).
+template <int CW>
 __device__ __forceinline__ bool consumer_sync_or(bool flag) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)flag), "n"(kCW * 32)
+        : "r"((uint32_t)flag), "n"(CW * 32)
         : "memory");
     return r != 0;
 }
 // named barrier 2: the control warp arrives when the plan is in shared memory, the consumer
-// warps wait for it (and for each other's group sums)
-__device__ __forceinline__ void plan_ready_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory"); }
-__device__ __forceinline__ void plan_ready_wait() { asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory"); }
+// warps wait for it
+template <int CW>
+__device__ __forceinline__ void plan_ready_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"((CW + 1) * 32) : "memory"); }
+template <int CW>
+__device__ __forceinline__ void plan_ready_wait() { asm volatile("bar.sync 2, %0;" ::"n"((CW + 1) * 32) : "memory"); }
 __device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long *p, unsigned long long v) {
     unsigned long long old;
     asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
@@ -171,6 +152,11 @@ __device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long
 }
 __device__ __forceinline__ void red_shared_f32(float *p, float v) {
     asm volatile("red.relaxed.cta.shared::cta.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_v4_f32(float *p, float4 v) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
 }
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
     unsigned long long v;
@@ -180,102 +166,32 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
-// bounded spin on a global word reaching `target` (one thread); false on expiry
-__device__ __forceinline__ bool wait_counter(const uint32_t *p, uint32_t target, uint64_t limit_ns,
-                                             uint32_t *status) {
-    if (ld_acquire_u32(p) >= target) return true;
-    const uint64_t t0 = global_timer();
-    while (true) {
-        __nanosleep(64);
-        if (ld_acquire_u32(p) >= target) return true;
-        if (global_timer() - t0 > limit_ns) {
-            atomicOr(status, kStatusTimeout);
-            return false;
-        }
-    }
-}
-
-// ------------------------------------------------------------------------------ job layout
-// A run of consecutive jobs of one expert and one phase: contiguous in the packed layer.
-struct Region {
-    const uint8_t *src;
-    int tiles, tb, bits, u, rb0, jg0, tpj;   // jg0: global index of the first job
-};
-
-__device__ __forceinline__ Region region_at(const DecodeSmem &S, const DecodeArgs &a, bool gu, int j) {
-    Region r;
-    const int G = a.H / kGroup, GI = a.I / kGroup;
-    const int per = gu ? a.I / 8 : a.H / 16;    // jobs per expert
-    const int end = gu ? S.g1 : S.d1;
-    r.u = j / per;
-    r.rb0 = j % per;
-    r.jg0 = j;
-    const int jend = min(end, (r.u + 1) * per);
-    r.tpj = gu ? G : GI;
-    r.tiles = (jend - j) * r.tpj;
-    r.bits = S.ubits[r.u];
-    r.tb = tile_bytes(r.bits);
-    const uint8_t *base = a.packed + (size_t)S.uoff[r.u] * 256;
-    r.src = gu ? base + (size_t)r.rb0 * G * r.tb : base + gu_tiles(a.H, a.I) * r.tb + (size_t)r.rb0 * GI * r.tb;
-    return r;
-}
-// Chunks of a region: at most one stage and at most maxjobs jobs' worth of tiles (gate/up
-// chunks, whose jobs keep partial sums in slots).
-__device__ __forceinline__ int region_chunks(const Region &r, int maxjobs) {
-    const int cap = min(kStageBytes / r.tb, maxjobs * r.tpj);
-    return (r.tiles + cap - 1) / cap;
-}
-// tiles [c0, c0 + m) of chunk i of a region (balanced split)
-__device__ __forceinline__ void chunk_range(const Region &r, int n, int i, int &c0, int &m) {
-    const int base = r.tiles / n, rem = r.tiles % n;
-    m = base + (i < rem ? 1 : 0);
-    c0 = i * base + (i < rem ? i : rem);
-}
-
-// First job (of the gate/up or down sequence) whose first 64-byte unit is at or after `pos`;
-// cum[u] = units of the jobs of expert slots < u, `per` jobs per expert.
-__device__ __forceinline__ int job_at_unit(const uint32_t *cum, int U, int per, uint32_t pos) {
-    if (pos == 0) return 0;
-    if (pos >= cum[U]) return U * per;
-    int lo = 0, hi = U;                 // largest u with cum[u] <= pos
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (cum[mid] <= pos) lo = mid; else hi = mid;
-    }
-    const uint32_t jb = (cum[lo + 1] - cum[lo]) / per;   // units per job of expert lo
-    return lo * per + (int)((pos - cum[lo] + jb - 1) / jb);
-}
-__device__ __forceinline__ uint32_t job_start_unit(const uint32_t *cum, int U, int per, int j) {
-    if (j >= U * per) return cum[U];
-    const int u = j / per;
-    return cum[u] + (cum[u + 1] - cum[u]) / per * (uint32_t)(j % per);
-}
-
-// ------------------------------------------------------------------------------ tile math
-// Operand sources of the current job for this lane: per n-tile, the row that the lane's B
-// column reads (x row for gate/up, h hi row for down; null where the column has no token),
-// the h lo row (down), and the group-sum rows of its two accumulator columns.
-template <int NT>
-struct JobCtx {
-    const uint16_t *b[NT];   // global rows (bg) or null
-    const uint16_t *b2[NT];
-    uint32_t sb[NT], sb2[NT];    // shared-memory rows (!bg)
-    uint32_t xs0[NT], xs1[NT];   // shared-memory group-sum rows
-    bool has[NT], has0[NT], has1[NT];
-    bool bg;   // B rows are in global memory (read through L2) rather than shared memory
-};
-
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float lds32f(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
     return v;
 }
 // predicated shared-memory store (no branch)
@@ -283,85 +199,6 @@ __device__ __forceinline__ void sts_if(bool p, int *addr, int v) {
     asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q st.shared.u32 [%1], %2;\n\t}" ::"r"((int)p),
                  "r"(smem_u32(addr)), "r"(v)
                  : "memory");
-}
-__device__ __forceinline__ float lds32f(uint32_t a) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-    return v;
-}
-
-template <int BITS, int NT, bool GU>
-__device__ __forceinline__ void consume_tile(const uint8_t *tile, int kg, const JobCtx<NT> &jc, int lane,
-                                             float (&acc)[NT][4]) {
-    const int g = lane >> 2, t = lane & 3;
-    const uint4 lo = *reinterpret_cast<const uint4 *>(tile + 16 * lane);
-    uint4 hi8 = make_uint4(0, 0, 0, 0);
-    uint2 hi6 = make_uint2(0, 0);
-    if (BITS == 8) hi8 = *reinterpret_cast<const uint4 *>(tile + kLoBytes + 16 * lane);
-    if (BITS == 6) hi6 = *reinterpret_cast<const uint2 *>(tile + kLoBytes + 8 * lane);
-    const uint2 sz = *reinterpret_cast<const uint2 *>(tile + kLoBytes + hi_bytes(BITS) + 8 * g);
-    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        // Up to two n-tiles every lane loads: a column without a token reads a valid row (the
-        // first pair's) and produces accumulator columns that nothing reads, with no divergent
-        // branch per tile. Four n-tiles keep the guard (their registers are tight).
-        uint32_t b[8] = {0, 0, 0, 0, 0, 0, 0, 0}, b2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (NT <= 2 || jc.has[nt]) {
-            uint4 v0, v1, w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-            if (jc.bg) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(jc.b[nt] + kg * kGroup + 16 * t);
-                v0 = __ldcg(p);
-                v1 = __ldcg(p + 1);
-                if (!GU) {
-                    const uint4 *p2 = reinterpret_cast<const uint4 *>(jc.b2[nt] + kg * kGroup + 16 * t);
-                    w0 = __ldcg(p2);
-                    w1 = __ldcg(p2 + 1);
-                }
-            } else {
-                const uint32_t o = (uint32_t)(kg * kGroup + 16 * t) * 2;
-                v0 = lds128(jc.sb[nt] + o);
-                v1 = lds128(jc.sb[nt] + o + 16);
-                if (!GU) {
-                    w0 = lds128(jc.sb2[nt] + o);
-                    w1 = lds128(jc.sb2[nt] + o + 16);
-                }
-            }
-            b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
-            b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
-            b2[0] = w0.x; b2[1] = w0.y; b2[2] = w0.z; b2[3] = w0.w;
-            b2[4] = w1.x; b2[5] = w1.y; b2[6] = w1.z; b2[7] = w1.w;
-        }
-        const float X0 = (NT <= 2 || jc.has0[nt]) ? lds32f(jc.xs0[nt] + kg * 4) : 0.f;
-        const float X1 = (NT <= 2 || jc.has1[nt]) ? lds32f(jc.xs1[nt] + kg * 4) : 0.f;
-        tile_group_mma<BITS>(lo, hi8, hi6, b, GU ? nullptr : b2, sA, zA, sB, zB, X0, X1, acc[nt]);
-    }
-}
-
-// All tiles [k0, k1) of a job owned by one warp, two at a time.
-template <int BITS, int NT>
-__device__ __forceinline__ void run_tiles_seq(const uint8_t *job_base, int tb, int k0, int k1, const JobCtx<NT> &jc,
-                                              int lane, float (&acc)[NT][4], float (&acc2)[NT][4]) {
-    int kg = k0;
-    for (; kg + 1 < k1; kg += 2) {
-        consume_tile<BITS, NT, false>(job_base + (size_t)kg * tb, kg, jc, lane, acc);
-        consume_tile<BITS, NT, false>(job_base + (size_t)(kg + 1) * tb, kg + 1, jc, lane, acc2);
-    }
-    if (kg < k1) consume_tile<BITS, NT, false>(job_base + (size_t)kg * tb, kg, jc, lane, acc);   // odd tail
-}
-
-// The warp's tiles of job `jb` (region-local) inside a chunk: k-tiles kg in [k0, k1) with
-// kg % kCW == warp, two at a time so that their MMA chains interleave.
-template <int BITS, int NT, bool GU>
-__device__ __forceinline__ void run_tiles(const uint8_t *job_base, int tb, int k0, int k1, int warp,
-                                          const JobCtx<NT> &jc, int lane, float (&acc)[NT][4],
-                                          float (&acc2)[NT][4]) {
-    int kg = k0 + ((warp - k0) % kCW + kCW) % kCW;   // first tile >= k0 with kg % kCW == warp
-    for (; kg + kCW < k1; kg += 2 * kCW) {
-        consume_tile<BITS, NT, GU>(job_base + (size_t)kg * tb, kg, jc, lane, acc);
-        consume_tile<BITS, NT, GU>(job_base + (size_t)(kg + kCW) * tb, kg + kCW, jc, lane, acc2);
-    }
-    if (kg < k1) consume_tile<BITS, NT, GU>(job_base + (size_t)kg * tb, kg, jc, lane, acc);   // odd tail
 }
 
 // ------------------------------------------------------------------------------ routing
@@ -535,68 +372,34 @@ __device__ bool token_topk(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t t
     return true;
 }
 
-// floor(X * cc / nC) without an integer division. Below 2^32 the product is divided by the
-// invariant-divisor method of Granlund and Montgomery (a multiply-high, an add and two shifts
-// with constants set up on the host, exact for every 32-bit dividend); above, the quotient is
-// taken through the double reciprocal of nC (X * cc < 2^53 is exact in double and the estimate
-// is floor or floor - 1) and corrected once.
-__device__ __forceinline__ uint32_t cut_units(const DecodeArgs &a, uint32_t X, int cc, int nC) {
-    const unsigned long long n = (unsigned long long)X * (unsigned)cc;
-    if (n < (1ull << 32)) {
-        const uint32_t n32 = (uint32_t)n, t = __umulhi(a.cm, n32);
-        return (t + ((n32 - t) >> a.cs1)) >> a.cs2;
-    }
-    unsigned long long q = (unsigned long long)((double)n * a.rnC);
-    q += ((q + 1ull) * (unsigned)nC <= n) ? 1ull : 0ull;
-    return (uint32_t)q;
-}
-// Smallest r with r * d >= n, for results below 2^16: the truncated float quotient (relative
-// error below 2^-20, so within 0.07 of n / d) is floor(n / d) - 1, floor(n / d) or ceil(n / d),
-// and two conditional increments reach ceil(n / d).
-__device__ __forceinline__ uint32_t ceil_div_small(uint32_t n, uint32_t d) {
-    uint32_t r = (uint32_t)__fdividef((float)n, (float)d);
-    r += ((unsigned long long)r * d < n) ? 1u : 0u;
-    r += ((unsigned long long)r * d < n) ? 1u : 0u;
-    return r;
-}
-// First job (of a gate/up or down sequence) whose first unit is at or after q, found by the
-// lanes of a warp of which some hold one expert slot each (U <= 32 slots, in any lane order):
-// such a lane holds the slot's index, its first unit lo, its end hi and its units per job jb;
-// `per` jobs per slot, `total` units in all. The slot holding q is the one with lo < q <= hi
-// (slot 0 for q = 0). `start` receives the job's first unit (total past the last job).
-__device__ __forceinline__ int job_at_unit_warp(uint32_t lo, uint32_t hi, uint32_t jb, int slot, bool slot_lane,
-                                                int per, int U, uint32_t q, uint32_t total, uint32_t &start) {
-    const bool holds = slot_lane && (q == 0 ? lo == 0 : (lo < q && q <= hi));
-    const uint32_t m = __ballot_sync(0xffffffffu, holds);
-    const uint32_t r = holds ? ceil_div_small(q - lo, jb) : 0u;
-    const uint32_t st = lo + r * jb;
-    const int j = slot * per + (int)r;
-    if (m == 0) {
-        start = total;
-        return U * per;
-    }
-    const int u = __ffs(m) - 1;
-    start = __shfl_sync(0xffffffffu, st, u);
-    return __shfl_sync(0xffffffffu, j, u);
-}
 
+// ------------------------------------------------------------------------------ plan
 __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
     const int w = e >> 5;
     return S.wordpre[w] + __popc(S.selmask[w] & ((1u << (e & 31)) - 1u));
 }
 
-// Plan for more than 32 pairs (several tokens), out of line: bitmap of the selection in shared
-// memory, per-slot counts and a stable fill of the pair lists 32 slots at a time, and the job
-// ranges by binary search over the slots' unit prefixes.
-__device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
-    const int E = a.E, H = a.H, I = a.I;
-    const int G = H / kGroup;
-    const int pg = I / 8, pd = H / 16;
-    const uint32_t ug = (uint32_t)pg * (uint32_t)G;
-    int U;
-    uint32_t GUB;
-    // Many pairs: bitmap of the selection in shared memory, per-slot counts and a stable
-    // fill of the pair lists, 32 slots per pass.
+// Expert slots of one token (P = k <= 32 pairs, distinct experts): slot j is selection j.
+__device__ __forceinline__ void plan_single(DecodeSmem &S, int P, int lane) {
+    if (lane < P) {
+        const int e = S.sel_idx[lane];
+        S.ubits[lane] = S.ebits[e];
+        S.uoff[lane] = S.eoff[e];
+        S.pfirst[lane] = lane;
+        S.ptok[lane] = 0;
+        S.pw[lane] = S.sel_w[lane];
+    }
+    if (lane == 0) {
+        S.U = P;
+        S.pfirst[P] = P;
+    }
+    __syncwarp();
+}
+
+// Expert slots of several tokens, by one warp: the distinct selected experts in ascending id,
+// each with its pairs in ascending pair id (token-major, so ascending token).
+__device__ __noinline__ void plan_many(const DecodeArgs &a, DecodeSmem &S, int P, int lane) {
+    const int E = a.E;
     for (int i = lane; i < kMaxE / 32; i += 32) S.selmask[i] = 0;
     __syncwarp();
     for (int p = lane; p < P; p += 32) atomicOr(&S.selmask[S.sel_idx[p] >> 5], 1u << (S.sel_idx[p] & 31));
@@ -614,7 +417,7 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
         if (lane == 31) S.U = incl;
     }
     __syncwarp();
-    U = S.U;
+    const int U = S.U;
     for (int u = lane; u < U; u += 32) S.cnt[u] = 0;
     __syncwarp();
     for (int p = lane; p < P; p += 32) {
@@ -626,37 +429,22 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
     }
     __syncwarp();
     int carry = 0;
-    uint32_t cts = 0;
     for (int base = 0; base < U; base += 32) {
         const int u = base + lane;
         const int n = (u < U) ? S.cnt[u] : 0;
-        const uint32_t tu = (u < U) ? (uint32_t)tile_bytes(S.ubits[u]) / 64u : 0u;
         int incl = n;
-        uint32_t it = tu;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            const uint32_t ot = __shfl_up_sync(0xffffffffu, it, off);
-            if (lane >= off) {
-                incl += o;
-                it += ot;
-            }
+            if (lane >= off) incl += o;
         }
         if (u < U) {
             S.pfirst[u] = carry + incl - n;
             S.cursor[u] = carry + incl - n;
-            S.cgu[u] = (cts + it - tu) * ug;
-            S.cd[u] = (cts + it - tu) * ug / 2u;
         }
         carry += __shfl_sync(0xffffffffu, incl, 31);
-        cts += __shfl_sync(0xffffffffu, it, 31);
     }
-    GUB = cts * ug;
-    if (lane == 0) {
-        S.pfirst[U] = carry;
-        S.cgu[U] = GUB;
-        S.cd[U] = GUB >> 1;
-    }
+    if (lane == 0) S.pfirst[U] = carry;
     __syncwarp();
     // stable fill: pairs in ascending pair id order
     for (int base = 0; base < P; base += 32) {
@@ -666,7 +454,6 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
         const int rank = __popc(peers & ((1u << lane) - 1u));
         if (p < P) {
             const int pos = S.cursor[u] + rank;
-            S.ppair[pos] = p;
             S.ptok[pos] = (int)(((uint32_t)p * a.kmul) >> 16);
             S.pw[pos] = S.sel_w[p];
         }
@@ -674,250 +461,263 @@ __device__ __noinline__ void make_plan_many(const DecodeArgs &a, DecodeSmem &S, 
         if (p < P && rank == 0) S.cursor[u] += __popc(peers);
         __syncwarp();
     }
-    const uint32_t DB = GUB >> 1, B = GUB + DB;
-    int g0, g1, d0, d1;
-    uint32_t mj = 0;   // largest gate/up job (units)
-    for (int u = lane; u < U; u += 32) mj = max(mj, (S.cgu[u + 1] - S.cgu[u]) / pg);
-    mj = __reduce_max_sync(0xffffffffu, mj);
-    const bool mono = (unsigned long long)(mj + 2u) * (unsigned)nC <= DB;
-    int gcut = 0;
-    if (lane < 2) {
-        const int cc = c + lane;
-        gcut = (cc >= nC) ? U * pg : job_at_unit(S.cgu, U, pg, cut_units(a, GUB, cc, nC));
+}
+
+// Bytes one work unit of an expert of width `bits` streams: its two gate/up row blocks, its down
+// quarter and the down scale/zero entries of its group column.
+__device__ __forceinline__ unsigned long long unit_bytes(const DecodeArgs &a, int bits) {
+    return (unsigned long long)(2 * (a.H / kGroup)) * tile_bytes(bits) +
+           (unsigned long long)(a.H / 64) * d_quarter_bytes(bits) + 4ull * a.H;
+}
+
+// This CTA's range of work units [u0, u1): units are numbered slot-major (I / 16 per slot); CTA c
+// takes the units whose first byte lies in [c * B / nC, (c + 1) * B / nC) of the B bytes of all.
+__device__ void plan_units(const DecodeArgs &a, DecodeSmem &S, int lane, int c, int nC) {
+    const int U = S.U, sp = a.I / kSlice;
+    unsigned long long carry = 0;
+    for (int base = 0; base < U; base += 32) {
+        const int j = base + lane;
+        const unsigned long long cj = j < U ? (unsigned long long)sp * unit_bytes(a, S.ubits[j]) : 0ull;
+        unsigned long long incl = cj;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned long long o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (j < U) S.ccost[j] = carry + incl - cj;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    g0 = __shfl_sync(0xffffffffu, gcut, 0);
-    g1 = __shfl_sync(0xffffffffu, gcut, 1);
-    int dcut = 0;
-    if (lane < 2) {
-        const int cc = c + lane;
-        const int gj = lane == 0 ? g0 : g1;
-        const uint32_t pos = mono ? cut_units(a, B, cc, nC) - job_start_unit(S.cgu, U, pg, gj)
-                                  : cut_units(a, DB, cc, nC);
-        dcut = (cc >= nC) ? U * pd : job_at_unit(S.cd, U, pd, pos);
-    }
-    d0 = __shfl_sync(0xffffffffu, dcut, 0);
-    d1 = __shfl_sync(0xffffffffu, dcut, 1);
+    if (lane == 0) S.ccost[U] = carry;
+    __syncwarp();
+    const unsigned long long B = carry;
+    auto unit_at = [&](unsigned long long pos) -> int {
+        if (pos >= B) return U * sp;
+        int jj = 0;
+        for (int base = 0; base < U; base += 32) {
+            const int j = base + lane;
+            const bool h = j < U && S.ccost[j] <= pos && pos < S.ccost[j + 1];
+            const uint32_t m = __ballot_sync(0xffffffffu, h);
+            if (m) {
+                jj = base + __ffs(m) - 1;
+                break;
+            }
+        }
+        const unsigned long long ub = unit_bytes(a, S.ubits[jj]);
+        return jj * sp + (int)((pos - S.ccost[jj] + ub - 1) / ub);
+    };
+    const int u0 = unit_at(B * (unsigned long long)c / (unsigned long long)nC);
+    const int u1 = (c + 1 >= nC) ? U * sp : unit_at(B * (unsigned long long)(c + 1) / (unsigned long long)nC);
     if (lane == 0) {
-        S.g0 = g0;
-        S.g1 = g1;
-        S.d0 = d0;
-        S.d1 = d1;
-        S.nGU = g1 - g0;
+        S.u0 = u0;
+        S.u1 = u1;
     }
     __syncwarp();
 }
 
-// The plan, by one warp: unique experts in ascending id (slots), each slot's pair list in
-// ascending pair id (token-major, so ascending token), unit prefixes of the gate/up and down
-// job sequences, and this CTA's job ranges. P = 0 (an aborted routing) gives an empty plan.
-// A 64-byte unit is the granule of the job sequences: a tile of `bits` is tile_bytes(bits) / 64
-// units, a gate/up job G tiles and a down job GI tiles, so that an expert's down units are
-// exactly half its gate/up units.
-__device__ void make_plan(const DecodeArgs &a, DecodeSmem &S, int P, int lane, int c, int nC) {
-    if (P > 32) {
-        make_plan_many(a, S, P, lane, c, nC);
-        return;
-    }
-    const int H = a.H, I = a.I;
-    const int G = H / kGroup, GI = I / kGroup;
-    const int pg = I / 8, pd = H / 16;
-    const uint32_t ug = (uint32_t)pg * (uint32_t)G;   // gate/up units of an expert per unit of tile size
-    int U;
-    uint32_t GUB;                      // gate/up units of all slots
-    uint32_t lo, hi, ts;               // slot lanes: the slot's gate/up units [lo, hi), units per tile
-    int slot;                          // slot of the lane's expert
-    bool slot_lane;                    // the lane holds the first pair of its expert
-    uint32_t mts;                      // largest units per tile over the slots
-    bool uniform;                      // every slot has the same tile size (all jobs alike)
-    {
-        // One pair per lane. Each lane counts, over a packed list of all pairs {expert, units
-        // per tile, first pair of its expert}, the distinct experts below its own (its slot),
-        // their units and the pairs below it; the totals come out of the same pass.
-        const bool v = lane < P;
-        const int e = v ? S.sel_idx[lane] : 0;
-        const float pw = v ? S.sel_w[lane] : 0.f;
-        const int eb = S.ebits[e];
-        const uint32_t eo = S.eoff[e];
-        const uint32_t tsl = (uint32_t)tile_bytes(eb) / 64u;
-        uint32_t same = 1u << lane;   // one token: its experts are distinct
-        if (a.T > 1) same = __match_any_sync(0xffffffffu, v ? e : -1 - lane);
-        const int rank = __popc(same & ((1u << lane) - 1u));
-        const bool first = v && rank == 0;
-        // entries past P: an id above every expert, no units, not first
-        S.plist[lane] = v ? ((uint32_t)e | (tsl << 16) | (first ? 0x80000000u : 0u)) : 0xFFFFu;
-        __syncwarp();
-        uint32_t nsl = 0, units = 0, pbelow = 0, nU = 0, tot = 0, mtsmin = 0xFFFFu;
-        mts = 0;
-        const uint4 *pl = reinterpret_cast<const uint4 *>(S.plist);
-        for (int q4 = 0; q4 < (P + 3) / 4; ++q4) {
-            const uint4 w4 = pl[q4];
-            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t w = ws[j];
-                const bool lt = (w & 0xFFFFu) < (uint32_t)e;
-                const uint32_t tq = (w >> 31) ? (w >> 16) & 0x7FFFu : 0u;   // units of a first entry
-                pbelow += lt ? 1u : 0u;
-                nsl += (lt && tq) ? 1u : 0u;
-                units += lt ? tq : 0u;
-                nU += tq ? 1u : 0u;
-                tot += tq;
-                mts = max(mts, tq);
-                mtsmin = min(mtsmin, tq ? tq : 0xFFFFu);
-            }
-        }
-        U = (int)nU;
-        uniform = mts == mtsmin;
-        slot = (int)nsl;
-        slot_lane = first;
-        ts = tsl;
-        lo = units * ug;
-        hi = lo + tsl * ug;
-        GUB = tot * ug;
-        if (first) {
-            S.ubits[slot] = eb;
-            S.uoff[slot] = eo;
-            S.pfirst[slot] = (int)pbelow;
-            S.cgu[slot] = lo;
-            S.cd[slot] = lo >> 1;
-        }
-        if (v) {
-            const int pos = (int)pbelow + rank;
-            S.ppair[pos] = lane;
-            S.ptok[pos] = (int)(((uint32_t)lane * a.kmul) >> 16);
-            S.pw[pos] = pw;
-        }
-        if (lane == 0) {
-            S.U = U;
-            S.pfirst[U] = P;
-            S.cgu[U] = GUB;
-            S.cd[U] = GUB >> 1;
-        }
-    }
-    // Job ranges. The gate/up sequence is cut at multiples of its units / nCTA; the down
-    // sequence is cut so that each CTA's gate/up + down units are the layer's units / nCTA. That
-    // cut is monotone in the CTA index when every CTA's down share exceeds one gate/up job (plus
-    // rounding); otherwise (tiny layers) the down sequence is cut on its own.
-    const uint32_t DB = GUB >> 1, B = GUB + DB;
-    int g0, g1, d0, d1;
-    {
-        const uint32_t jbg = ts * (uint32_t)G, jbd = ts * (uint32_t)GI;   // units per job of the lane's slot
-        const uint32_t mj = mts * (uint32_t)G;                            // largest gate/up job
-        const bool mono = (unsigned long long)(mj + 2u) * (unsigned)nC <= DB;
-        uint32_t st0, st1, unused;
-        if (uniform && U > 0) {
-            // all jobs of a sequence alike: the first job at or after q is ceil(q / job units)
-            const uint32_t ug1 = mts * (uint32_t)G, ud1 = mts * (uint32_t)GI;
-            const int NG = U * pg, ND = U * pd;
-            g0 = min(NG, (int)ceil_div_small(cut_units(a, GUB, c, nC), ug1));
-            g1 = (c + 1 < nC) ? min(NG, (int)ceil_div_small(cut_units(a, GUB, c + 1, nC), ug1)) : NG;
-            const uint32_t q0 = mono ? cut_units(a, B, c, nC) - (uint32_t)g0 * ug1 : cut_units(a, DB, c, nC);
-            const uint32_t q1 = mono ? cut_units(a, B, c + 1, nC) - (uint32_t)g1 * ug1 : cut_units(a, DB, c + 1, nC);
-            d0 = min(ND, (int)ceil_div_small(q0, ud1));
-            d1 = (c + 1 < nC) ? min(ND, (int)ceil_div_small(q1, ud1)) : ND;
-        } else {
-        g0 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(a, GUB, c, nC), GUB, st0);
-        if (c + 1 < nC) {
-            g1 = job_at_unit_warp(lo, hi, jbg, slot, slot_lane, pg, U, cut_units(a, GUB, c + 1, nC), GUB, st1);
-        } else {
-            g1 = U * pg;
-            st1 = GUB;
-        }
-        const uint32_t q0 = mono ? cut_units(a, B, c, nC) - st0 : cut_units(a, DB, c, nC);
-        d0 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q0, DB, unused);
-        if (c + 1 < nC) {
-            const uint32_t q1 = mono ? cut_units(a, B, c + 1, nC) - st1 : cut_units(a, DB, c + 1, nC);
-            d1 = job_at_unit_warp(lo >> 1, hi >> 1, jbd, slot, slot_lane, pd, U, q1, DB, unused);
-        } else {
-            d1 = U * pd;
-        }
-        }
-    }
-    if (lane == 0) {
-        S.g0 = g0;
-        S.g1 = g1;
-        S.d0 = d0;
-        S.d1 = d1;
-        S.nGU = g1 - g0;
-    }
-    __syncwarp();
+// ------------------------------------------------------------------------------ work units
+struct UnitGeo {
+    const uint8_t *gu, *sz, *q;   // gate/up tiles, down scale/zero entries, down quarter
+    int j, i, bits;               // expert slot, 16-row slice, code width
+};
+__device__ __forceinline__ UnitGeo unit_geo(const DecodeArgs &a, const DecodeSmem &S, int u) {
+    const int sp = a.I / kSlice;
+    UnitGeo g;
+    g.j = u / sp;
+    g.i = u - g.j * sp;
+    g.bits = S.ubits[g.j];
+    const int tb = tile_bytes(g.bits);
+    const uint8_t *base = a.packed + (size_t)S.uoff[g.j] * 256;
+    g.gu = base + (size_t)(2 * g.i) * (a.H / kGroup) * tb;
+    const uint8_t *blk = base + gu_tiles(a.H, a.I) * tb + (size_t)(g.i >> 2) * d_block_bytes(a.H, g.bits);
+    g.sz = blk;
+    g.q = blk + d_quarter_offset(a.H, g.bits, g.i & 3);
+    return g;
+}
+// chunks of a unit: its 2 * KG gate/up tiles, then its H / 64 down super-tiles (each chunk one
+// ring stage), cut into nearly equal parts
+__device__ __forceinline__ int gu_chunks(int KG, int tb) {
+    const int cap = kStageBytes / tb;
+    return (2 * KG + cap - 1) / cap;
+}
+__device__ __forceinline__ int d_chunks(int nst, int qb) {
+    const int cap = kStageBytes / (256 + qb);
+    return (nst + cap - 1) / cap;
+}
+__device__ __forceinline__ void split_range(int n, int parts, int i, int &b, int &e) {
+    const int base = n / parts, rem = n % parts;
+    b = i * base + (i < rem ? i : rem);
+    e = b + base + (i < rem ? 1 : 0);
 }
 
-// ------------------------------------------------------------------------------ finalisation
-// Gate/up job gj: SiLU-GLU of the slot's sums (rows 0-7 gate, 8-15 up of intermediate rows
-// 8 rb .. 8 rb + 7), h stored as a bf16 pair hi + lo (exact to about 2^-17 relative); the
-// slot is cleared for its next job.
+// ------------------------------------------------------------------------------ tile math
+// Operand sources of the current expert slot for this lane: per n-tile, the x row that the
+// lane's B column reads (a valid row also where the column has no token: those columns are
+// never used) and the group-sum rows of its two accumulator columns.
 template <int NT>
-__device__ __forceinline__ void finalize_gu(const DecodeArgs &a, const DecodeSmem &S, int gj, float *slot, int lane) {
-    const int pg = a.I / 8;
-    const int u = gj / pg, rb = gj % pg;
-    const int pf = S.pfirst[u], nu = S.pfirst[u + 1] - pf;
+struct GuCtx {
+    const uint16_t *b[NT];   // global x rows (!xs_on)
+    uint32_t sb[NT];         // shared-memory x rows (xs_on)
+    uint32_t xs0[NT], xs1[NT];
+    bool bg;
+};
+
+template <int BITS, int NT>
+__device__ __forceinline__ void gu_tile(const uint8_t *tile, int kg, const GuCtx<NT> &jc, int lane,
+                                        float (&acc)[NT][4]) {
     const int g = lane >> 2, t = lane & 3;
+    const uint4 lo = *reinterpret_cast<const uint4 *>(tile + 16 * lane);
+    uint4 hi8 = make_uint4(0, 0, 0, 0);
+    uint2 hi6 = make_uint2(0, 0);
+    if (BITS == 8) hi8 = *reinterpret_cast<const uint4 *>(tile + kLoBytes + 16 * lane);
+    if (BITS == 6) hi6 = *reinterpret_cast<const uint2 *>(tile + kLoBytes + 8 * lane);
+    const uint2 sz = *reinterpret_cast<const uint2 *>(tile + kLoBytes + hi_bytes(BITS) + 8 * g);
+    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-        float *sp = slot + nt * 128 + lane;
-        const float gate[2] = {sp[0], sp[32]}, up[2] = {sp[64], sp[96]};
-        sp[0] = sp[32] = sp[64] = sp[96] = 0.f;
+        uint4 v0, v1;
+        if (jc.bg) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(jc.b[nt] + kg * kGroup + 16 * t);
+            v0 = __ldcg(p);
+            v1 = __ldcg(p + 1);
+        } else {
+            const uint32_t o = (uint32_t)(kg * kGroup + 16 * t) * 2;
+            v0 = lds128(jc.sb[nt] + o);
+            v1 = lds128(jc.sb[nt] + o + 16);
+        }
+        const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const float X0 = lds32f(jc.xs0[nt] + kg * 4), X1 = lds32f(jc.xs1[nt] + kg * 4);
+        tile_group_mma<BITS>(lo, hi8, hi6, b, nullptr, sA, zA, sB, zB, X0, X1, acc[nt]);
+    }
+}
+
+// The warp's gate/up tiles of a chunk holding the unit's tiles [t0, t1) (tile tt = row block
+// tt / KG, group column tt % KG): group column kg goes to warp kg % CW, two tiles at a time so
+// that their MMA chains interleave.
+template <int BITS, int NT, int CW>
+__device__ __forceinline__ void gu_chunk(const uint8_t *stage, int t0, int t1, int KG, int warp,
+                                         const GuCtx<NT> &jc, int lane, float (&acc)[2][NT][4]) {
+    constexpr int tb = tile_bytes(BITS);
+#pragma unroll
+    for (int rbl = 0; rbl < 2; ++rbl) {
+        const int lo_t = max(t0, rbl * KG), hi_t = min(t1, (rbl + 1) * KG);
+        if (lo_t >= hi_t) continue;
+        const int k0 = lo_t - rbl * KG, k1 = hi_t - rbl * KG;
+        int kg = k0 + ((warp - k0) % CW + CW) % CW;
+        const uint8_t *p0 = stage + (size_t)(rbl * KG - t0) * tb;
+        for (; kg + CW < k1; kg += 2 * CW) {
+            gu_tile<BITS, NT>(p0 + (size_t)kg * tb, kg, jc, lane, acc[rbl]);
+            gu_tile<BITS, NT>(p0 + (size_t)(kg + CW) * tb, kg + CW, jc, lane, acc[rbl]);
+        }
+        if (kg < k1) gu_tile<BITS, NT>(p0 + (size_t)kg * tb, kg, jc, lane, acc[rbl]);
+    }
+}
+
+// Down operands of the current unit for this lane: h of the unit's 16 rows for the lane's B
+// column (pair g of each n-tile) as bf16 hi / lo pairs (and x16 copies for the 6/8-bit high code
+// planes), the sums X of h over the 16 rows and the routing weights of its two accumulator
+// columns (0 where the column has no pair).
+template <int NT>
+struct DnCtx {
+    uint32_t hb[NT][2], lb[NT][2], hb16[NT][2], lb16[NT][2];
+    float X0[NT], X1[NT], w0[NT], w1[NT];
+};
+
+// One 64-row super-tile of the unit's down quarter: four 16x16 MMAs (per n-tile and h half), the
+// row's scale and zero and the column's weight applied in fp32: acc += w * s * (sum - (off + z) X).
+template <int BITS, int NT>
+__device__ __forceinline__ void down_st(uint32_t szp, uint32_t qp, const DnCtx<NT> &dc, int lane,
+                                        float (&acc)[4][NT][4]) {
+    const int g = lane >> 2;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const uint32_t w = lds32(qp + r * 128 + 4 * lane);
+        uint32_t hw = 0;
+        if (BITS == 8) hw = lds32(qp + kLoBytes + r * 128 + 4 * lane);
+        if (BITS == 6) hw = __byte_perm(lds16(qp + kLoBytes + r * 64 + 2 * lane), 0u, 0x4140);
+        const uint2 sz = lds64(szp + r * 64 + 8 * g);
+        const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
+        const uint32_t a0 = code_pair<0x000F000Fu>(w, 0), a1 = code_pair<0x000F000Fu>(w, 4);
+        const uint32_t a2 = code_pair<0x000F000Fu>(w, 8), a3 = code_pair<0x000F000Fu>(w, 12);
+        uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+        if (BITS == 8) {
+            h0 = code_pair<0x000F000Fu>(hw, 0);
+            h1 = code_pair<0x000F000Fu>(hw, 4);
+            h2 = code_pair<0x000F000Fu>(hw, 8);
+            h3 = code_pair<0x000F000Fu>(hw, 12);
+        }
+        if (BITS == 6) {
+            h0 = code_pair<0x00030003u>(hw, 0);
+            h1 = code_pair<0x00030003u>(hw, 2);
+            h2 = code_pair<0x00030003u>(hw, 4);
+            h3 = code_pair<0x00030003u>(hw, 6);
+        }
+        const float off = (BITS == 4) ? 128.f : 2176.f;   // 128 per plane, the hi plane weighted 16x
+        const float oA = off + zA, oB = off + zB;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(c, a0, a1, a2, a3, dc.hb[nt][0], dc.hb[nt][1]);
+            mma_bf16(d, a0, a1, a2, a3, dc.lb[nt][0], dc.lb[nt][1]);
+            if (BITS != 4) {
+                mma_bf16(c, h0, h1, h2, h3, dc.hb16[nt][0], dc.hb16[nt][1]);
+                mma_bf16(d, h0, h1, h2, h3, dc.lb16[nt][0], dc.lb16[nt][1]);
+            }
+            acc[r][nt][0] += (sA * dc.w0[nt]) * ((c[0] + d[0]) - oA * dc.X0[nt]);
+            acc[r][nt][1] += (sA * dc.w1[nt]) * ((c[1] + d[1]) - oA * dc.X1[nt]);
+            acc[r][nt][2] += (sB * dc.w0[nt]) * ((c[2] + d[2]) - oB * dc.X0[nt]);
+            acc[r][nt][3] += (sB * dc.w1[nt]) * ((c[3] + d[3]) - oB * dc.X1[nt]);
+        }
+    }
+}
+
+// Adds one super-tile's accumulators into the fp32 output: rows 64 st + 16 r + g (+8), the
+// tokens of the lane's columns (pairs pf + nt * 8 + 2t + col of the slot, nj of them).
+template <int NT>
+__device__ __forceinline__ void emit_st(const DecodeArgs &a, const DecodeSmem &S, int pf, int nj, int st,
+                                        const float (&acc)[4][NT][4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int col = 0; col < 2; ++col) {
             const int q = nt * 8 + 2 * t + col;
-            if (q < nu) {
-                const float h = __fdividef(gate[col], 1.f + __expf(-gate[col])) * up[col];
-                const __nv_bfloat16 hi = __float2bfloat16_rn(h);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
-                const size_t o = (size_t)S.ppair[pf + q] * a.I + rb * 8 + g;
-                a.h_hi[o] = __bfloat16_as_ushort(hi);
-                a.h_lo[o] = __bfloat16_as_ushort(lo);
+            if (q < nj) {
+                float *o = a.out_acc + (size_t)S.ptok[pf + q] * a.H + 64 * st + g;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    red_add_f32(o + 16 * r, acc[r][nt][col]);
+                    red_add_f32(o + 16 * r + 8, acc[r][nt][2 + col]);
+                }
             }
         }
-    }
-
-}
-// Down job dj, computed whole by one warp: w * y of rows 16 rb + g and 16 rb + g + 8 added into
-// the fp32 output accumulator.
-// Down job dj, summed in one warp's registers: w * y added into the fp32 output accumulator.
-template <int NT>
-__device__ __forceinline__ void finalize_down(const DecodeArgs &a, const DecodeSmem &S, int dj, const float (&acc)[NT][4],
-                                              const float (&acc2)[NT][4], int lane) {
-    const int pd = a.H / 16;
-    const int u = dj / pd, rb = dj % pd;
-    const int pf = S.pfirst[u], nu = S.pfirst[u + 1] - pf;
-    const int g = lane >> 2, t = lane & 3;
-    const int row = rb * 16 + g;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int col = 0; col < 2; ++col) {
-            const int q = nt * 8 + 2 * t + col;
-            if (q < nu) {
-                float *o = a.out_acc + (size_t)S.ptok[pf + q] * a.H + row;
-                const float wgt = S.pw[pf + q];
-                red_add_f32(o, wgt * (acc[nt][col] + acc2[nt][col]));
-                red_add_f32(o + 8, wgt * (acc[nt][2 + col] + acc2[nt][2 + col]));
-            }
-        }
-    }
 }
 
 // ------------------------------------------------------------------------------ kernel
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a, const DecodeLayout L) {
+// NT: MMA n-tiles (8 tokens each) per unit; CW: consumer warps; STW: how a warp keeps the output
+// rows of its super-tiles across units: > 0, in registers, STW super-tiles per warp (several
+// tokens: the units of one expert slot); 0, not at all (each super-tile's rows are added out at
+// once); -1, in shared memory (one token: all units of the CTA).
+template <int NT, int STW, int CW>
+__global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a, const DecodeLayout L) {
+    constexpr int kCW = CW, kPW = CW, kWarps = CW + 1, kThreads = kWarps * 32;
     extern __shared__ __align__(128) uint8_t dyn[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(dyn);
-    uint8_t *act = dyn + L.act;
-    float *accs = reinterpret_cast<float *>(dyn + L.accs);
-    float *Xs = reinterpret_cast<float *>(dyn + L.xs);
     uint8_t *ring = dyn + L.ring;
-    constexpr int NSLOT = slots_for<NT>();
-    constexpr int SF = slot_floats<NT>();
+    float *Xs = reinterpret_cast<float *>(dyn + L.xsum);
+    float *gred = reinterpret_cast<float *>(dyn + L.gred);
+    uint16_t *hhi = reinterpret_cast<uint16_t *>(dyn + L.hbuf);
+    uint16_t *hlo = hhi + NT * 8 * 16;
+    float *hX = reinterpret_cast<float *>(dyn + L.hcol);
+    float *hW = hX + NT * 8;
+    float *ycta = reinterpret_cast<float *>(dyn + L.ycta);
     const int NS = L.stages;
-    const int T = a.T, H = a.H, I = a.I, E = a.E, K = a.k, P = T * K;
-    const int G = H / kGroup, GI = I / kGroup;
+    const int T = a.T, H = a.H, E = a.E, K = a.k, P = T * K;
+    const int G = H / kGroup, KG = G, nst = H / 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nC = gridDim.x, c = blockIdx.x;
     uint32_t *status = &a.ctl->status;
     const bool xs_on = (size_t)T * H * 2 <= (size_t)kActBytes;
-    const uint16_t *xsm = reinterpret_cast<const uint16_t *>(act);
+    const uint16_t *xsm = reinterpret_cast<const uint16_t *>(dyn + L.xs);
     const int ne = (E > c) ? (E - c + nC - 1) / nC : 0;   // router rows of this CTA: c, c+nC, ...
     const bool wr_on = (size_t)ne * H * 4 <= (size_t)NS * kStageBytes;
     const float *wsm = reinterpret_cast<const float *>(ring);
@@ -932,7 +732,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         mbar_init(smem_u32(&S.xbar), 1);
         fence_barrier_init();
         S.abort = 0;
-        S.is_last = 0;
         if (wr_on && ne > 0) {
             const uint32_t rowb = (uint32_t)H * 4;
             mbar_expect_tx(smem_u32(&S.wbar), rowb * ne);
@@ -950,7 +749,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             S.ebits[e] = (uint8_t)v.bits;
         }
     }
-    for (int i = threadIdx.x; i < NSLOT * SF; i += kThreads) accs[i] = 0.f;
+    for (int i = threadIdx.x; i < 2 * NT * 4 * 32; i += kThreads) gred[i] = 0.f;
+    if (STW < 0)
+        for (int i = threadIdx.x; i < H; i += kThreads) ycta[i] = 0.f;
     // the router bias of this CTA's rows (a weight), off the logits' critical path
     if (threadIdx.x < ne && threadIdx.x < kBiasRows) S.bias[threadIdx.x] = a.bias ? a.bias[c + threadIdx.x * nC] : 0.f;
     __syncthreads();
@@ -963,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (xs_on) {
             const uint32_t bytes = (uint32_t)(T * H * 2);
             mbar_expect_tx(smem_u32(&S.xbar), bytes);
-            bulk_g2s(smem_u32(act), a.x, bytes, smem_u32(&S.xbar));
+            bulk_g2s(smem_u32(dyn + L.xs), a.x, bytes, smem_u32(&S.xbar));
         }
         S.epoch = *reinterpret_cast<volatile unsigned long long *>(&a.ctl->done) / (unsigned long long)nC;
     }
@@ -975,9 +776,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const uint16_t *xr = xs_on ? xsm : a.x;
     // The CTA's ne * T dot products over H. With fewer of them than warps each is split into
     // slices of whole 256-element strides, one slice per warp, and the slices' sums are added
-    // in slice order.
-    // Every logit word goes to lrep copies of the T x E block (lstride words apart, spread over
-    // the L2 slices); CTA c polls copy c mod lrep, so that no slice serves all CTAs' polls.
+    // in slice order. Every logit word goes to lrep copies of the T x E block (lstride words
+    // apart, spread over the L2 slices); CTA c polls copy c mod lrep.
     auto row_bias = [&](int i, int e) -> float { return i < kBiasRows ? S.bias[i] : (a.bias ? a.bias[e] : 0.f); };
     auto publish_logit = [&](int t, int e, float l) {
         const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(l);
@@ -1052,59 +852,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // tokens go to warps from the control warp on, so that with one token the control warp routes
     // it and makes the plan without a CTA barrier in between
     for (int t = (warp + 1) % kWarps; t < T; t += kWarps) route_token(t);
-    if (warp != kCW || T > 1) group_sums(threadIdx.x, T > 1 ? kThreads : kCW * 32);
+    if (warp != kPW || T > 1) group_sums(threadIdx.x, T > 1 ? kThreads : kCW * 32);
     if (T > 1) __syncthreads();
-    if (warp == kCW) {
+    if (warp == kPW) {
         __syncwarp();
-        make_plan(a, S, S.abort ? 0 : P, lane, c, nC);
-        __syncwarp();
+        const int Pp = S.abort ? 0 : P;
+        if (T == 1) plan_single(S, Pp, lane);
+        else plan_many(a, S, Pp, lane);
+        plan_units(a, S, lane, c, nC);
         // hand the plan to the consumer warps and start streaming without waiting for them
-        plan_ready_arrive();
+        plan_ready_arrive<CW>();
         // ------------------------------------------------------------ producer (one thread)
         if (lane != 0) return;
         uint32_t cc = 0;
         bool ok = true;
-        const bool has_down = S.d1 > S.d0;
-        for (int ph = 0; ph < 2 && ok; ++ph) {
-            const bool gu = ph == 0;
-            const int jend = gu ? S.g1 : S.d1;
-            for (int j = gu ? S.g0 : S.d0; j < jend && ok;) {
-                const Region r = region_at(S, a, gu, j);
-                const int nch = region_chunks(r, gu ? chunk_jobs<NT>() : kStageBytes);
-                const int jnext = j + r.tiles / r.tpj;
-                for (int ch = 0; ch < nch; ++ch) {
-                    int c0, m;
-                    chunk_range(r, nch, ch, c0, m);
-                    const int s = cc % NS;
-                    const uint32_t use = cc / NS;
-                    if (use > 0 && (S.abort || !mbar_wait(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
-                        S.abort = 1;
-                        ok = false;
-                        break;
-                    }
-                    // the chunk's descriptor, published to the consumers by the barrier's arrival
-                    const int jlo = c0 / r.tpj, jhi = (c0 + m - 1) / r.tpj;
-                    ChunkDesc dd;
-                    dd.job0 = r.jg0 + jlo;
-                    dd.base_off = (jlo * r.tpj - c0) * r.tb;
-                    dd.njobs = (short)(jhi - jlo + 1);
-                    dd.k0 = (short)(c0 - jlo * r.tpj);
-                    dd.k1 = (short)(c0 + m - jhi * r.tpj);
-                    dd.tpj = (short)r.tpj;
-                    dd.tb = (unsigned short)r.tb;
-                    dd.bits = (unsigned char)r.bits;
-                    const bool last = ch == nch - 1 && jnext >= jend && (!gu || !has_down);
-                    dd.flags = (unsigned char)((gu ? 1 : 0) | (last ? 2 : 0));
-                    dd.u = (short)r.u;
-                    dd.pad = 0;
-                    S.desc[s] = dd;
-                    const uint32_t bytes = (uint32_t)(m * r.tb);
-                    const uint32_t fb = smem_u32(&S.full[s]);
-                    mbar_expect_tx(fb, bytes);
-                    bulk_g2s(smem_u32(ring + (size_t)s * kStageBytes), r.src + (size_t)c0 * r.tb, bytes, fb);
-                    ++cc;
+        for (int u = S.u0; u < S.u1 && ok; ++u) {
+            const UnitGeo ug = unit_geo(a, S, u);
+            const int tb = tile_bytes(ug.bits), qb = d_quarter_bytes(ug.bits);
+            const int ngc = gu_chunks(KG, tb), ndc = d_chunks(nst, qb);
+            for (int ch = 0; ch < ngc + ndc; ++ch) {
+                const int s = cc % NS;
+                const uint32_t use = cc / NS;
+                if (use > 0 && (S.abort || !mbar_wait(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
+                    S.abort = 1;
+                    ok = false;
+                    break;
                 }
-                j = jnext;
+                const uint32_t fb = smem_u32(&S.full[s]);
+                uint8_t *dst = ring + (size_t)s * kStageBytes;
+                int b0, b1;
+                if (ch < ngc) {
+                    split_range(2 * KG, ngc, ch, b0, b1);
+                    const uint32_t bytes = (uint32_t)((b1 - b0) * tb);
+                    mbar_expect_tx(fb, bytes);
+                    bulk_g2s(smem_u32(dst), ug.gu + (size_t)b0 * tb, bytes, fb);
+                } else {
+                    split_range(nst, ndc, ch - ngc, b0, b1);
+                    const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * qb);
+                    mbar_expect_tx(fb, zb + qbytes);
+                    bulk_g2s(smem_u32(dst), ug.sz + (size_t)b0 * 256, zb, fb);
+                    bulk_g2s(smem_u32(dst + zb), ug.q + (size_t)b0 * qb, qbytes, fb);
+                }
+                ++cc;
             }
         }
         // copies still in flight land before the CTA may exit
@@ -1114,219 +903,245 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
 
     // ---------------------------------------------------------------- consumers
-    plan_ready_wait();
+    plan_ready_wait<CW>();
     const int g = lane >> 2, t = lane & 3;
-    float acc[NT][4], acc2[NT][4];
-    auto zero_acc = [&]() {
+    constexpr int NL = STW > 0 ? STW : 1;
+    static_assert(STW >= 0 || NT == 1, "shared-memory output rows serve one token");
+    float yacc[NL][4][NT][4];
+    auto zero_y = [&]() {
 #pragma unroll
-        for (int i = 0; i < NT; ++i) {
-            acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-            acc2[i][0] = acc2[i][1] = acc2[i][2] = acc2[i][3] = 0.f;
-        }
-    };
-    JobCtx<NT> jc;
-    bool hfit = true;
-    const uint16_t *hh = nullptr, *hl = nullptr;
-    const float *hs = nullptr;
-
-    // h of expert slot u into shared memory (with its per-group sums), after the expert's
-    // gate/up rows are published by every CTA that computed some; all consumer warps take part.
-    // This CTA's gate/up rows are all stored (their finalisers passed a consumer barrier since):
-    // one fence makes them visible GPU-wide, then each expert's counter grows by the CTA's jobs.
-    bool published = false;
-    auto publish_h = [&]() {
-        if (threadIdx.x == 0 && !published && S.g1 > S.g0) {
-            __threadfence();
-            const int pg = I / 8;
-            const int u0 = S.g0 / pg, u1 = (S.g1 - 1) / pg;
-            for (int u = u0; u <= u1; ++u)
-                atomicAdd(&a.h_ready[u], (uint32_t)(min(S.g1, (u + 1) * pg) - max(S.g0, u * pg)));
-        }
-        published = true;
-    };
-    auto load_h = [&](int u) {
-        consumer_sync();   // nobody still reads the previous contents of act
-        if (!S.abort) publish_h();
-        if (threadIdx.x == 0 && !S.abort &&
-            !wait_counter(&a.h_ready[u], (uint32_t)(I / 8), a.wait_ns, status))
-            S.abort = 1;
-        consumer_sync();
-        const int pf = S.pfirst[u], nu = S.pfirst[u + 1] - pf;
-        const size_t hsb = align_up((size_t)nu * GI * 4, 16), hb = (size_t)nu * I * 2;
-        hfit = hsb + 2 * hb <= (size_t)kActBytes;
-        float *hsw = reinterpret_cast<float *>(act);
-        uint16_t *hhw = reinterpret_cast<uint16_t *>(act + hsb), *hlw = hhw + (size_t)nu * I;
-        if (!S.abort) {
-            // eight threads per group of 64 values: one 16-byte piece of h hi and of h lo each,
-            // the group's sum over a 3-step shuffle
-            const int n8 = nu * GI * 8;
-            for (int base = threadIdx.x - lane; base < n8; base += kCW * 32) {
-                const int i8 = base + lane;
-                const bool v = i8 < n8;
-                const int item = i8 >> 3, part = i8 & 7;
-                const int q = item / GI, grp = item - q * GI;
-                uint4 vh = make_uint4(0, 0, 0, 0), vl = make_uint4(0, 0, 0, 0);
-                if (v) {
-                    const size_t o = (size_t)S.ppair[pf + q] * I + (size_t)grp * kGroup + part * 8;
-                    vh = __ldcg(reinterpret_cast<const uint4 *>(a.h_hi + o));
-                    vl = __ldcg(reinterpret_cast<const uint4 *>(a.h_lo + o));
-                }
-                const uint32_t w8[8] = {vh.x, vh.y, vh.z, vh.w, vl.x, vl.y, vl.z, vl.w};
-                float sum = 0.f;
+        for (int l = 0; l < NL; ++l)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) sum += __uint_as_float(w8[j] << 16) + __uint_as_float(w8[j] & 0xFFFF0000u);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-                if (v && part == 0) hsw[item] = sum;
-                if (v && hfit) {
-                    const size_t d = (size_t)q * I + (size_t)grp * kGroup + part * 8;
-                    *reinterpret_cast<uint4 *>(hhw + d) = vh;
-                    *reinterpret_cast<uint4 *>(hlw + d) = vl;
-                }
-            }
-        }
-        consumer_sync();
-        hs = hsw;
-        hh = hhw;
-        hl = hlw;
-    };
-    auto set_ctx = [&](int u, bool gu) {
-        const int pf = S.pfirst[u];
-        const int nu = S.pfirst[u + 1] - pf;
+            for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int q = nt * 8 + g, q0 = nt * 8 + 2 * t, q1 = q0 + 1;
-            jc.has[nt] = q < nu;
-            jc.has0[nt] = q0 < nu;
-            jc.has1[nt] = q1 < nu;
-            const int qq = q < nu ? q : 0, qq0 = q0 < nu ? q0 : 0, qq1 = q1 < nu ? q1 : 0;
-            if (gu) {
-                const int tok = S.ptok[pf + qq];
-                jc.b[nt] = a.x + (size_t)tok * H;
-                jc.b2[nt] = nullptr;
-                jc.sb[nt] = smem_u32(xsm) + (uint32_t)(tok * H * 2);
-                jc.sb2[nt] = 0;
-                jc.xs0[nt] = smem_u32(Xs) + (uint32_t)(S.ptok[pf + qq0] * G * 4);
-                jc.xs1[nt] = smem_u32(Xs) + (uint32_t)(S.ptok[pf + qq1] * G * 4);
-            } else {
-                jc.b[nt] = a.h_hi + (size_t)S.ppair[pf + qq] * I;
-                jc.b2[nt] = a.h_lo + (size_t)S.ppair[pf + qq] * I;
-                jc.sb[nt] = smem_u32(hh) + (uint32_t)(qq * I * 2);
-                jc.sb2[nt] = smem_u32(hl) + (uint32_t)(qq * I * 2);
-                jc.xs0[nt] = smem_u32(hs) + (uint32_t)(qq0 * GI * 4);
-                jc.xs1[nt] = smem_u32(hs) + (uint32_t)(qq1 * GI * 4);
-            }
-        }
-        jc.bg = gu ? !xs_on : !hfit;
+                for (int nt = 0; nt < NT; ++nt) yacc[l][r][nt][0] = yacc[l][r][nt][1] = yacc[l][r][nt][2] = yacc[l][r][nt][3] = 0.f;
     };
-    // Gate/up jobs are split along K: tile k of a job goes to warp k % kCW, which adds its partial
-    // sums into the job's slot (CTA-local job q uses slot q % NSLOT) after its last tile of the
-    // job. A down job (a few tiles) belongs to one warp and is finalised from its registers.
-    auto add_partial = [&](int q) {
-        float *sp = accs + (q % NSLOT) * SF;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) red_shared_f32(sp + (nt * 4 + i) * 32 + lane, acc[nt][i] + acc2[nt][i]);
-        zero_acc();
-    };
-    // Gate/up jobs fj0 .. fj0 + fn - 1 have all their partials in their slots (after the barrier
-    // that follows the chunk that completed them); warp gj % kCW finalises job gj.
-    int fj0 = 0, fn = 0;
-    auto finalize_pending = [&]() {
-        for (int i = 0; i < fn; ++i) {
-            const int gj = fj0 + i;
-            if (gj % kCW == warp) finalize_gu<NT>(a, S, gj, accs + ((gj - S.g0) % NSLOT) * SF, lane);
-        }
-        fn = 0;
-    };
-
-    zero_acc();
+    zero_y();
+    GuCtx<NT> jc;
+    jc.bg = !xs_on;
     int s = 0;
     uint32_t par = 0;
-    int cur_u = -1, cur_gu = -1, tpj = 1, kl = -1;
-    bool more = S.g1 > S.g0 || S.d1 > S.d0;
-    while (more) {
-        const bool got = !S.abort && mbar_wait(smem_u32(&S.full[s]), par, a.wait_ns, status);
-        // One barrier per chunk: every warp's partials of the previous chunk are in, and all
-        // warps take the same abort decision.
-        if (consumer_sync_or(!got || S.abort)) {
-            if (lane == 0) S.abort = 1;
-            break;
-        }
-        finalize_pending();
-        const ChunkDesc d = S.desc[s];
-        const bool gu = d.flags & 1;
-        if (d.u != cur_u || (int)gu != cur_gu) {
-            if (!gu) load_h(d.u);
-            set_ctx(d.u, gu);
-            cur_u = d.u;
-            cur_gu = gu;
-            tpj = d.tpj;
-            kl = (warp < tpj) ? warp + kCW * ((tpj - 1 - warp) / kCW) : -1;   // this warp's last tile of a job
-        }
-        const uint8_t *sb = ring + (size_t)s * kStageBytes + d.base_off;
-        for (int i = 0; i < d.njobs; ++i) {
-            const int k0 = i == 0 ? d.k0 : 0, k1 = i == d.njobs - 1 ? d.k1 : tpj;
-            const uint8_t *job_base = sb + (size_t)i * tpj * d.tb;
-            const int gj = d.job0 + i;
-            if (gu) {
-                if (d.bits == 4) run_tiles<4, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
-                else if (d.bits == 6) run_tiles<6, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
-                else run_tiles<8, NT, true>(job_base, d.tb, k0, k1, warp, jc, lane, acc, acc2);
-                if (kl >= k0 && kl < k1) add_partial(gj - S.g0);
-            } else if ((gj - S.d0) % kCW == warp) {
-                if (d.bits == 4) run_tiles_seq<4, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
-                else if (d.bits == 6) run_tiles_seq<6, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
-                else run_tiles_seq<8, NT>(job_base, d.tb, k0, k1, jc, lane, acc, acc2);
-                if (k1 == tpj) {
-                    finalize_down<NT>(a, S, gj, acc, acc2, lane);
-                    zero_acc();
-                }
+    bool bad = false, aborted = false;
+    int cur = -1, cur_pf = 0, cur_nj = 0;
+    // the carried output rows of the current slot (several tokens: its pairs' tokens)
+    auto flush_slot = [&]() {
+        if (STW > 0) {
+#pragma unroll
+            for (int l = 0; l < NL; ++l) {
+                const int st = warp + l * kCW;
+                if (st < nst) emit_st<NT>(a, S, cur_pf, cur_nj, st, yacc[l], lane);
             }
+            zero_y();
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
-        fj0 = d.job0;
-        fn = gu ? d.njobs - (d.k1 < tpj ? 1 : 0) : 0;
-        more = !(d.flags & 2);
+    };
+    auto next_stage = [&]() {
         if (++s == NS) {
             s = 0;
             par ^= 1u;
         }
-    }
-    if (!consumer_sync_or(S.abort)) {
-        finalize_pending();
-        if (!published) {
-            // no down job here: the gate/up rows are published after their finalisers are done
-            consumer_sync();
-            publish_h();
+    };
+    auto wait_full = [&]() {
+        if (!bad && (S.abort || !mbar_wait(smem_u32(&S.full[s]), par, a.wait_ns, status))) bad = true;
+    };
+    auto release_stage = [&]() {
+        __syncwarp();
+        if (!bad && lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
+        next_stage();
+    };
+    for (int u = S.u0; u < S.u1; ++u) {
+        const UnitGeo ug = unit_geo(a, S, u);
+        if (ug.j != cur) {
+            if (T > 1 && cur >= 0 && !bad) flush_slot();
+            cur = ug.j;
+            cur_pf = S.pfirst[cur];
+            cur_nj = S.pfirst[cur + 1] - cur_pf;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int q = nt * 8 + g, q0 = nt * 8 + 2 * t, q1 = q0 + 1;
+                const int tok = S.ptok[cur_pf + (q < cur_nj ? q : 0)];
+                jc.b[nt] = a.x + (size_t)tok * H;
+                jc.sb[nt] = smem_u32(xsm) + (uint32_t)(tok * H * 2);
+                jc.xs0[nt] = smem_u32(Xs) + (uint32_t)(S.ptok[cur_pf + (q0 < cur_nj ? q0 : 0)] * G * 4);
+                jc.xs1[nt] = smem_u32(Xs) + (uint32_t)(S.ptok[cur_pf + (q1 < cur_nj ? q1 : 0)] * G * 4);
+            }
+        }
+        const int tb = tile_bytes(ug.bits), qb = d_quarter_bytes(ug.bits);
+        const int ngc = gu_chunks(KG, tb), ndc = d_chunks(nst, qb);
+        // gate/up: split K over the warps, partial sums into shared memory
+        float gacc[2][NT][4];
+#pragma unroll
+        for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) gacc[rb][nt][0] = gacc[rb][nt][1] = gacc[rb][nt][2] = gacc[rb][nt][3] = 0.f;
+        for (int ch = 0; ch < ngc; ++ch) {
+            wait_full();
+            if (!bad) {
+                int t0, t1;
+                split_range(2 * KG, ngc, ch, t0, t1);
+                const uint8_t *stg = ring + (size_t)s * kStageBytes;
+                if (ug.bits == 4) gu_chunk<4, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+                else if (ug.bits == 6) gu_chunk<6, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+                else gu_chunk<8, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+            }
+            release_stage();
+        }
+        if (!bad) {
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) red_shared_f32(gred + ((rb * NT + nt) * 4 + i) * 32 + lane, gacc[rb][nt][i]);
+        }
+        if (consumer_sync_or<CW>(bad || S.abort)) {
+            aborted = true;
+            break;
+        }
+        // SiLU-GLU of the unit's 16 rows, one warp per n-tile: h(row 8 rb + g, pair 2t + col)
+        if (warp < NT) {
+            const int nt = warp;
+            float xs0 = 0.f, xs1 = 0.f;
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+                float v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float *p = gred + ((rb * NT + nt) * 4 + i) * 32 + lane;
+                    v[i] = *p;
+                    *p = 0.f;
+                }
+#pragma unroll
+                for (int col = 0; col < 2; ++col) {
+                    const float gt = v[col], up = v[2 + col];
+                    const float h = __fdividef(gt, 1.f + __expf(-gt)) * up;
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+                    const int o = (nt * 8 + 2 * t + col) * 16 + 8 * rb + g;
+                    hhi[o] = __bfloat16_as_ushort(hi);
+                    hlo[o] = __bfloat16_as_ushort(lo);
+                    const float hs = __bfloat162float(hi) + __bfloat162float(lo);
+                    if (col == 0) xs0 += hs;
+                    else xs1 += hs;
+                }
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                xs0 += __shfl_xor_sync(0xffffffffu, xs0, off);
+                xs1 += __shfl_xor_sync(0xffffffffu, xs1, off);
+            }
+            if (g == 0) {
+                hX[nt * 8 + 2 * t] = xs0;
+                hX[nt * 8 + 2 * t + 1] = xs1;
+            }
+            if (lane < 8) {
+                const int q = nt * 8 + lane;
+                hW[nt * 8 + lane] = q < cur_nj ? S.pw[cur_pf + q] : 0.f;
+            }
+        }
+        consumer_sync<CW>();
+        DnCtx<NT> dc;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const uint32_t o = (uint32_t)(((nt * 8 + g) * 16 + 4 * t) * 2);
+            const uint2 vh = lds64(smem_u32(hhi) + o), vl = lds64(smem_u32(hlo) + o);
+            dc.hb[nt][0] = vh.x;
+            dc.hb[nt][1] = vh.y;
+            dc.lb[nt][0] = vl.x;
+            dc.lb[nt][1] = vl.y;
+            if (ug.bits != 4) {
+                dc.hb16[nt][0] = bf16x2_mul16(vh.x);
+                dc.hb16[nt][1] = bf16x2_mul16(vh.y);
+                dc.lb16[nt][0] = bf16x2_mul16(vl.x);
+                dc.lb16[nt][1] = bf16x2_mul16(vl.y);
+            } else {
+                dc.hb16[nt][0] = dc.hb16[nt][1] = dc.lb16[nt][0] = dc.lb16[nt][1] = 0u;
+            }
+            dc.X0[nt] = hX[nt * 8 + 2 * t];
+            dc.X1[nt] = hX[nt * 8 + 2 * t + 1];
+            dc.w0[nt] = hW[nt * 8 + 2 * t];
+            dc.w1[nt] = hW[nt * 8 + 2 * t + 1];
+        }
+        // down: super-tile st of the unit's quarter goes to warp st % kCW
+        for (int ch = 0; ch < ndc; ++ch) {
+            wait_full();
+            if (!bad) {
+                int s0, s1;
+                split_range(nst, ndc, ch, s0, s1);
+                const uint32_t zb = smem_u32(ring + (size_t)s * kStageBytes), qbase = zb + (uint32_t)((s1 - s0) * 256);
+                if (STW > 0) {
+#pragma unroll
+                    for (int l = 0; l < NL; ++l) {
+                        const int st = warp + l * kCW;
+                        if (st >= s0 && st < s1) {
+                            const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
+                            if (ug.bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[l]);
+                            else if (ug.bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[l]);
+                            else down_st<8, NT>(zp, qp, dc, lane, yacc[l]);
+                        }
+                    }
+                } else {
+                    for (int st = s0 + ((warp - s0) % kCW + kCW) % kCW; st < s1; st += kCW) {
+                        const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
+                        if (ug.bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[0]);
+                        else if (ug.bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[0]);
+                        else down_st<8, NT>(zp, qp, dc, lane, yacc[0]);
+                        if (STW == 0) {
+                            emit_st<NT>(a, S, cur_pf, cur_nj, st, yacc[0], lane);
+                        } else if (t == 0) {
+                            // one token (column 0): this warp owns the super-tile's rows
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                ycta[64 * st + 16 * r + g] += yacc[0][r][0][0];
+                                ycta[64 * st + 16 * r + g + 8] += yacc[0][r][0][2];
+                            }
+                        }
+                        zero_y();
+                    }
+                }
+            }
+            release_stage();
         }
     }
-
+    if (!aborted && consumer_sync_or<CW>(bad || S.abort)) aborted = true;
+    // ---------------------------------------------------------------- output rows
+    if (!aborted && S.u1 > S.u0) {
+        if (STW < 0) {
+            // one token: the CTA's rows, one vector addition per 4 rows
+            consumer_sync<CW>();
+            for (int i = threadIdx.x; i < H / 4; i += kCW * 32)
+                red_add_v4_f32(a.out_acc + 4 * i, *reinterpret_cast<const float4 *>(ycta + 4 * i));
+        } else if (STW > 0) {
+            flush_slot();
+        }
+    }
     // ---------------------------------------------------------------- completion
-    consumer_sync();
-    if (threadIdx.x == 0) {
-        // release (this CTA's additions, ordered before it by the barrier) and acquire (the
-        // other CTAs' additions, for the last CTA) in one step
-        const unsigned long long old = atom_add_acq_rel_u64(&a.ctl->done, 1ull);
-        S.is_last = (old + 1ull == (epoch + 1ull) * (unsigned long long)nC) ? 1 : 0;
-    }
-    consumer_sync();
-    if (S.is_last) {
-        // every CTA's additions are complete: convert, then leave the accumulator and the
-        // readiness counters zero for the next call
-        float4 *acc4 = reinterpret_cast<float4 *>(a.out_acc);
-        uint2 *out4 = reinterpret_cast<uint2 *>(a.out);
-        for (int i = threadIdx.x; i < T * H / 4; i += kCW * 32) {
-            const float4 v = __ldcg(acc4 + i);
-            const __nv_bfloat162 lo2 = __floats2bfloat162_rn(v.x, v.y), hi2 = __floats2bfloat162_rn(v.z, v.w);
-            out4[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&lo2), *reinterpret_cast<const uint32_t *>(&hi2));
-            __stcg(acc4 + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    // Each row group's counter grows by one per CTA and call; the CTA whose addition completes a
+    // call's count converts the group to bf16 and clears it (release of this CTA's additions,
+    // ordered before by the barrier, and acquire of the others', in one step).
+    consumer_sync<CW>();
+    const int ngr = (H + kRowGroup - 1) / kRowGroup;
+    for (int gi = warp; gi < ngr; gi += kCW) {
+        int last = 0;
+        if (lane == 0) {
+            const unsigned long long old = atom_add_acq_rel_u64(a.rowcnt + gi, 1ull);
+            last = ((old + 1ull) % (unsigned long long)nC) == 0ull ? 1 : 0;
         }
-        for (int i = threadIdx.x; i < kMaxP; i += kCW * 32) a.h_ready[i] = 0u;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        __syncwarp();
+        if (last) {
+            const int r0 = gi * kRowGroup, n4 = (min(H, r0 + kRowGroup) - r0) / 4;
+            for (int i = lane; i < T * n4; i += 32) {
+                const int tt = i / n4, c4 = i - tt * n4;
+                float4 *p = reinterpret_cast<float4 *>(a.out_acc + (size_t)tt * H + r0) + c4;
+                const float4 v = __ldcg(p);
+                const __nv_bfloat162 lo2 = __floats2bfloat162_rn(v.x, v.y), hi2 = __floats2bfloat162_rn(v.z, v.w);
+                reinterpret_cast<uint2 *>(a.out + (size_t)tt * H + r0)[c4] =
+                    make_uint2(*reinterpret_cast<const uint32_t *>(&lo2), *reinterpret_cast<const uint32_t *>(&hi2));
+                __stcg(p, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+        }
     }
+    if (threadIdx.x == 0) atomicAdd(&a.ctl->done, 1ull);
 }
 
 // Copies of the exchanged logit words within the fixed logit region (kMaxT x kMaxE words): the
@@ -1337,22 +1152,24 @@ void logit_copies(int T, int E, int &rep, int &stride) {
     while (rep < 32 && (size_t)(rep * 2) * stride <= (size_t)kMaxT * kMaxE) rep *= 2;
 }
 
-template <int NT>
+template <int NT, int STW, int CW>
 moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t st) {
     const DecodeLayout L = decode_layout<NT>(a.T, a.H, dev->max_smem_optin);
     if (L.stages < 2) return MOE_ERR_UNSUPPORTED;
-    static bool attr_set[64] = {false};
+    // the kernel attribute, once per device (concurrent first calls from several host threads
+    // set the same value; the flag is atomic)
+    static std::atomic<bool> attr_set[64];
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return MOE_ERR_CUDA;
-    if (!attr_set[d]) {
-        if (cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!attr_set[d].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(decode_kernel<NT, STW, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dev->max_smem_optin) != cudaSuccess)
             return MOE_ERR_CUDA;
-        attr_set[d] = true;
+        attr_set[d].store(true, std::memory_order_release);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dev->sms);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3((CW + 1) * 32);
     cfg.dynamicSmemBytes = L.total;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -1360,7 +1177,7 @@ moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_kernel<NT>, a, L) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<NT, STW, CW>, a, L) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
@@ -1369,8 +1186,7 @@ moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t 
 moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias, const void *packed,
                            int T, int H, int I, int E, int k, uint16_t *out, int32_t *idx_out,
                            float *w_out, void *ws, cudaStream_t st) {
-    // (I bound: the per-group sums of one expert's h must fit the activation region)
-    if (T * k > kMaxP || T > kMaxT || H > kDecodeMaxH || I > 16384) return MOE_ERR_UNSUPPORTED;
+    if (T * k > kMaxP || T > kMaxT || H > kDecodeMaxH) return MOE_ERR_UNSUPPORTED;
     const DeviceInfo *dev = device_info();
     if (!dev) return MOE_ERR_CUDA;
     const DecodeWs W = decode_ws_layout(T, H, I, E, k);
@@ -1381,26 +1197,17 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     a.out = out; a.idx_out = idx_out; a.w_out = w_out;
     a.ctl = reinterpret_cast<Control *>(w8);
     a.logits = reinterpret_cast<unsigned long long *>(w8 + W.logits);
-    a.h_ready = reinterpret_cast<uint32_t *>(w8 + W.h_ready);
+    a.rowcnt = reinterpret_cast<unsigned long long *>(w8 + W.rowcnt);
     a.out_acc = reinterpret_cast<float *>(w8 + W.out_acc);
-    a.h_hi = reinterpret_cast<uint16_t *>(w8 + W.h_hi);
-    a.h_lo = reinterpret_cast<uint16_t *>(w8 + W.h_lo);
     a.wait_ns = wait_limit_ns();
-    a.rnC = 1.0 / (double)dev->sms;
-    {
-        // Granlund-Montgomery constants for division by the number of CTAs
-        const uint32_t d = (uint32_t)dev->sms;
-        uint32_t l = 0;
-        while ((1ull << l) < d) ++l;   // ceil(log2 d)
-        a.cm = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1ull);
-        a.cs1 = l < 1 ? l : 1u;
-        a.cs2 = l > 0 ? l - 1u : 0u;
-    }
     a.kmul = (uint32_t)((65536 + k - 1) / k);
     logit_copies(T, E, a.lrep, a.lstride);
-    if (T <= 8) return launch_nt<1>(a, dev, st);
-    if (T <= 16) return launch_nt<2>(a, dev, st);
-    return launch_nt<4>(a, dev, st);
+    // One token: 16 consumer warps, the CTA's output rows in shared memory. Several tokens: every
+    // super-tile's rows are added into the output at once.
+    if (T == 1) return launch_nt<1, -1, 16>(a, dev, st);
+    if (T <= 8) return launch_nt<1, 0, 16>(a, dev, st);
+    if (T <= 16) return launch_nt<2, 0, 16>(a, dev, st);
+    return launch_nt<4, 0, 8>(a, dev, st);
 }
 
 }  // namespace moe

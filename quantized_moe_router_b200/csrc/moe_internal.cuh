@@ -1,21 +1,38 @@
 // moe_internal.cuh -- layouts and device helpers shared by the library's kernels.
 //
 // Packed expert layout (written by moe_pack_layer, read by the decode and prefill kernels).
-// Every matrix is cut into tiles of 16 rows x 64 input columns (one quantisation group):
-//   gate/up ("GU") tiles: rows 0-7 are gate rows 8rb..8rb+7, rows 8-15 the up rows with the
-//       same indices, so one tile holds both projections of eight intermediate rows;
-//       tile (rb, kg) for rb < I/8, kg < H/64, stored rb-major (a row block's K sweep is
-//       contiguous).
-//   down ("D") tiles: rows 16rb..16rb+15 of Wd, tile (rb, kg) for rb < H/16, kg < I/64.
-// A tile is [lo nibble plane 512 B][hi plane: 0 B (4-bit), 256 B (6-bit), 512 B (8-bit)]
-// [scale/zero 64 B]. Lane L of a warp (g = L/4, t = L%4) owns bytes 16L..16L+15 of the lo
-// plane: word j (j = 0..3) holds the eight codes that lane feeds to MMA j as its A operand
-// (rows g and g+8, group columns 16t+4j .. 16t+4j+3), arranged so that shifting the word right
-// by 0, 4, 8, 12 and masking 0x000F000F yields the four bf16x2 operand registers directly.
-// The hi plane holds code >> 4 (8-bit: same nibble arrangement; 6-bit: 2-bit fields, 16 per
-// word, pair s of word m at bits 2s and 16+2s feeding MMA 2m + s/4, register s%4).
-// The scale/zero block is 8 entries of 8 bytes: entry g = {s(row g), z(row g), s(row g+8),
-// z(row g+8)} as fp16.
+// An expert is its gate/up part followed by its down part.
+//
+// Gate/up ("GU") tiles: 16 rows x 64 input columns (one quantisation group); rows 0-7 are gate
+// rows 8rb..8rb+7, rows 8-15 the up rows with the same indices, so one tile holds both
+// projections of eight intermediate rows; tile (rb, kg) for rb < I/8, kg < H/64, stored rb-major
+// (a row block's K sweep is contiguous). A tile is [lo nibble plane 512 B][hi plane: 0 B
+// (4-bit), 256 B (6-bit), 512 B (8-bit)][scale/zero 64 B]. Lane L of a warp (g = L/4, t = L%4)
+// owns bytes 16L..16L+15 of the lo plane: word j (j = 0..3) holds the eight codes that lane feeds
+// to MMA j as its A operand (rows g and g+8, group columns 16t+4j .. 16t+4j+3), arranged so that
+// shifting the word right by 0, 4, 8, 12 and masking 0x000F000F yields the four bf16x2 operand
+// registers directly (column c+0 in bits 0/4, c+1 in 16/20, c+2 in 8/12, c+3 in 24/28; row g in
+// the lower nibble of each pair). The hi plane holds code >> 4 (8-bit: the same nibble
+// arrangement; 6-bit: 2-bit fields, 16 per word, pair s of word m at bits 2s and 16+2s feeding
+// MMA 2m + s/4, register s%4). The scale/zero block is 8 entries of 8 bytes: entry g =
+// {s(row g), z(row g), s(row g+8), z(row g+8)} as fp16.
+//
+// Down ("D") part: Wd [H x I] in blocks of one group column kg (64 input columns), block kg at
+// kg * (H/16) * tile_bytes. Rows are taken in super-tiles of 64 (four 16-row blocks r = 0..3) and
+// the group's 64 columns in four quarters of 16 (quarter q = columns 16q..16q+15), so that the
+// 16 columns of one quarter are contiguous for all H rows:
+//   [scale/zero: H/64 super-tiles x 256 B: super-tile st, block r, entry g (8 B) =
+//                {s, z of row 64st+16r+g, s, z of row 64st+16r+g+8}]
+//   [quarter 0][quarter 1][quarter 2][quarter 3], each H/64 super-tiles x qbytes(bits), where a
+//   super-tile's quarter is [lo: 4 blocks r x 32 lanes x 4 B][hi: 8-bit 4 x 32 x 4 B,
+//   6-bit 4 x 32 x 2 B]. Word (r, lane g,t) of quarter q holds rows 64st+16r+g and +8, columns
+//   16q + 4t + {0,1,2,3} in the nibble arrangement above, i.e. it is word j = t of lane (g, q) of
+//   the 16x64 tile of those rows; its 6-bit hi half-word holds the two bytes of that tile's 6-bit
+//   hi plane that feed MMA j = t (bits 8(j%2).. and 16+8(j%2).. of word j/2) as its low and high
+//   byte.
+// One quarter across all rows is therefore the down half of a decode work unit (16 intermediate
+// rows), and the four 16-byte pieces {r, lanes 4g..4g+3} of the four quarters are exactly lane
+// (g, t)'s 16 lo bytes of the 16x64 tile, which is how prefill reads them.
 // Packed layer = header (32 B) + E expert entries (16 B) + expert data (256-B aligned).
 #pragma once
 #include <cstdint>
@@ -31,7 +48,7 @@ constexpr int kGroup = 64;
 constexpr int kLoBytes = 512;
 constexpr int kSzBytes = 64;
 constexpr uint32_t kPackedMagic = 0x50454F4Du;  // "MOEP"
-constexpr uint32_t kPackedVersion = 1;
+constexpr uint32_t kPackedVersion = 2;
 constexpr int kMaxT = 32;                       // decode token limit
 constexpr int kMaxK = 32;
 constexpr int kMaxE = 1024;
@@ -59,6 +76,13 @@ __host__ __device__ inline size_t d_tiles(int H, int I) { return (size_t)(H / 16
 __host__ __device__ inline size_t expert_bytes(int H, int I, int bits) {
     return (gu_tiles(H, I) + d_tiles(H, I)) * tile_bytes(bits);
 }
+// down part: bytes of one group-column block, of one super-tile's quarter, and the offset of
+// quarter q within a block
+__host__ __device__ inline size_t d_block_bytes(int H, int bits) { return (size_t)(H / 16) * tile_bytes(bits); }
+__host__ __device__ constexpr int d_quarter_bytes(int bits) { return kLoBytes + hi_bytes(bits); }
+__host__ __device__ inline size_t d_quarter_offset(int H, int bits, int q) {
+    return (size_t)4 * H + (size_t)q * (H / 64) * d_quarter_bytes(bits);
+}
 __host__ __device__ inline size_t packed_data_start(int E) {
     return align_up(sizeof(PackedHeader) + (size_t)E * sizeof(PackedExpert), 256);
 }
@@ -75,28 +99,29 @@ constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusCheck = 2u;
 constexpr int kDecodeMaxP = 256;   // decode limit on T*k
 
-// Decode workspace, fixed regions first so that one workspace can serve decode calls of any
-// shape: logits, kMaxT x kMaxE 8-byte words {fp32 logit bits (low word), call tag (high word)}
-// (a call writes entry t * E + e of each of its copies of the T x E block); h_ready, finished gate/up row blocks per selected expert;
-// out_acc, fp32 [T x H] (up to kMaxT x kDecodeMaxH); then h_hi / h_lo, bf16 h of every
-// (token, slot) pair [T*k x I]. h_ready and out_acc are zero between calls: the last CTA of
-// every call clears what the call used.
+// Decode workspace, fixed regions only, so that one workspace serves decode calls of any shape:
+// logits, kMaxT x kMaxE 8-byte words {fp32 logit bits (low word), call tag (high word)} (a call
+// writes entry t * E + e of each of its copies of the T x E block); rowcnt, one 64-bit counter per
+// 256 output rows (kDecodeMaxH / 256), each grown by every CTA once per call, so that the CTA that
+// completes a row group converts it; out_acc, fp32 [T x H] (up to kMaxT x kDecodeMaxH), zero
+// between calls (each row group is cleared by the CTA that converts it).
 constexpr int kDecodeMaxH = 8192;
+constexpr int kRowGroup = 256;
 struct DecodeWs {
-    size_t logits, h_ready, out_acc, h_hi, h_lo, total;
+    size_t logits, rowcnt, out_acc, total;
 };
 inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
+    (void)T;
     (void)H;
+    (void)I;
     (void)E;
+    (void)k;
     DecodeWs w;
     size_t o = 256;
     auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
-    const size_t P = (size_t)T * k;
     w.logits = take((size_t)kMaxT * kMaxE * 8);
-    w.h_ready = take((size_t)kDecodeMaxP * 4);
+    w.rowcnt = take((size_t)(kDecodeMaxH / kRowGroup) * 8);
     w.out_acc = take((size_t)kMaxT * kDecodeMaxH * 4);
-    w.h_hi = take(P * I * 2);
-    w.h_lo = take(P * I * 2);
     w.total = o;
     return w;
 }

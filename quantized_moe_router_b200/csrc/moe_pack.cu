@@ -1,7 +1,9 @@
 // moe_pack.cu -- canonical expert tensors -> the packed tile layout of moe_internal.cuh.
 //
 // A pure byte/bit permutation (no value is rounded): each thread builds one lane's share of one
-// tile -- its 16 lo-plane bytes, its hi-plane bytes and (for t == 0) its scale/zero entry.
+// 16x64 tile -- its 16 lo-plane bytes, its hi-plane bytes and (for t == 0) its scale/zero entry --
+// and stores it at the tile's place (gate/up) or scatters it over the four quarters of its
+// super-tile (down).
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -48,7 +50,6 @@ __global__ void pack_expert_kernel(PackSrc src, int H, int I, uint8_t *dst, long
         kg = (int)(dt % GI);
         mA = 2; mB = 2; rowA = rb * 16 + g; rowB = rb * 16 + g + 8; cols = I;
     }
-    uint8_t *tp = dst + tile * tile_bytes(BITS);
     uint32_t lo[4], hi8[4], hi6[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -77,15 +78,37 @@ __global__ void pack_expert_kernel(PackSrc src, int H, int I, uint8_t *dst, long
         lo[j] = wl;
         hi8[j] = wh;
     }
-    *reinterpret_cast<uint4 *>(tp + 16 * lane) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    if (BITS == 8) *reinterpret_cast<uint4 *>(tp + kLoBytes + 16 * lane) = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
-    if (BITS == 6) *reinterpret_cast<uint2 *>(tp + kLoBytes + 8 * lane) = make_uint2(hi6[0], hi6[1]);
+    const int GA = cols / kGroup;
+    uint2 sz = make_uint2(0u, 0u);
     if (t == 0) {
-        const int GA = cols / kGroup;
         const uint32_t sA = src.scale[mA][(size_t)rowA * GA + kg], zA = src.zero[mA][(size_t)rowA * GA + kg];
         const uint32_t sB = src.scale[mB][(size_t)rowB * GA + kg], zB = src.zero[mB][(size_t)rowB * GA + kg];
-        *reinterpret_cast<uint2 *>(tp + kLoBytes + hi_bytes(BITS) + 8 * g) =
-            make_uint2(sA | (zA << 16), sB | (zB << 16));
+        sz = make_uint2(sA | (zA << 16), sB | (zB << 16));
+    }
+    if (tile < ngu) {
+        uint8_t *tp = dst + tile * tile_bytes(BITS);
+        *reinterpret_cast<uint4 *>(tp + 16 * lane) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (BITS == 8) *reinterpret_cast<uint4 *>(tp + kLoBytes + 16 * lane) = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
+        if (BITS == 6) *reinterpret_cast<uint2 *>(tp + kLoBytes + 8 * lane) = make_uint2(hi6[0], hi6[1]);
+        if (t == 0) *reinterpret_cast<uint2 *>(tp + kLoBytes + hi_bytes(BITS) + 8 * g) = sz;
+    } else {
+        // word j of this lane (g, t) is word (r, lane 4g + j) of quarter t of super-tile st
+        const int rb = rowA / 16, st = rb >> 2, r = rb & 3;
+        uint8_t *blk = dst + (size_t)ngu * tile_bytes(BITS) + (size_t)kg * d_block_bytes(H, BITS);
+        uint8_t *qp = blk + d_quarter_offset(H, BITS, t) + (size_t)st * d_quarter_bytes(BITS);
+        *reinterpret_cast<uint4 *>(qp + r * 128 + 16 * g) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (BITS == 8) *reinterpret_cast<uint4 *>(qp + kLoBytes + r * 128 + 16 * g) = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
+        if (BITS == 6) {
+            // MMA j's two bytes of hi word j/2 (bits 8(j%2).. and 16+8(j%2)..) as one half-word
+            uint32_t h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t w = hi6[j >> 1] >> (8 * (j & 1));
+                h[j] = (w & 0xFFu) | ((w >> 8) & 0xFF00u);
+            }
+            *reinterpret_cast<uint2 *>(qp + kLoBytes + r * 64 + 8 * g) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+        }
+        if (t == 0) *reinterpret_cast<uint2 *>(blk + (size_t)st * 256 + r * 64 + 8 * g) = sz;
     }
 }
 

@@ -212,15 +212,18 @@ __device__ __forceinline__ uint32_t fma2_h_hi(float x0, float x1, float y0, floa
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one packed tile (its image in
-// shared memory at `rawt`), stored as fp16 into the swizzled A tile rows 16b+g and 16b+g+8.
-// Word j of the lo plane holds columns 16t+4j+{0,1,2,3} in bytes {0,2,1,3}: row g in the low
+// The 16 values of row g (cols 16t .. 16t+15) and of row g+8 of one 16x64 tile, stored as fp16
+// into the swizzled A tile rows 16b+g and 16b+g+8. lo16: the lane's 16 lo-plane bytes; hip: its
+// hi-plane bytes (8-bit: 16 bytes in the lo arrangement; 6-bit: the tile's two hi words, or, with
+// DQ, the four half-words of the down layout, one per MMA); szp: its scale/zero entry (8 bytes).
+// Word j of the lo bytes holds columns 16t+4j+{0,1,2,3} in bytes {0,2,1,3}: row g in the low
 // nibbles, row g+8 in the high nibbles.
-template <int BITS>
-__device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uint8_t *As, int b) {
+template <int BITS, bool DQ>
+__device__ __forceinline__ void dequant_fragment(const uint8_t *lo16, const uint8_t *hip, const uint8_t *szp, int L,
+                                                 uint8_t *As, int b) {
     const int g = L >> 2, t = L & 3;
-    const uint4 lo = *reinterpret_cast<const uint4 *>(rawt + 16 * L);
-    const uint2 sz = *reinterpret_cast<const uint2 *>(rawt + kLoBytes + hi_bytes(BITS) + 8 * g);
+    const uint4 lo = *reinterpret_cast<const uint4 *>(lo16);
+    const uint2 sz = *reinterpret_cast<const uint2 *>(szp);
     const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
     const uint32_t w[4] = {lo.x, lo.y, lo.z, lo.w};
     uint32_t ra[8], rb[8];
@@ -237,7 +240,7 @@ __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uin
         }
     } else if (BITS == 8) {
         // q = lo + 16 hi, the hi plane in the same nibble arrangement
-        const uint4 hi = *reinterpret_cast<const uint4 *>(rawt + 512 + 16 * L);
+        const uint4 hi = *reinterpret_cast<const uint4 *>(hip);
         const uint32_t v[4] = {hi.x, hi.y, hi.z, hi.w};
         const float SA = 256.f * sA, SA2 = 4096.f * sA, CA = -(128.f + 2048.f + zA) * sA;
         const float SB = 2048.f * sB, SB2 = 32768.f * sB, CB = -(2048.f + 32768.f + zB) * sB;
@@ -257,7 +260,12 @@ __device__ __forceinline__ void dequant_fragment(const uint8_t *rawt, int L, uin
     } else {
         // 6-bit: q = lo + 16 hi, hi in 2-bit fields (word j/2, pair s = 4(j&1) + r at bits 2s and
         // 16 + 2s; r = 0: row g cols +0/+1, 1: row g+8 cols +0/+1, 2: row g +2/+3, 3: row g+8 +2/+3)
-        const uint2 hi = *reinterpret_cast<const uint2 *>(rawt + 512 + 8 * L);
+        uint2 hi = *reinterpret_cast<const uint2 *>(hip);
+        if (DQ) {
+            // half-words {MMA 0, 1} and {MMA 2, 3} -> the tile's hi words (bytes lo0 lo1 hi0 hi1)
+            hi.x = __byte_perm(hi.x, 0u, 0x3120);
+            hi.y = __byte_perm(hi.y, 0u, 0x3120);
+        }
         const float SA = 256.f * sA, SA2 = 16.f * sA, CA = -(128.f + zA) * sA;
         const float SB = 2048.f * sB, SB2 = 16.f * sB, CB = -(2048.f + zB) * sB;
 #pragma unroll
@@ -397,17 +405,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 uint8_t *As = ring + (size_t)slot * stage_bytes;
-                const uint8_t *rawt0 = raw + (size_t)rs * slot_bytes + (size_t)(b0 * KC + jk) * tb;
-                const uint8_t *rawt1 = raw + (size_t)rs * slot_bytes + (size_t)(b1 * KC + jk) * tb;
+                // the lane's lo / hi / scale-zero bytes of row block b of this K step: gate/up
+                // slots hold [row block][K chunk] tiles; down slots hold per K step the scale/zero
+                // entries of the unit's super-tiles and its four quarters
+                auto frag = [&](int b, const uint8_t *&lo16, const uint8_t *&hip, const uint8_t *&szp) {
+                    if (GU) {
+                        const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + jk) * tb;
+                        lo16 = rawt + 16 * lane;
+                        hip = rawt + kLoBytes + (bits == 8 ? 16 : 8) * lane;
+                        szp = rawt + kLoBytes + hi_bytes(bits) + 8 * (lane >> 2);
+                    } else {
+                        const int qb = d_quarter_bytes(bits), g = lane >> 2, t = lane & 3;
+                        const uint8_t *base = raw + (size_t)rs * slot_bytes + (size_t)jk * 8 * tb;
+                        const uint8_t *qp = base + 512 + (size_t)t * 2 * qb + (size_t)(b >> 2) * qb;
+                        lo16 = qp + (b & 3) * 128 + 16 * g;
+                        hip = qp + kLoBytes + (b & 3) * (bits == 8 ? 128 : 64) + (bits == 8 ? 16 : 8) * g;
+                        szp = base + (b >> 2) * 256 + (b & 3) * 64 + 8 * g;
+                    }
+                };
+                const uint8_t *l0, *h0, *z0, *l1, *h1, *z1;
+                frag(b0, l0, h0, z0);
+                frag(b1, l1, h1, z1);
                 if (have0 && have1 && bits == 4) {
-                    dequant_fragment<4>(rawt0, lane, As, b0);
-                    dequant_fragment<4>(rawt1, lane, As, b1);
+                    dequant_fragment<4, !GU>(l0, h0, z0, lane, As, b0);
+                    dequant_fragment<4, !GU>(l1, h1, z1, lane, As, b1);
                 } else {
 #pragma unroll 1
                     for (int bb = 0; bb < 2; ++bb) {
                         const int b = bb ? b1 : b0;
                         const bool have = bb ? have1 : have0;
-                        const uint8_t *rawt = bb ? rawt1 : rawt0;
+                        const uint8_t *lo16 = bb ? l1 : l0, *hip = bb ? h1 : h0, *szp = bb ? z1 : z0;
                         if (!have) {
                             const uint4 z = make_uint4(0, 0, 0, 0);
                             const int g = lane >> 2, t = lane & 3;
@@ -416,11 +443,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                             *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t)) = z;
                             *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g + 8, 2 * t + 1)) = z;
                         } else if (bits == 4) {
-                            dequant_fragment<4>(rawt, lane, As, b);
+                            dequant_fragment<4, !GU>(lo16, hip, szp, lane, As, b);
                         } else if (bits == 8) {
-                            dequant_fragment<8>(rawt, lane, As, b);
+                            dequant_fragment<8, !GU>(lo16, hip, szp, lane, As, b);
                         } else {
-                            dequant_fragment<6>(rawt, lane, As, b);
+                            dequant_fragment<6, !GU>(lo16, hip, szp, lane, As, b);
                         }
                     }
                 }
@@ -534,9 +561,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     }
                     const uint32_t fb = smem_u32(&S.raw_full[rs]);
                     mbar_expect_tx(fb, (uint32_t)(nb * KC * tb));
-                    for (int b = 0; b < nb; ++b)
-                        bulk_g2s(smem_u32(raw + (size_t)rs * slot_bytes + (size_t)b * KC * tb),
-                                 mat + ((size_t)(8 * U.mt + b) * G.KG + k0) * tb, (uint32_t)(KC * tb), fb);
+                    uint8_t *slot = raw + (size_t)rs * slot_bytes;
+                    if (GU) {
+                        for (int b = 0; b < nb; ++b)
+                            bulk_g2s(smem_u32(slot + (size_t)b * KC * tb),
+                                     mat + ((size_t)(8 * U.mt + b) * G.KG + k0) * tb, (uint32_t)(KC * tb), fb);
+                    } else {
+                        // per K step: the scale/zero entries of the unit's super-tiles, then its
+                        // piece of each quarter (nb / 4 super-tiles from super-tile 2 * mt)
+                        const int nst = nb / 4, qb = d_quarter_bytes(ex.bits);
+                        for (int kk = 0; kk < KC; ++kk) {
+                            const uint8_t *blk = mat + (size_t)(k0 + kk) * d_block_bytes(a.H, ex.bits);
+                            uint8_t *dstk = slot + (size_t)kk * 8 * tb;
+                            bulk_g2s(smem_u32(dstk), blk + (size_t)2 * U.mt * 256, (uint32_t)(nst * 256), fb);
+                            for (int q = 0; q < 4; ++q)
+                                bulk_g2s(smem_u32(dstk + 512 + (size_t)q * 2 * qb),
+                                         blk + d_quarter_offset(a.H, ex.bits, q) + (size_t)2 * U.mt * qb,
+                                         (uint32_t)(nst * qb), fb);
+                        }
+                    }
                 }
             }
             // copies still in flight land before the CTA may exit

@@ -24,7 +24,7 @@ vp, i32 = C.c_void_p, C.c_int
 
 # packed format (documented with moe_pack_layer): 32-byte header, 16-byte entries, 256-byte aligned
 # expert blocks of 16 x 64 tiles of 576 / 832 / 1088 bytes for 4 / 6 / 8-bit codes
-MAGIC, VERSION = 0x50454F4D, 1
+MAGIC, VERSION = 0x50454F4D, 2
 TILE = {4: 576, 6: 832, 8: 1088}
 
 

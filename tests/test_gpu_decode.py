@@ -46,6 +46,20 @@ def test_decode_hand_layers(T, E, H, I, k, widths):
     check_block(oracle.get(), x, layer.wr_np, layer.bias_np, layer.expert_fn, E, H, I, k, out, idx, w)
 
 
+@pytest.mark.parametrize("T,E,H,I,k,widths", [
+    (1, 24, 256, 512, 8, [4, 6, 8]),      # one token, per-expert widths: work cut by bytes
+    (1, 16, 8192, 128, 8, [4, 6, 8]),     # the largest H: 128 row super-tiles, 5 gate/up chunks per unit
+    (1, 1024, 256, 64, 32, [4]),          # the largest E and k: wide top-k, 32 slots of 4 units
+    (16, 48, 2048, 192, 8, [6, 8, 4]),    # several tokens with shared experts, mixed widths
+    (1, 6, 4096, 64, 6, [8])])            # few units (24) over all CTAs, all 8-bit
+def test_decode_unit_cuts_and_limits(T, E, H, I, k, widths):
+    rng = np.random.default_rng(T * 7 + E + H)
+    layer = hand_layer(rng, E, H, I, widths)
+    x = synth.to_bf16_bits(rng.normal(0, 1, (T, H)))
+    out, idx, w = decode_call(layer, x, I, E, k)
+    check_block(oracle.get(), x, layer.wr_np, layer.bias_np, layer.expert_fn, E, H, I, k, out, idx, w)
+
+
 def test_decode_workspace_reuse_and_zero_expert():
     rng = np.random.default_rng(5)
     E, H, I, T, k = 6, 128, 64, 4, 2
