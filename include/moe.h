@@ -253,26 +253,33 @@ moe_status_t moe_expert_forward_decode(const uint16_t *x, const float *w_router,
                                        moe_stream_t stream);
 
 /* Decode path without a caller workspace. Same computation, arguments, limits and results as
- * moe_expert_forward_decode, but the scratch memory lives in a fixed 4 MiB array inside this
+ * moe_expert_forward_decode, but the scratch memory lives in a fixed 2 MiB array inside this
  * library's device memory, so the caller passes only inputs and outputs and nothing is
  * allocated. The pages describe no such entry point; it exists for callers that cannot call
  * cudaMalloc: for example an operator plugin that a host runtime hands only its input and
  * output buffers, or a process whose device memory is owned by another allocator.
- *  - Shapes whose decode workspace (moe_workspace_bytes(..., MOE_MODE_DECODE)) exceeds 4 MiB
- *    are rejected with MOE_ERR_UNSUPPORTED before anything is launched.
+ *  - Arguments are checked on the host exactly as for moe_expert_forward_decode, before the
+ *    device is touched; shapes whose decode workspace (moe_workspace_bytes(..., MOE_MODE_DECODE))
+ *    would exceed 2 MiB are rejected with MOE_ERR_UNSUPPORTED before anything is launched (the
+ *    decode workspace has fixed regions, so every supported decode shape fits today).
  *  - The first call on a device looks up the array's device address (once per device, with
  *    that device current); make that first call before any stream capture.
  *  - Every call on a device shares the one array, which keeps the previous call's contents
  *    (the kernel clears what must start at zero itself). Calls whose executions overlap on the
  *    GPU (other streams, other host threads) race on it: order them.
- *  - Every GPU that loads the library holds the 4 MiB until the process exits.
- *  - A device-side wait that expires leaves `out` undefined; its status word is in the array
- *    and cannot be read through moe_get_device_status. */
+ *  - Every GPU that loads the library holds the 2 MiB until the process exits.
+ *  - A device-side wait that expires leaves `out` undefined and sets the array's status word;
+ *    read (and clear) it with moe_noalloc_get_device_status. */
 moe_status_t moe_expert_forward_decode_noalloc(const uint16_t *x, const float *w_router,
                                                const float *bias, const void *packed, int T,
                                                int H, int I, int E, int k, uint16_t *out,
                                                int32_t *idx_out, float *w_out,
                                                moe_stream_t stream);
+
+/* moe_get_device_status for the fixed array of moe_expert_forward_decode_noalloc on the current
+ * device: synchronises `stream`, returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK and
+ * clears a non-zero status word. Allocates nothing. */
+moe_status_t moe_noalloc_get_device_status(moe_stream_t stream);
 
 /* Prefill path, any T >= 1: routing, bucketing of the T*k (token, expert) pairs per expert
  * (stable: ascending token within an expert), a grouped gate/up GEMM with a SiLU-GLU

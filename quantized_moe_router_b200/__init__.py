@@ -32,6 +32,7 @@ SIGNATURES = {
     "moe_expert_forward_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_forward_prefill": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_forward_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_noalloc_get_device_status": (_i, [_vp]),
     "moe_prefill_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "moe_prefill_experts": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
@@ -366,6 +367,12 @@ def forward_decode_noalloc(x, w_router, bias, packed, I, E, k, out=None, idx_out
                                                    _p(out), _p(idx_out), _p(w_out), _stream(stream)),
            "moe_expert_forward_decode_noalloc")
     return out
+
+
+def noalloc_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the status of the fixed scratch array
+    that forward_decode_noalloc uses on the current device."""
+    return lib().moe_noalloc_get_device_status(_stream(stream))
 
 
 def device_status(ws: torch.Tensor, stream=None) -> int:

@@ -73,26 +73,52 @@ bool shape_ok(int T, int H, int I, int E, int k) {
 
 bool packed_ok(const void *packed) { return packed && aligned(packed, 256); }
 
+// Host-side checks shared by the forward entry points (everything but the workspace).
+moe_status_t block_args_ok(const uint16_t *x, const float *w_router, const float *bias, const void *packed, int T,
+                           int H, int I, int E, int k, uint16_t *out, int32_t *idx_out, float *w_out) {
+    if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
+    if (!x || !w_router || !out || !packed_ok(packed)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
+    if ((idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
 moe_status_t forward_common(const uint16_t *x, const float *w_router, const float *bias, const void *packed, int T,
                             int H, int I, int E, int k, uint16_t *out, int32_t *idx_out, float *w_out, void *ws,
                             size_t ws_bytes, int mode) {
-    if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
-    if (!x || !w_router || !out || !ws || !packed_ok(packed)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ws, 256) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
-    if (bias && !aligned(bias, 4)) return MOE_ERR_INVALID_ARG;
-    if ((idx_out && !aligned(idx_out, 4)) || (w_out && !aligned(w_out, 4))) return MOE_ERR_INVALID_ARG;
+    const moe_status_t s = block_args_ok(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out);
+    if (s != MOE_OK) return s;
+    if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < moe_workspace_bytes(T, H, I, E, k, mode)) return MOE_ERR_INVALID_ARG;
     return check_device();
 }
 
+bool decode_shape_supported(int T, int H, int k) { return T <= kMaxT && (long long)T * k <= kDecodeMaxP && H <= kDecodeMaxH; }
+
 // Scratch of moe_expert_forward_decode_noalloc: a fixed array in the library's own device memory,
 // zero-initialised when the library is loaded on a device and kept (with the last call's
 // contents) until the process exits. Host code may not use the array's name as an address; the
-// entry point resolves the device address once per device with cudaGetSymbolAddress.
-constexpr size_t kNoAllocScratchBytes = 4u << 20;   // 4 MiB
+// device address is resolved once per device, with that device current, by cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = 2u << 20;   // 2 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 std::mutex g_noalloc_mu;
 void *g_noalloc_addr[64] = {nullptr};
+
+// The array's device address on the current device (the set-up of the first call per device).
+moe_status_t noalloc_scratch(void **addr) {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return MOE_ERR_CUDA;
+    if (d < 0 || d >= 64) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[d]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        g_noalloc_addr[d] = p;
+    }
+    *addr = g_noalloc_addr[d];
+    return MOE_OK;
+}
 
 }  // namespace
 
@@ -195,32 +221,34 @@ moe_status_t moe_expert_forward_decode(const uint16_t *x, const float *w_router,
     moe_status_t s = forward_common(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, ws, ws_bytes,
                                     MOE_MODE_DECODE);
     if (s != MOE_OK) return s;
-    if (T > kMaxT || (long long)T * k > 256 || H > 8192) return MOE_ERR_UNSUPPORTED;
+    if (!decode_shape_supported(T, H, k)) return MOE_ERR_UNSUPPORTED;
     return launch_decode(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, ws, (cudaStream_t)stream);
 }
 
 moe_status_t moe_expert_forward_decode_noalloc(const uint16_t *x, const float *w_router, const float *bias,
                                                const void *packed, int T, int H, int I, int E, int k, uint16_t *out,
                                                int32_t *idx_out, float *w_out, moe_stream_t stream) {
-    const size_t need = moe_workspace_bytes(T, H, I, E, k, MOE_MODE_DECODE);
-    if (need == 0) return MOE_ERR_INVALID_ARG;
-    if (need > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess) return MOE_ERR_CUDA;
-    if (d < 0 || d >= 64) return MOE_ERR_UNSUPPORTED;
+    // the same host-side checks as moe_expert_forward_decode, before the device is touched
+    moe_status_t s = block_args_ok(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out);
+    if (s != MOE_OK) return s;
+    if (!decode_shape_supported(T, H, k)) return MOE_ERR_UNSUPPORTED;
+    if (moe_workspace_bytes(T, H, I, E, k, MOE_MODE_DECODE) > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+    s = check_device();
+    if (s != MOE_OK) return s;
     void *scratch = nullptr;
-    {
-        // set-up, once per device and with that device current: the array's device address
-        std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_addr[d]) {
-            void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-            g_noalloc_addr[d] = p;
-        }
-        scratch = g_noalloc_addr[d];
-    }
+    s = noalloc_scratch(&scratch);
+    if (s != MOE_OK) return s;
     return moe_expert_forward_decode(x, w_router, bias, packed, T, H, I, E, k, out, idx_out, w_out, scratch,
                                      kNoAllocScratchBytes, stream);
+}
+
+moe_status_t moe_noalloc_get_device_status(moe_stream_t stream) {
+    moe_status_t s = check_device();
+    if (s != MOE_OK) return s;
+    void *scratch = nullptr;
+    s = noalloc_scratch(&scratch);
+    if (s != MOE_OK) return s;
+    return moe_get_device_status(scratch, stream);
 }
 
 moe_status_t moe_expert_forward_prefill(const uint16_t *x, const float *w_router, const float *bias,

@@ -721,6 +721,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     const int ne = (E > c) ? (E - c + nC - 1) / nC : 0;   // router rows of this CTA: c, c+nC, ...
     const bool wr_on = (size_t)ne * H * 4 <= (size_t)NS * kStageBytes;
     const float *wsm = reinterpret_cast<const float *>(ring);
+    const uint64_t drain_ns = a.wait_ns > 1000000ull ? a.wait_ns : 1000000ull;
 
     // ---------------------------------------------------------------- prologue (weights only)
     if (threadIdx.x == 0) {
@@ -896,9 +897,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 ++cc;
             }
         }
-        // copies still in flight land before the CTA may exit
+        // copies still in flight land before the CTA may exit (bounded by at least 1 ms, also when
+        // the wait limit is 0)
         for (uint32_t q = cc > (uint32_t)NS ? cc - NS : 0; q < cc; ++q)
-            mbar_wait(smem_u32(&S.full[q % NS]), (q / NS) & 1u, a.wait_ns, status);
+            mbar_wait(smem_u32(&S.full[q % NS]), (q / NS) & 1u, drain_ns, status);
         return;
     }
 
@@ -1141,7 +1143,13 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             }
         }
     }
-    if (threadIdx.x == 0) atomicAdd(&a.ctl->done, 1ull);
+    if (threadIdx.x == 0) {
+        atomicAdd(&a.ctl->done, 1ull);
+        // the prologue's copies have landed before the CTA exits (they may not have if a wait
+        // for them expired)
+        if (xs_on) mbar_wait(smem_u32(&S.xbar), 0, drain_ns, status);
+        if (wr_on && ne > 0) mbar_wait(smem_u32(&S.wbar), 0, drain_ns, status);
+    }
 }
 
 // Copies of the exchanged logit words within the fixed logit region (kMaxT x kMaxE words): the

@@ -106,6 +106,17 @@ def test_host_validation_before_any_launch(L):
     assert L.moe_prefill_experts(fake, fake, 4, 2000, 512, 256, 8, fake, fake, big, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_workspace_init(None, 1024, None) == qm.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_status(None, None) == qm.MOE_ERR_INVALID_ARG
+    # the allocation-free decode call checks its arguments on the host as the workspace call
+    # does, before it touches the device (so these hold without a GPU as well)
+    nf = L.moe_expert_forward_decode_noalloc
+    assert nf(None, fake, None, fake, 1, 2048, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_INVALID_ARG
+    assert nf(fake + 2, fake, None, fake, 1, 2048, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_INVALID_ARG
+    assert nf(fake, fake, None, fake + 16, 1, 2048, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_INVALID_ARG
+    assert nf(fake, fake, None, fake, 1, 100, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_INVALID_ARG
+    assert nf(fake, fake, None, fake, 33, 2048, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_UNSUPPORTED
+    assert nf(fake, fake, None, fake, 1, 16384, 512, 256, 8, fake, None, None, None) == qm.MOE_ERR_UNSUPPORTED
+    assert L.moe_expert_forward_decode(fake, fake, None, fake, 33, 2048, 512, 256, 8, fake, None, None, fake, 1 << 30,
+                                       None) in (qm.MOE_ERR_UNSUPPORTED, qm.MOE_ERR_CUDA)
 
 
 def test_quantizer_host_validation(L):
