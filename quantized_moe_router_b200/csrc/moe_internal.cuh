@@ -132,7 +132,8 @@ inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
 // largest hexp of each pair; nt_start: N-tile prefix of the experts ([E] = total, [E+1] = the
 // largest N tile, rows rounded to 16).
 struct PrefillWs {
-    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, x16, xexp, h, hexp, fexp, out_acc, total;
+    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, x16, xexp, h, hexp, fexp, out_acc, planes, lg,
+        total;
     int nblk;  // token blocks of the stable scatter
 };
 constexpr int kScatterTokens = 64;
@@ -156,6 +157,8 @@ inline PrefillWs prefill_ws_layout(int T, int H, int I, int E, int k) {
     w.hexp = take(P * (I / 16));
     w.fexp = take(P * 4);
     w.out_acc = take((size_t)T * H * 4);
+    w.planes = take((size_t)3 * E * H * 2);   // router rows as three bf16 planes
+    w.lg = take((size_t)T * E * 4);           // fp32 router logits
     w.total = o;
     return w;
 }

@@ -14,6 +14,9 @@ namespace moe {
 
 moe_status_t launch_route(const uint16_t *x, const float *wr, const float *bias, int T, int H, int E, int k,
                           int32_t *idx_out, float *w_out, cudaStream_t st);
+moe_status_t launch_route_tc(const uint16_t *x, const float *wr, const float *bias, int T, int H, int E, int k,
+                             int32_t *idx_out, float *w_out, uint16_t *planes, float *lg, uint32_t *status,
+                             cudaStream_t st);
 moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I, int E, int k, const int32_t *counts,
                                      const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
                                      const float *pair_w, const uint16_t *x, uint16_t *x16, int32_t *xexp,
@@ -123,7 +126,8 @@ moe_status_t launch_prefill_route(const uint16_t *x, const float *wr, const floa
     int32_t *ptok = reinterpret_cast<int32_t *>(w8 + L.pair_tok);
     float *pw = reinterpret_cast<float *>(w8 + L.pair_w);
     const size_t P = (size_t)T * k;
-    moe_status_t s = launch_route(x, wr, bias, T, H, E, k, idx, wt, st);
+    moe_status_t s = launch_route_tc(x, wr, bias, T, H, E, k, idx, wt, reinterpret_cast<uint16_t *>(w8 + L.planes),
+                                     reinterpret_cast<float *>(w8 + L.lg), &reinterpret_cast<Control *>(w8)->status, st);
     if (s != MOE_OK) return s;
     if (idx_out && cudaMemcpyAsync(idx_out, idx, P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
     if (w_out && cudaMemcpyAsync(w_out, wt, P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -27,10 +27,7 @@
 // fp16 operands (11-bit significands) keep the block within its error bound where bf16
 // operands (8-bit) would not; every scaling is by a power of two and exact.
 // Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "moe_internal.cuh"
+#include "moe_tc.cuh"
 
 namespace moe {
 
@@ -117,46 +114,6 @@ __device__ __forceinline__ Unit unit_at(const TcArgs &a, int u, int mtiles) {
     return U;
 }
 
-// ------------------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    // K-major operand, 128-byte swizzle: 8-row x 128-byte atoms stacked 1024 bytes apart
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFF);
-    d |= (uint64_t)1 << 16;              // leading byte offset (unused with this swizzle)
-    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset: next 8-row atom
-    d |= (uint64_t)1 << 46;              // descriptor version
-    d |= (uint64_t)2 << 61;              // SWIZZLE_128B
-    return d;
-}
-__device__ __forceinline__ uint32_t idesc_f16_f32(int M, int N) {
-    // D fp32 (bits 4-5 = 1), A and B fp16 (format 0), both K-major, N >> 3 at bit 17, M >> 4 at bit 24
-    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // Bounded mbarrier wait that also gives up when another role of the CTA has aborted.
 __device__ __forceinline__ bool tc_wait(TcShared &S, const TcArgs &a, uint64_t *bar, uint32_t parity) {
     const uint32_t b = smem_u32(bar);
@@ -172,9 +129,6 @@ __device__ __forceinline__ bool tc_wait(TcShared &S, const TcArgs &a, uint64_t *
         }
     }
 }
-
-// byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled K-major tile
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
 // 2^e as fp32 for |e| <= 126
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
@@ -788,25 +742,9 @@ __global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, int P, int
     }
 }
 
-// 2-D tensor map of a row-major fp16 matrix [rows x cols] read in boxes of 64 columns (128 bytes,
-// 128-byte swizzle) by kRowBox rows; rows past the matrix read as zeros.
+// 2-D tensor map of a row-major fp16 matrix [rows x cols] read in boxes of 64 columns by kRowBox rows
 bool make_row_map(CUtensorMap *map, const void *base, int rows, int cols) {
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    if (encode == nullptr) {
-        cudaDriverEntryPointQueryResult q;
-        void *fn = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || fn == nullptr)
-            return false;
-        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kGroup, (cuuint32_t)kRowBox};
-    const cuuint32_t estr[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return make_tmap_2d_16(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rows, cols, kRowBox);
 }
 
 template <bool GU>
