@@ -70,7 +70,19 @@ struct DecodeArgs {
     int lstride;                 // words between copies
 };
 
+// Chunking of one work unit for one code width: gate/up tiles and down super-tiles, each cut into
+// nearly equal chunks of at most one ring stage (chunk c of n items: c * base + min(c, rem), with
+// base + 1 items for c < rem), and the byte offsets of an expert's parts.
+struct WidthPlan {
+    int tb, qb;                   // gate/up tile bytes, down super-tile quarter bytes
+    int ngc, gbase, grem;         // gate/up chunks of the unit's 2 * KG tiles
+    int ndc, dbase, drem;         // down chunks of its H / 64 super-tiles
+    uint32_t gu_part, d_block;    // bytes of the expert's gate/up part, of one down group block
+};
+__device__ __forceinline__ int width_index(int bits) { return (bits - 4) >> 1; }
+
 struct __align__(16) DecodeSmem {
+    WidthPlan wplan[3];
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
     uint64_t xbar, wbar;
@@ -470,6 +482,14 @@ __device__ __forceinline__ unsigned long long unit_bytes(const DecodeArgs &a, in
            (unsigned long long)(a.H / 64) * d_quarter_bytes(bits) + 4ull * a.H;
 }
 
+// floor(n / d) for n < 2^53 through the double quotient (within one of the result), corrected
+__device__ __forceinline__ unsigned long long div_floor(unsigned long long n, unsigned long long d) {
+    unsigned long long q = (unsigned long long)((double)n / (double)d);
+    if (q * d > n) --q;
+    if ((q + 1) * d <= n) ++q;
+    return q;
+}
+
 // This CTA's range of work units [u0, u1): units are numbered slot-major (I / 16 per slot); CTA c
 // takes the units whose first byte lies in [c * B / nC, (c + 1) * B / nC) of the B bytes of all.
 __device__ void plan_units(const DecodeArgs &a, DecodeSmem &S, int lane, int c, int nC) {
@@ -503,10 +523,10 @@ __device__ void plan_units(const DecodeArgs &a, DecodeSmem &S, int lane, int c, 
             }
         }
         const unsigned long long ub = unit_bytes(a, S.ubits[jj]);
-        return jj * sp + (int)((pos - S.ccost[jj] + ub - 1) / ub);
+        return jj * sp + (int)div_floor(pos - S.ccost[jj] + ub - 1, ub);
     };
-    const int u0 = unit_at(B * (unsigned long long)c / (unsigned long long)nC);
-    const int u1 = (c + 1 >= nC) ? U * sp : unit_at(B * (unsigned long long)(c + 1) / (unsigned long long)nC);
+    const int u0 = unit_at(div_floor(B * (unsigned long long)c, (unsigned long long)nC));
+    const int u1 = (c + 1 >= nC) ? U * sp : unit_at(div_floor(B * (unsigned long long)(c + 1), (unsigned long long)nC));
     if (lane == 0) {
         S.u0 = u0;
         S.u1 = u1;
@@ -515,38 +535,38 @@ __device__ void plan_units(const DecodeArgs &a, DecodeSmem &S, int lane, int c, 
 }
 
 // ------------------------------------------------------------------------------ work units
+__device__ __forceinline__ WidthPlan make_width_plan(int H, int I, int bits) {
+    WidthPlan w;
+    const int KG = H / kGroup, nst = H / 64;
+    w.tb = tile_bytes(bits);
+    w.qb = d_quarter_bytes(bits);
+    const int gcap = kStageBytes / w.tb, dcap = kStageBytes / (256 + w.qb);
+    w.ngc = (2 * KG + gcap - 1) / gcap;
+    w.gbase = 2 * KG / w.ngc;
+    w.grem = 2 * KG - w.gbase * w.ngc;
+    w.ndc = (nst + dcap - 1) / dcap;
+    w.dbase = nst / w.ndc;
+    w.drem = nst - w.dbase * w.ndc;
+    w.gu_part = (uint32_t)(gu_tiles(H, I) * w.tb);
+    w.d_block = (uint32_t)d_block_bytes(H, bits);
+    return w;
+}
+// items [b, e) of chunk c: n = base * parts + rem items cut as above
+__device__ __forceinline__ void chunk_items(int base, int rem, int c, int &b, int &e) {
+    b = c * base + (c < rem ? c : rem);
+    e = b + base + (c < rem ? 1 : 0);
+}
+// the three pieces of unit (slot j, slice i): gate/up tiles, down scale/zero entries, down quarter
 struct UnitGeo {
-    const uint8_t *gu, *sz, *q;   // gate/up tiles, down scale/zero entries, down quarter
-    int j, i, bits;               // expert slot, 16-row slice, code width
+    const uint8_t *gu, *sz, *q;
 };
-__device__ __forceinline__ UnitGeo unit_geo(const DecodeArgs &a, const DecodeSmem &S, int u) {
-    const int sp = a.I / kSlice;
+__device__ __forceinline__ UnitGeo unit_geo(const DecodeArgs &a, const DecodeSmem &S, const WidthPlan &w, int j, int i) {
     UnitGeo g;
-    g.j = u / sp;
-    g.i = u - g.j * sp;
-    g.bits = S.ubits[g.j];
-    const int tb = tile_bytes(g.bits);
-    const uint8_t *base = a.packed + (size_t)S.uoff[g.j] * 256;
-    g.gu = base + (size_t)(2 * g.i) * (a.H / kGroup) * tb;
-    const uint8_t *blk = base + gu_tiles(a.H, a.I) * tb + (size_t)(g.i >> 2) * d_block_bytes(a.H, g.bits);
-    g.sz = blk;
-    g.q = blk + d_quarter_offset(a.H, g.bits, g.i & 3);
+    const uint8_t *base = a.packed + (size_t)S.uoff[j] * 256;
+    g.gu = base + (size_t)(2 * i) * (a.H / kGroup) * w.tb;
+    g.sz = base + w.gu_part + (size_t)(i >> 2) * w.d_block;
+    g.q = g.sz + (size_t)4 * a.H + (size_t)(i & 3) * (a.H / 64) * w.qb;
     return g;
-}
-// chunks of a unit: its 2 * KG gate/up tiles, then its H / 64 down super-tiles (each chunk one
-// ring stage), cut into nearly equal parts
-__device__ __forceinline__ int gu_chunks(int KG, int tb) {
-    const int cap = kStageBytes / tb;
-    return (2 * KG + cap - 1) / cap;
-}
-__device__ __forceinline__ int d_chunks(int nst, int qb) {
-    const int cap = kStageBytes / (256 + qb);
-    return (nst + cap - 1) / cap;
-}
-__device__ __forceinline__ void split_range(int n, int parts, int i, int &b, int &e) {
-    const int base = n / parts, rem = n % parts;
-    b = i * base + (i < rem ? i : rem);
-    e = b + base + (i < rem ? 1 : 0);
 }
 
 // ------------------------------------------------------------------------------ tile math
@@ -750,6 +770,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             S.ebits[e] = (uint8_t)v.bits;
         }
     }
+    if (threadIdx.x < 3) S.wplan[threadIdx.x] = make_width_plan(H, a.I, 4 + 2 * threadIdx.x);
     for (int i = threadIdx.x; i < 2 * NT * 4 * 32; i += kThreads) gred[i] = 0.f;
     if (STW < 0)
         for (int i = threadIdx.x; i < H; i += kThreads) ycta[i] = 0.f;
@@ -769,8 +790,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         }
         S.epoch = *reinterpret_cast<volatile unsigned long long *>(&a.ctl->done) / (unsigned long long)nC;
     }
-    if (xs_on && !mbar_wait(smem_u32(&S.xbar), 0, a.wait_ns, status)) S.abort = 1;
-    if (wr_on && ne > 0 && !mbar_wait(smem_u32(&S.wbar), 0, a.wait_ns, status)) S.abort = 1;
+    if (xs_on && !mbar_wait_idle(smem_u32(&S.xbar), 0, a.wait_ns, status)) S.abort = 1;
+    if (wr_on && ne > 0 && !mbar_wait_idle(smem_u32(&S.wbar), 0, a.wait_ns, status)) S.abort = 1;
     __syncthreads();
     const unsigned long long epoch = S.epoch;
     const uint32_t tag = (uint32_t)(epoch + 1ull);
@@ -866,35 +887,44 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         // ------------------------------------------------------------ producer (one thread)
         if (lane != 0) return;
         uint32_t cc = 0;
+        int s = 0;
+        uint32_t use = 0;
         bool ok = true;
+        const int sp = a.I / kSlice;
+        int j = S.u0 / sp, i = S.u0 - (S.u0 / sp) * sp;   // slot and slice of the current unit
         for (int u = S.u0; u < S.u1 && ok; ++u) {
-            const UnitGeo ug = unit_geo(a, S, u);
-            const int tb = tile_bytes(ug.bits), qb = d_quarter_bytes(ug.bits);
-            const int ngc = gu_chunks(KG, tb), ndc = d_chunks(nst, qb);
-            for (int ch = 0; ch < ngc + ndc; ++ch) {
-                const int s = cc % NS;
-                const uint32_t use = cc / NS;
-                if (use > 0 && (S.abort || !mbar_wait(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
+            const WidthPlan w = S.wplan[width_index(S.ubits[j])];
+            const UnitGeo ug = unit_geo(a, S, w, j, i);
+            for (int ch = 0; ch < w.ngc + w.ndc; ++ch) {
+                if (use > 0 && (S.abort || !mbar_wait_idle(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
                     S.abort = 1;
                     ok = false;
                     break;
                 }
                 const uint32_t fb = smem_u32(&S.full[s]);
-                uint8_t *dst = ring + (size_t)s * kStageBytes;
+                const uint32_t dst = smem_u32(ring + (size_t)s * kStageBytes);
                 int b0, b1;
-                if (ch < ngc) {
-                    split_range(2 * KG, ngc, ch, b0, b1);
-                    const uint32_t bytes = (uint32_t)((b1 - b0) * tb);
+                if (ch < w.ngc) {
+                    chunk_items(w.gbase, w.grem, ch, b0, b1);
+                    const uint32_t bytes = (uint32_t)((b1 - b0) * w.tb);
                     mbar_expect_tx(fb, bytes);
-                    bulk_g2s(smem_u32(dst), ug.gu + (size_t)b0 * tb, bytes, fb);
+                    bulk_g2s(dst, ug.gu + (size_t)b0 * w.tb, bytes, fb);
                 } else {
-                    split_range(nst, ndc, ch - ngc, b0, b1);
-                    const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * qb);
+                    chunk_items(w.dbase, w.drem, ch - w.ngc, b0, b1);
+                    const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * w.qb);
                     mbar_expect_tx(fb, zb + qbytes);
-                    bulk_g2s(smem_u32(dst), ug.sz + (size_t)b0 * 256, zb, fb);
-                    bulk_g2s(smem_u32(dst + zb), ug.q + (size_t)b0 * qb, qbytes, fb);
+                    bulk_g2s(dst, ug.sz + (size_t)b0 * 256, zb, fb);
+                    bulk_g2s(dst + zb, ug.q + (size_t)b0 * w.qb, qbytes, fb);
                 }
                 ++cc;
+                if (++s == NS) {
+                    s = 0;
+                    ++use;
+                }
+            }
+            if (++i == sp) {
+                i = 0;
+                ++j;
             }
         }
         // copies still in flight land before the CTA may exit (bounded by at least 1 ms, also when
@@ -943,18 +973,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         }
     };
     auto wait_full = [&]() {
-        if (!bad && (S.abort || !mbar_wait(smem_u32(&S.full[s]), par, a.wait_ns, status))) bad = true;
+        if (!bad && (S.abort || !mbar_wait_idle(smem_u32(&S.full[s]), par, a.wait_ns, status))) bad = true;
     };
     auto release_stage = [&]() {
         __syncwarp();
         if (!bad && lane == 0) mbar_arrive(smem_u32(&S.empty[s]));
         next_stage();
     };
+    const int sp = a.I / kSlice;
+    int uj = S.u0 / sp, ui = S.u0 - (S.u0 / sp) * sp;   // slot and slice of the current unit
     for (int u = S.u0; u < S.u1; ++u) {
-        const UnitGeo ug = unit_geo(a, S, u);
-        if (ug.j != cur) {
+        const int bits = S.ubits[uj];
+        const WidthPlan w = S.wplan[width_index(bits)];
+        if (uj != cur) {
             if (T > 1 && cur >= 0 && !bad) flush_slot();
-            cur = ug.j;
+            cur = uj;
             cur_pf = S.pfirst[cur];
             cur_nj = S.pfirst[cur + 1] - cur_pf;
 #pragma unroll
@@ -967,8 +1000,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 jc.xs1[nt] = smem_u32(Xs) + (uint32_t)(S.ptok[cur_pf + (q1 < cur_nj ? q1 : 0)] * G * 4);
             }
         }
-        const int tb = tile_bytes(ug.bits), qb = d_quarter_bytes(ug.bits);
-        const int ngc = gu_chunks(KG, tb), ndc = d_chunks(nst, qb);
+        if (++ui == sp) {
+            ui = 0;
+            ++uj;
+        }
+        const int ngc = w.ngc, ndc = w.ndc, qb = w.qb;
         // gate/up: split K over the warps, partial sums into shared memory
         float gacc[2][NT][4];
 #pragma unroll
@@ -979,10 +1015,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             wait_full();
             if (!bad) {
                 int t0, t1;
-                split_range(2 * KG, ngc, ch, t0, t1);
+                chunk_items(w.gbase, w.grem, ch, t0, t1);
                 const uint8_t *stg = ring + (size_t)s * kStageBytes;
-                if (ug.bits == 4) gu_chunk<4, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
-                else if (ug.bits == 6) gu_chunk<6, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+                if (bits == 4) gu_chunk<4, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+                else if (bits == 6) gu_chunk<6, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
                 else gu_chunk<8, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
             }
             release_stage();
@@ -1050,7 +1086,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             dc.hb[nt][1] = vh.y;
             dc.lb[nt][0] = vl.x;
             dc.lb[nt][1] = vl.y;
-            if (ug.bits != 4) {
+            if (bits != 4) {
                 dc.hb16[nt][0] = bf16x2_mul16(vh.x);
                 dc.hb16[nt][1] = bf16x2_mul16(vh.y);
                 dc.lb16[nt][0] = bf16x2_mul16(vl.x);
@@ -1068,7 +1104,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             wait_full();
             if (!bad) {
                 int s0, s1;
-                split_range(nst, ndc, ch, s0, s1);
+                chunk_items(w.dbase, w.drem, ch, s0, s1);
                 const uint32_t zb = smem_u32(ring + (size_t)s * kStageBytes), qbase = zb + (uint32_t)((s1 - s0) * 256);
                 if (STW > 0) {
 #pragma unroll
@@ -1076,16 +1112,16 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                         const int st = warp + l * kCW;
                         if (st >= s0 && st < s1) {
                             const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
-                            if (ug.bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[l]);
-                            else if (ug.bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[l]);
+                            if (bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[l]);
+                            else if (bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[l]);
                             else down_st<8, NT>(zp, qp, dc, lane, yacc[l]);
                         }
                     }
                 } else {
                     for (int st = s0 + ((warp - s0) % kCW + kCW) % kCW; st < s1; st += kCW) {
                         const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
-                        if (ug.bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[0]);
-                        else if (ug.bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[0]);
+                        if (bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[0]);
+                        else if (bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[0]);
                         else down_st<8, NT>(zp, qp, dc, lane, yacc[0]);
                         if (STW == 0) {
                             emit_st<NT>(a, S, cur_pf, cur_nj, st, yacc[0], lane);

@@ -223,6 +223,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
         }
     }
 }
+// The same bounded wait, suspending the thread between checks (try_wait with a time hint), so that
+// waiting warps take no issue slots from the warps that work.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity, uint64_t limit_ns, uint32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+        if (global_timer() - t0 > limit_ns) {
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
 // 1-D bulk copy global -> shared, completion counted on an mbarrier (no multicast).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
     asm volatile(
