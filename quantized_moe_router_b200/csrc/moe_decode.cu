@@ -112,7 +112,7 @@ struct DecodeLayout {
     size_t xs, xsum, gred, hbuf, hcol, ycta, ring, total;
     int stages;
 };
-template <int NT>
+template <int NT, int CW>
 DecodeLayout decode_layout(int T, int H, int smem_limit) {
     DecodeLayout L;
     size_t o = align_up(sizeof(DecodeSmem), 128);
@@ -120,12 +120,12 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
     if ((size_t)T * H * 2 <= (size_t)kActBytes) o += align_up((size_t)T * H * 2, 128);
     L.xsum = o;                                   // x group sums [T x H/64] fp32
     o += align_up((size_t)T * (H / kGroup) * 4, 128);
-    L.gred = o;                                   // gate/up partial sums [2][NT][4][32] fp32
-    o += (size_t)2 * NT * 4 * 32 * 4;
+    L.gred = o;                                   // gate/up partial sums of each warp [CW][2][NT][4][32] fp32
+    o += (size_t)CW * 2 * NT * 4 * 32 * 4;
     L.hbuf = o;                                   // h hi / lo [2][NT][8 pairs][16] bf16
     o += (size_t)2 * NT * 8 * 16 * 2;
-    L.hcol = o;                                   // per pair column: X = sum h [NT x 8], weight [NT x 8]
-    o += (size_t)2 * NT * 8 * 4;
+    L.hcol = o;                                   // h of each of the 16 rows and pair columns [16][NT x 8] fp32
+    o += (size_t)16 * NT * 8 * 4;
     L.ycta = o;                                   // one token: the CTA's output rows [H] fp32
     if (T == 1) o += align_up((size_t)H * 4, 128);
     L.ring = align_up(o, 128);
@@ -161,9 +161,6 @@ __device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long
     unsigned long long old;
     asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
     return old;
-}
-__device__ __forceinline__ void red_shared_f32(float *p, float v) {
-    asm volatile("red.relaxed.cta.shared::cta.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
 __device__ __forceinline__ void red_add_v4_f32(float *p, float4 v) {
     asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
@@ -581,6 +578,56 @@ struct GuCtx {
     bool bg;
 };
 
+// D = A * B + D (m16n8k16, bf16 operands, fp32 accumulators). Not volatile: independent MMAs of
+// a warp may be scheduled back to back (each has a latency of about 90 cycles on this part).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16x64 gate/up tile against one n-tile: the group's four MMAs into four separate
+// accumulators (no MMA waits for another), then the group's affine correction
+// out += s * (sum - (off + z) * X) with X the group sums of the lane's two accumulator columns.
+template <int BITS>
+__device__ __forceinline__ void gu_group_mma(const uint4 &lo, const uint4 &hi8, const uint2 &hi6,
+                                             const uint32_t (&b)[8], float sA, float zA, float sB, float zB,
+                                             float X0, float X1, float (&out)[4]) {
+    float c[4][4];
+    const uint32_t low[4] = {lo.x, lo.y, lo.z, lo.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
+        const uint32_t w = low[j];
+        mma16816(c[j], code_pair<0x000F000Fu>(w, 0), code_pair<0x000F000Fu>(w, 4), code_pair<0x000F000Fu>(w, 8),
+                 code_pair<0x000F000Fu>(w, 12), b[2 * j], b[2 * j + 1]);
+    }
+    if (BITS != 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t b0 = bf16x2_mul16(b[2 * j]), b1 = bf16x2_mul16(b[2 * j + 1]);
+            if (BITS == 8) {
+                const uint32_t w = (j == 0) ? hi8.x : (j == 1) ? hi8.y : (j == 2) ? hi8.z : hi8.w;
+                mma16816(c[j], code_pair<0x000F000Fu>(w, 0), code_pair<0x000F000Fu>(w, 4),
+                         code_pair<0x000F000Fu>(w, 8), code_pair<0x000F000Fu>(w, 12), b0, b1);
+            } else {
+                const uint32_t w = (j < 2) ? hi6.x : hi6.y;
+                const int s0 = (j & 1) * 8;
+                mma16816(c[j], code_pair<0x00030003u>(w, s0 + 0), code_pair<0x00030003u>(w, s0 + 2),
+                         code_pair<0x00030003u>(w, s0 + 4), code_pair<0x00030003u>(w, s0 + 6), b0, b1);
+            }
+        }
+    }
+    const float off = (BITS == 4) ? 128.f : 2176.f;   // 128 per plane, the hi plane weighted 16x
+    const float s0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]), s1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+    const float s2 = (c[0][2] + c[1][2]) + (c[2][2] + c[3][2]), s3 = (c[0][3] + c[1][3]) + (c[2][3] + c[3][3]);
+    out[0] += sA * (s0 - (off + zA) * X0);
+    out[1] += sA * (s1 - (off + zA) * X1);
+    out[2] += sB * (s2 - (off + zB) * X0);
+    out[3] += sB * (s3 - (off + zB) * X1);
+}
+
 template <int BITS, int NT>
 __device__ __forceinline__ void gu_tile(const uint8_t *tile, int kg, const GuCtx<NT> &jc, int lane,
                                         float (&acc)[NT][4]) {
@@ -606,7 +653,7 @@ __device__ __forceinline__ void gu_tile(const uint8_t *tile, int kg, const GuCtx
         }
         const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         const float X0 = lds32f(jc.xs0[nt] + kg * 4), X1 = lds32f(jc.xs1[nt] + kg * 4);
-        tile_group_mma<BITS>(lo, hi8, hi6, b, nullptr, sA, zA, sB, zB, X0, X1, acc[nt]);
+        gu_group_mma<BITS>(lo, hi8, hi6, b, sA, zA, sB, zB, X0, X1, acc[nt]);
     }
 }
 
@@ -648,44 +695,52 @@ template <int BITS, int NT>
 __device__ __forceinline__ void down_st(uint32_t szp, uint32_t qp, const DnCtx<NT> &dc, int lane,
                                         float (&acc)[4][NT][4]) {
     const int g = lane >> 2;
+    float c[4][NT][4], d[4][NT][4];
+    // the MMAs of all four 16-row blocks, each into its own accumulators
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const uint32_t w = lds32(qp + r * 128 + 4 * lane);
-        uint32_t hw = 0;
-        if (BITS == 8) hw = lds32(qp + kLoBytes + r * 128 + 4 * lane);
-        if (BITS == 6) hw = __byte_perm(lds16(qp + kLoBytes + r * 64 + 2 * lane), 0u, 0x4140);
-        const uint2 sz = lds64(szp + r * 64 + 8 * g);
-        const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
         const uint32_t a0 = code_pair<0x000F000Fu>(w, 0), a1 = code_pair<0x000F000Fu>(w, 4);
         const uint32_t a2 = code_pair<0x000F000Fu>(w, 8), a3 = code_pair<0x000F000Fu>(w, 12);
         uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
         if (BITS == 8) {
+            const uint32_t hw = lds32(qp + kLoBytes + r * 128 + 4 * lane);
             h0 = code_pair<0x000F000Fu>(hw, 0);
             h1 = code_pair<0x000F000Fu>(hw, 4);
             h2 = code_pair<0x000F000Fu>(hw, 8);
             h3 = code_pair<0x000F000Fu>(hw, 12);
         }
         if (BITS == 6) {
+            const uint32_t hw = __byte_perm(lds16(qp + kLoBytes + r * 64 + 2 * lane), 0u, 0x4140);
             h0 = code_pair<0x00030003u>(hw, 0);
             h1 = code_pair<0x00030003u>(hw, 2);
             h2 = code_pair<0x00030003u>(hw, 4);
             h3 = code_pair<0x00030003u>(hw, 6);
         }
-        const float off = (BITS == 4) ? 128.f : 2176.f;   // 128 per plane, the hi plane weighted 16x
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) c[r][nt][i] = d[r][nt][i] = 0.f;
+            mma16816(c[r][nt], a0, a1, a2, a3, dc.hb[nt][0], dc.hb[nt][1]);
+            mma16816(d[r][nt], a0, a1, a2, a3, dc.lb[nt][0], dc.lb[nt][1]);
+            if (BITS != 4) {
+                mma16816(c[r][nt], h0, h1, h2, h3, dc.hb16[nt][0], dc.hb16[nt][1]);
+                mma16816(d[r][nt], h0, h1, h2, h3, dc.lb16[nt][0], dc.lb16[nt][1]);
+            }
+        }
+    }
+    const float off = (BITS == 4) ? 128.f : 2176.f;   // 128 per plane, the hi plane weighted 16x
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const uint2 sz = lds64(szp + r * 64 + 8 * g);
+        const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
         const float oA = off + zA, oB = off + zB;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16(c, a0, a1, a2, a3, dc.hb[nt][0], dc.hb[nt][1]);
-            mma_bf16(d, a0, a1, a2, a3, dc.lb[nt][0], dc.lb[nt][1]);
-            if (BITS != 4) {
-                mma_bf16(c, h0, h1, h2, h3, dc.hb16[nt][0], dc.hb16[nt][1]);
-                mma_bf16(d, h0, h1, h2, h3, dc.lb16[nt][0], dc.lb16[nt][1]);
-            }
-            acc[r][nt][0] += (sA * dc.w0[nt]) * ((c[0] + d[0]) - oA * dc.X0[nt]);
-            acc[r][nt][1] += (sA * dc.w1[nt]) * ((c[1] + d[1]) - oA * dc.X1[nt]);
-            acc[r][nt][2] += (sB * dc.w0[nt]) * ((c[2] + d[2]) - oB * dc.X0[nt]);
-            acc[r][nt][3] += (sB * dc.w1[nt]) * ((c[3] + d[3]) - oB * dc.X1[nt]);
+            acc[r][nt][0] += (sA * dc.w0[nt]) * ((c[r][nt][0] + d[r][nt][0]) - oA * dc.X0[nt]);
+            acc[r][nt][1] += (sA * dc.w1[nt]) * ((c[r][nt][1] + d[r][nt][1]) - oA * dc.X1[nt]);
+            acc[r][nt][2] += (sB * dc.w0[nt]) * ((c[r][nt][2] + d[r][nt][2]) - oB * dc.X0[nt]);
+            acc[r][nt][3] += (sB * dc.w1[nt]) * ((c[r][nt][3] + d[r][nt][3]) - oB * dc.X1[nt]);
         }
     }
 }
@@ -727,8 +782,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     float *gred = reinterpret_cast<float *>(dyn + L.gred);
     uint16_t *hhi = reinterpret_cast<uint16_t *>(dyn + L.hbuf);
     uint16_t *hlo = hhi + NT * 8 * 16;
-    float *hX = reinterpret_cast<float *>(dyn + L.hcol);
-    float *hW = hX + NT * 8;
+    float *hrow = reinterpret_cast<float *>(dyn + L.hcol);
     float *ycta = reinterpret_cast<float *>(dyn + L.ycta);
     const int NS = L.stages;
     const int T = a.T, H = a.H, E = a.E, K = a.k, P = T * K;
@@ -771,7 +825,6 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         }
     }
     if (threadIdx.x < 3) S.wplan[threadIdx.x] = make_width_plan(H, a.I, 4 + 2 * threadIdx.x);
-    for (int i = threadIdx.x; i < 2 * NT * 4 * 32; i += kThreads) gred[i] = 0.f;
     if (STW < 0)
         for (int i = threadIdx.x; i < H; i += kThreads) ycta[i] = 0.f;
     // the router bias of this CTA's rows (a weight), off the logits' critical path
@@ -1023,57 +1076,41 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             }
             release_stage();
         }
+        // each warp's partial sums into its own slice of shared memory (plain stores)
         if (!bad) {
+            float *gw = gred + (size_t)warp * 2 * NT * 4 * 32 + lane;
 #pragma unroll
             for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) red_shared_f32(gred + ((rb * NT + nt) * 4 + i) * 32 + lane, gacc[rb][nt][i]);
+                    for (int i = 0; i < 4; ++i) gw[((rb * NT + nt) * 4 + i) * 32] = gacc[rb][nt][i];
         }
         if (consumer_sync_or<CW>(bad || S.abort)) {
             aborted = true;
             break;
         }
-        // SiLU-GLU of the unit's 16 rows, one warp per n-tile: h(row 8 rb + g, pair 2t + col)
-        if (warp < NT) {
-            const int nt = warp;
-            float xs0 = 0.f, xs1 = 0.f;
+        // SiLU-GLU, one intermediate row k of the unit per warp (warps k, k + CW), one pair column
+        // per lane: the gate and up sums over the warps' partials, h as a bf16 hi + lo pair, and
+        // hi + lo of every (row, column) for the down step's correction sums.
+        for (int k = warp; k < 16; k += kCW) {
+            if (lane < 8 * NT) {
+                const int nt = lane >> 3, pcol = lane & 7;
+                const int rb = k >> 3, src = ((k & 7) << 2) + (pcol >> 1), col = pcol & 1;
+                const float *gp = gred + ((rb * NT + nt) * 4 + col) * 32 + src;
+                float gt = 0.f, up = 0.f;
 #pragma unroll
-            for (int rb = 0; rb < 2; ++rb) {
-                float v[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float *p = gred + ((rb * NT + nt) * 4 + i) * 32 + lane;
-                    v[i] = *p;
-                    *p = 0.f;
+                for (int w2 = 0; w2 < kCW; ++w2) {
+                    gt += gp[(size_t)w2 * 2 * NT * 4 * 32];
+                    up += gp[(size_t)w2 * 2 * NT * 4 * 32 + 2 * 32];
                 }
-#pragma unroll
-                for (int col = 0; col < 2; ++col) {
-                    const float gt = v[col], up = v[2 + col];
-                    const float h = __fdividef(gt, 1.f + __expf(-gt)) * up;
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(h);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
-                    const int o = (nt * 8 + 2 * t + col) * 16 + 8 * rb + g;
-                    hhi[o] = __bfloat16_as_ushort(hi);
-                    hlo[o] = __bfloat16_as_ushort(lo);
-                    const float hs = __bfloat162float(hi) + __bfloat162float(lo);
-                    if (col == 0) xs0 += hs;
-                    else xs1 += hs;
-                }
-            }
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                xs0 += __shfl_xor_sync(0xffffffffu, xs0, off);
-                xs1 += __shfl_xor_sync(0xffffffffu, xs1, off);
-            }
-            if (g == 0) {
-                hX[nt * 8 + 2 * t] = xs0;
-                hX[nt * 8 + 2 * t + 1] = xs1;
-            }
-            if (lane < 8) {
-                const int q = nt * 8 + lane;
-                hW[nt * 8 + lane] = q < cur_nj ? S.pw[cur_pf + q] : 0.f;
+                const float h = __fdividef(gt, 1.f + __expf(-gt)) * up;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+                const int o = (nt * 8 + pcol) * 16 + k;
+                hhi[o] = __bfloat16_as_ushort(hi);
+                hlo[o] = __bfloat16_as_ushort(lo);
+                hrow[k * NT * 8 + lane] = __bfloat162float(hi) + __bfloat162float(lo);
             }
         }
         consumer_sync<CW>();
@@ -1094,10 +1131,19 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             } else {
                 dc.hb16[nt][0] = dc.hb16[nt][1] = dc.lb16[nt][0] = dc.lb16[nt][1] = 0u;
             }
-            dc.X0[nt] = hX[nt * 8 + 2 * t];
-            dc.X1[nt] = hX[nt * 8 + 2 * t + 1];
-            dc.w0[nt] = hW[nt * 8 + 2 * t];
-            dc.w1[nt] = hW[nt * 8 + 2 * t + 1];
+            // X of the lane's accumulator columns (pairs 2t, 2t + 1): the sums over the 16 rows
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float2 v = *reinterpret_cast<const float2 *>(hrow + k * NT * 8 + nt * 8 + 2 * t);
+                x0 += v.x;
+                x1 += v.y;
+            }
+            dc.X0[nt] = x0;
+            dc.X1[nt] = x1;
+            const int q0 = nt * 8 + 2 * t, q1 = q0 + 1;
+            dc.w0[nt] = q0 < cur_nj ? S.pw[cur_pf + q0] : 0.f;
+            dc.w1[nt] = q1 < cur_nj ? S.pw[cur_pf + q1] : 0.f;
         }
         // down: super-tile st of the unit's quarter goes to warp st % kCW
         for (int ch = 0; ch < ndc; ++ch) {
@@ -1198,7 +1244,7 @@ void logit_copies(int T, int E, int &rep, int &stride) {
 
 template <int NT, int STW, int CW>
 moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t st) {
-    const DecodeLayout L = decode_layout<NT>(a.T, a.H, dev->max_smem_optin);
+    const DecodeLayout L = decode_layout<NT, CW>(a.T, a.H, dev->max_smem_optin);
     if (L.stages < 2) return MOE_ERR_UNSUPPORTED;
     // the kernel attribute, once per device (concurrent first calls from several host threads
     // set the same value; the flag is atomic)
