@@ -68,6 +68,7 @@ struct DecodeArgs {
     uint32_t kmul;               // ceil(2^16 / k): p / k = (p * kmul) >> 16 for p < 2048
     int lrep;                    // copies of the logit words (a power of two)
     int lstride;                 // words between copies
+    int lsh, lsl;                // slices per router dot product (2^lsh) and their length
 };
 
 // Chunking of one work unit for one code width: gate/up tiles and down super-tiles, each cut into
@@ -103,7 +104,7 @@ struct __align__(16) DecodeSmem {
     float pw[kMaxP];
     int sel_idx[kMaxP];
     float sel_w[kMaxP];
-    float lpart[kMaxWarps];             // slice sums of the router dot products
+    float lpart[4 * kMaxWarps];         // slice sums of the router dot products
     float bias[kBiasRows];              // router bias of the CTA's rows c, c + nCTA, ...
 };
 
@@ -479,6 +480,72 @@ __device__ __forceinline__ unsigned long long unit_bytes(const DecodeArgs &a, in
            (unsigned long long)(a.H / 64) * d_quarter_bytes(bits) + 4ull * a.H;
 }
 
+// 64-bit compare-exchange of a descending sequence: the larger value first
+__device__ __forceinline__ void ce64(unsigned long long &a, unsigned long long &b) {
+    const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+    a = hi;
+    b = lo;
+}
+// Top-k of token t for E <= 256 and k <= 8, by merging: every lane sorts its 8 keys (expert
+// lane + 32 m), then five butterfly steps each keep the 8 largest of two lanes' lists (the
+// element-wise maximum of one list and the other reversed is a bitonic sequence holding them,
+// sorted by a 3-stage network), after which every lane holds the selection in order. Keys are
+// 64-bit {order key of the logit, 2^32 - 1 - expert}, so equal logits put the lower expert
+// first exactly. The softmax terms are formed one per lane. Writes as token_topk.
+__device__ bool token_topk_merge(const DecodeArgs &a, DecodeSmem &S, int t, uint32_t tag, int lane, int c) {
+    uint32_t sk[8];
+    if (!poll_keys<8>(a, t, tag, lane, sk)) return false;
+    int sm_[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) sm_[m] = m;
+    sort_ce(sk[0], sm_[0], sk[2], sm_[2]); sort_ce(sk[1], sm_[1], sk[3], sm_[3]);
+    sort_ce(sk[4], sm_[4], sk[6], sm_[6]); sort_ce(sk[5], sm_[5], sk[7], sm_[7]);
+    sort_ce(sk[0], sm_[0], sk[4], sm_[4]); sort_ce(sk[1], sm_[1], sk[5], sm_[5]);
+    sort_ce(sk[2], sm_[2], sk[6], sm_[6]); sort_ce(sk[3], sm_[3], sk[7], sm_[7]);
+    sort_ce(sk[0], sm_[0], sk[1], sm_[1]); sort_ce(sk[2], sm_[2], sk[3], sm_[3]);
+    sort_ce(sk[4], sm_[4], sk[5], sm_[5]); sort_ce(sk[6], sm_[6], sk[7], sm_[7]);
+    sort_ce(sk[2], sm_[2], sk[4], sm_[4]); sort_ce(sk[3], sm_[3], sk[5], sm_[5]);
+    sort_ce(sk[1], sm_[1], sk[4], sm_[4]); sort_ce(sk[3], sm_[3], sk[6], sm_[6]);
+    sort_ce(sk[1], sm_[1], sk[2], sm_[2]); sort_ce(sk[3], sm_[3], sk[4], sm_[4]);
+    sort_ce(sk[5], sm_[5], sk[6], sm_[6]);
+    unsigned long long v[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+        v[m] = sk[m] ? ((unsigned long long)sk[m] << 32) | (0xFFFFFFFFu - (uint32_t)(lane + 32 * sm_[m])) : 0ull;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        unsigned long long o[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) o[m] = __shfl_xor_sync(0xffffffffu, v[m], d);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) v[m] = v[m] > o[7 - m] ? v[m] : o[7 - m];
+        ce64(v[0], v[4]); ce64(v[1], v[5]); ce64(v[2], v[6]); ce64(v[3], v[7]);
+        ce64(v[0], v[2]); ce64(v[1], v[3]); ce64(v[4], v[6]); ce64(v[5], v[7]);
+        ce64(v[0], v[1]); ce64(v[2], v[3]); ce64(v[4], v[5]); ce64(v[6], v[7]);
+    }
+    const int K = a.k;
+    unsigned long long mine = v[0];
+#pragma unroll
+    for (int m = 1; m < 8; ++m) mine = (lane == m) ? v[m] : mine;
+    const float v0 = key_value((uint32_t)(v[0] >> 32));
+    const float my_v = key_value((uint32_t)(mine >> 32));
+    float ex = 0.f;
+    if (lane < K) ex = (v0 == -INFINITY) ? 1.f : expf(my_v - v0);
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < K) {
+        const int e = (int)(0xFFFFFFFFu - (uint32_t)mine);
+        const float w = ex / sum;
+        S.sel_idx[t * K + lane] = e;
+        S.sel_w[t * K + lane] = w;
+        if (c == 0 && a.idx_out) a.idx_out[t * K + lane] = e;
+        if (c == 0 && a.w_out) a.w_out[t * K + lane] = w;
+    }
+    __syncwarp();
+    return true;
+}
+
 // floor(n / d) for n < 2^53 through the double quotient (within one of the result), corrected
 __device__ __forceinline__ unsigned long long div_floor(unsigned long long n, unsigned long long d) {
     unsigned long long q = (unsigned long long)((double)n / (double)d);
@@ -491,6 +558,20 @@ __device__ __forceinline__ unsigned long long div_floor(unsigned long long n, un
 // takes the units whose first byte lies in [c * B / nC, (c + 1) * B / nC) of the B bytes of all.
 __device__ void plan_units(const DecodeArgs &a, DecodeSmem &S, int lane, int c, int nC) {
     const int U = S.U, sp = a.I / kSlice;
+    {
+        // all slots of one width (the usual case): equal units, a 32-bit cut
+        bool same = true;
+        for (int j = lane; j < U; j += 32) same = same && S.ubits[j] == S.ubits[0];
+        if (__all_sync(0xffffffffu, same)) {
+            const uint32_t N = (uint32_t)(U * sp);
+            if (lane == 0) {
+                S.u0 = (int)((uint32_t)c * N / (uint32_t)nC);
+                S.u1 = (int)((uint32_t)(c + 1) * N / (uint32_t)nC);
+            }
+            __syncwarp();
+            return;
+        }
+    }
     unsigned long long carry = 0;
     for (int base = 0; base < U; base += 32) {
         const int j = base + lane;
@@ -854,22 +935,23 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     // in slice order. Every logit word goes to lrep copies of the T x E block (lstride words
     // apart, spread over the L2 slices); CTA c polls copy c mod lrep.
     auto row_bias = [&](int i, int e) -> float { return i < kBiasRows ? S.bias[i] : (a.bias ? a.bias[e] : 0.f); };
+    // every lane r < lrep stores copy r of a logit word
     auto publish_logit = [&](int t, int e, float l) {
         const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(l);
-        for (int r = 0; r < a.lrep; ++r) st_relaxed_u64(a.logits + (size_t)r * a.lstride + (size_t)t * E + e, w);
+        if (lane < a.lrep) st_relaxed_u64(a.logits + (size_t)lane * a.lstride + (size_t)t * E + e, w);
     };
-    const int nq = ne * T;
-    const int nstr = (H + 255) / 256;
-    const int nsl = (nq > 0 && nq < kWarps) ? min(kWarps / nq, nstr) : 1;
+    // slices: nsl = 2^lsh per dot product, each lsl elements (a multiple of 256), so that the
+    // CTA's dot products spread over its warps without integer division
+    const int nq = ne * T, nsl = 1 << a.lsh;
     for (int it = warp; it < nq * nsl; it += kWarps) {
-        const int q = it / nsl, sl = it - q * nsl;
-        const int i = q / T, t = q % T;
+        const int q = it >> a.lsh, sl = it & (nsl - 1);
+        const int i = T == 1 ? q : q / T, t = T == 1 ? 0 : q - (q / T) * T;
         const int e = c + i * nC;
         const float *wrow = wr_on ? wsm + (size_t)i * H : a.wr + (size_t)e * H;
         const uint16_t *xrow = xr + (size_t)t * H;
-        const int h1 = min(H, (sl + 1) * nstr / nsl * 256);
+        const int h1 = min(H, (sl + 1) * a.lsl);
         float acc0 = 0.f, acc1 = 0.f;
-        for (int h = sl * nstr / nsl * 256 + lane * 8; h < h1; h += 256) {
+        for (int h = sl * a.lsl + lane * 8; h < h1; h += 256) {
             const float4 w0 = *reinterpret_cast<const float4 *>(wrow + h);
             const float4 w1 = *reinterpret_cast<const float4 *>(wrow + h + 4);
             const uint4 xv = xs_on ? *reinterpret_cast<const uint4 *>(xrow + h) : __ldcg(reinterpret_cast<const uint4 *>(xrow + h));
@@ -881,15 +963,14 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         float acc = acc0 + acc1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-            if (nsl == 1) publish_logit(t, e, acc + row_bias(i, e));
-            else S.lpart[it] = acc;
-        }
+        if (nsl == 1) publish_logit(t, e, acc + row_bias(i, e));
+        else if (lane == 0) S.lpart[it] = acc;
     }
     if (nsl > 1) {
+        // the slices' sums added in slice order (the same logit bits on every run)
         __syncthreads();
-        if (threadIdx.x < nq) {
-            const int q = threadIdx.x, i = q / T, t = q % T;
+        for (int q = warp; q < nq; q += kWarps) {
+            const int i = T == 1 ? q : q / T, t = T == 1 ? 0 : q - (q / T) * T;
             const int e = c + i * nC;
             float l = 0.f;
             for (int sl = 0; sl < nsl; ++sl) l += S.lpart[q * nsl + sl];
@@ -921,7 +1002,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     };
     // ---------------------------------------------------------------- top-k (every CTA) + plan
     auto route_token = [&](int t) {
-        const bool ok = !S.abort && (E <= 256 ? token_topk(a, S, t, tag, lane, c) : token_topk_wide(a, S, t, tag, lane, c));
+        const bool ok = !S.abort && (E <= 256 ? (K <= 8 ? token_topk_merge(a, S, t, tag, lane, c) : token_topk(a, S, t, tag, lane, c))
+                                              : token_topk_wide(a, S, t, tag, lane, c));
         if (!ok && lane == 0) S.abort = 1;
     };
     // tokens go to warps from the control warp on, so that with one token the control warp routes
@@ -1292,6 +1374,17 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     a.wait_ns = wait_limit_ns();
     a.kmul = (uint32_t)((65536 + k - 1) / k);
     logit_copies(T, E, a.lrep, a.lstride);
+    {
+        // the most slices (a power of two dividing H / 256) that give every warp of the CTA with
+        // the most router rows one dot-product slice at most
+        const int warps = T == 1 ? 17 : (T <= 16 ? 17 : 9);
+        const int nq = ((E + dev->sms - 1) / dev->sms) * T;
+        const int nstr = (H + 255) / 256;
+        int sh = 0;
+        while (nstr % (2 << sh) == 0 && nq * (2 << sh) <= warps && (2 << sh) <= 4 * kMaxWarps / max(nq, 1)) ++sh;
+        a.lsh = sh;
+        a.lsl = (nstr >> sh) * 256;
+    }
     // One token: 16 consumer warps, the CTA's output rows in shared memory. Several tokens: every
     // super-tile's rows are added into the output at once.
     if (T == 1) return launch_nt<1, -1, 16>(a, dev, st);

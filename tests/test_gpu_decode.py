@@ -145,7 +145,9 @@ def test_decode_workspace_shared_across_shapes():
 
 @pytest.mark.parametrize("E,k,dups", [
     (16, 16, [(2, 5), (0, 15)]),      # one expert per lane: ties between lanes (the exact fallback)
-    (40, 32, [(3, 35), (10, 20)])])   # a tie inside a lane (3, 35) and one between lanes (10, 20)
+    (40, 32, [(3, 35), (10, 20)]),    # a tie inside a lane (3, 35) and one between lanes (10, 20)
+    (64, 8, [(3, 35), (10, 20), (0, 63)]),    # the merging selection (k <= 8): ties across lanes and lists
+    (256, 4, [(7, 200), (100, 101)])])
 def test_decode_exact_ties_take_lower_index(E, k, dups):
     rng = np.random.default_rng(E * 31 + k)
     T, H, I = 5, 128, 64
