@@ -76,7 +76,7 @@ struct DecodeArgs {
 // base + 1 items for c < rem), and the byte offsets of an expert's parts.
 struct WidthPlan {
     int tb, qb;                   // gate/up tile bytes, down super-tile quarter bytes
-    int ngc, gbase, grem;         // gate/up chunks of the unit's 2 * KG tiles
+    int ngc, gbase, grem;         // gate/up chunks of the unit's KG group columns (2 tiles each)
     int ndc, dbase, drem;         // down chunks of its H / 64 super-tiles
     uint32_t gu_part, d_block;    // bytes of the expert's gate/up part, of one down group block
 };
@@ -618,10 +618,10 @@ __device__ __forceinline__ WidthPlan make_width_plan(int H, int I, int bits) {
     const int KG = H / kGroup, nst = H / 64;
     w.tb = tile_bytes(bits);
     w.qb = d_quarter_bytes(bits);
-    const int gcap = kStageBytes / w.tb, dcap = kStageBytes / (256 + w.qb);
-    w.ngc = (2 * KG + gcap - 1) / gcap;
-    w.gbase = 2 * KG / w.ngc;
-    w.grem = 2 * KG - w.gbase * w.ngc;
+    const int gcap = kStageBytes / (2 * w.tb), dcap = kStageBytes / (256 + w.qb);
+    w.ngc = (KG + gcap - 1) / gcap;
+    w.gbase = KG / w.ngc;
+    w.grem = KG - w.gbase * w.ngc;
     w.ndc = (nst + dcap - 1) / dcap;
     w.dbase = nst / w.ndc;
     w.drem = nst - w.dbase * w.ndc;
@@ -671,7 +671,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // One 16x64 gate/up tile against one n-tile: the group's four MMAs into four separate
 // accumulators (no MMA waits for another), then the group's affine correction
 // out += s * (sum - (off + z) * X) with X the group sums of the lane's two accumulator columns.
-template <int BITS>
+template <int BITS, bool ONE>
 __device__ __forceinline__ void gu_group_mma(const uint4 &lo, const uint4 &hi8, const uint2 &hi6,
                                              const uint32_t (&b)[8], float sA, float zA, float sB, float zB,
                                              float X0, float X1, float (&out)[4]) {
@@ -701,25 +701,39 @@ __device__ __forceinline__ void gu_group_mma(const uint4 &lo, const uint4 &hi8, 
         }
     }
     const float off = (BITS == 4) ? 128.f : 2176.f;   // 128 per plane, the hi plane weighted 16x
-    const float s0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]), s1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
-    const float s2 = (c[0][2] + c[1][2]) + (c[2][2] + c[3][2]), s3 = (c[0][3] + c[1][3]) + (c[2][3] + c[3][3]);
+    const float s0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]), s2 = (c[0][2] + c[1][2]) + (c[2][2] + c[3][2]);
     out[0] += sA * (s0 - (off + zA) * X0);
-    out[1] += sA * (s1 - (off + zA) * X1);
     out[2] += sB * (s2 - (off + zB) * X0);
-    out[3] += sB * (s3 - (off + zB) * X1);
+    if (!ONE) {   // one token: accumulator column 1 holds no pair
+        const float s1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]), s3 = (c[0][3] + c[1][3]) + (c[2][3] + c[3][3]);
+        out[1] += sA * (s1 - (off + zA) * X1);
+        out[3] += sB * (s3 - (off + zB) * X1);
+    }
 }
 
-template <int BITS, int NT>
-__device__ __forceinline__ void gu_tile(const uint8_t *tile, int kg, const GuCtx<NT> &jc, int lane,
-                                        float (&acc)[NT][4]) {
+// The two tiles of one group column kg (row blocks 2i and 2i + 1 of the unit, adjacent in the
+// packed layer) against the same n-tile operands: the x rows and group sums are read once, and the
+// tiles' eight MMAs are independent of each other.
+template <int BITS, int NT, bool ONE>
+__device__ __forceinline__ void gu_pair(const uint8_t *tile, int kg, const GuCtx<NT> &jc, int lane,
+                                        float (&acc)[2][NT][4]) {
+    constexpr int tb = tile_bytes(BITS);
     const int g = lane >> 2, t = lane & 3;
-    const uint4 lo = *reinterpret_cast<const uint4 *>(tile + 16 * lane);
-    uint4 hi8 = make_uint4(0, 0, 0, 0);
-    uint2 hi6 = make_uint2(0, 0);
-    if (BITS == 8) hi8 = *reinterpret_cast<const uint4 *>(tile + kLoBytes + 16 * lane);
-    if (BITS == 6) hi6 = *reinterpret_cast<const uint2 *>(tile + kLoBytes + 8 * lane);
-    const uint2 sz = *reinterpret_cast<const uint2 *>(tile + kLoBytes + hi_bytes(BITS) + 8 * g);
-    const float sA = half_lo(sz.x), zA = half_hi(sz.x), sB = half_lo(sz.y), zB = half_hi(sz.y);
+    uint4 lo[2], hi8[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    uint2 hi6[2] = {make_uint2(0, 0), make_uint2(0, 0)};
+    float sA[2], zA[2], sB[2], zB[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint8_t *tp = tile + r * tb;
+        lo[r] = *reinterpret_cast<const uint4 *>(tp + 16 * lane);
+        if (BITS == 8) hi8[r] = *reinterpret_cast<const uint4 *>(tp + kLoBytes + 16 * lane);
+        if (BITS == 6) hi6[r] = *reinterpret_cast<const uint2 *>(tp + kLoBytes + 8 * lane);
+        const uint2 sz = *reinterpret_cast<const uint2 *>(tp + kLoBytes + hi_bytes(BITS) + 8 * g);
+        sA[r] = half_lo(sz.x);
+        zA[r] = half_hi(sz.x);
+        sB[r] = half_lo(sz.y);
+        zB[r] = half_hi(sz.y);
+    }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         uint4 v0, v1;
@@ -733,31 +747,21 @@ __device__ __forceinline__ void gu_tile(const uint8_t *tile, int kg, const GuCtx
             v1 = lds128(jc.sb[nt] + o + 16);
         }
         const uint32_t b[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        const float X0 = lds32f(jc.xs0[nt] + kg * 4), X1 = lds32f(jc.xs1[nt] + kg * 4);
-        gu_group_mma<BITS>(lo, hi8, hi6, b, sA, zA, sB, zB, X0, X1, acc[nt]);
+        const float X0 = lds32f(jc.xs0[nt] + kg * 4), X1 = ONE ? 0.f : lds32f(jc.xs1[nt] + kg * 4);
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            gu_group_mma<BITS, ONE>(lo[r], hi8[r], hi6[r], b, sA[r], zA[r], sB[r], zB[r], X0, X1, acc[r][nt]);
     }
 }
 
-// The warp's gate/up tiles of a chunk holding the unit's tiles [t0, t1) (tile tt = row block
-// tt / KG, group column tt % KG): group column kg goes to warp kg % CW, two tiles at a time so
-// that their MMA chains interleave.
-template <int BITS, int NT, int CW>
-__device__ __forceinline__ void gu_chunk(const uint8_t *stage, int t0, int t1, int KG, int warp,
-                                         const GuCtx<NT> &jc, int lane, float (&acc)[2][NT][4]) {
+// The warp's gate/up work in a chunk holding the unit's group columns [k0, k1) (two tiles each):
+// group column kg goes to warp kg % CW.
+template <int BITS, int NT, int CW, bool ONE>
+__device__ __forceinline__ void gu_chunk(const uint8_t *stage, int k0, int k1, int warp, const GuCtx<NT> &jc,
+                                         int lane, float (&acc)[2][NT][4]) {
     constexpr int tb = tile_bytes(BITS);
-#pragma unroll
-    for (int rbl = 0; rbl < 2; ++rbl) {
-        const int lo_t = max(t0, rbl * KG), hi_t = min(t1, (rbl + 1) * KG);
-        if (lo_t >= hi_t) continue;
-        const int k0 = lo_t - rbl * KG, k1 = hi_t - rbl * KG;
-        int kg = k0 + ((warp - k0) % CW + CW) % CW;
-        const uint8_t *p0 = stage + (size_t)(rbl * KG - t0) * tb;
-        for (; kg + CW < k1; kg += 2 * CW) {
-            gu_tile<BITS, NT>(p0 + (size_t)kg * tb, kg, jc, lane, acc[rbl]);
-            gu_tile<BITS, NT>(p0 + (size_t)(kg + CW) * tb, kg + CW, jc, lane, acc[rbl]);
-        }
-        if (kg < k1) gu_tile<BITS, NT>(p0 + (size_t)kg * tb, kg, jc, lane, acc[rbl]);
-    }
+    for (int kg = k0 + ((warp - k0) % CW + CW) % CW; kg < k1; kg += CW)
+        gu_pair<BITS, NT, ONE>(stage + (size_t)(kg - k0) * 2 * tb, kg, jc, lane, acc);
 }
 
 // Down operands of the current unit for this lane: h of the unit's 16 rows for the lane's B
@@ -772,7 +776,7 @@ struct DnCtx {
 
 // One 64-row super-tile of the unit's down quarter: four 16x16 MMAs (per n-tile and h half), the
 // row's scale and zero and the column's weight applied in fp32: acc += w * s * (sum - (off + z) X).
-template <int BITS, int NT>
+template <int BITS, int NT, bool ONE>
 __device__ __forceinline__ void down_st(uint32_t szp, uint32_t qp, const DnCtx<NT> &dc, int lane,
                                         float (&acc)[4][NT][4]) {
     const int g = lane >> 2;
@@ -802,11 +806,14 @@ __device__ __forceinline__ void down_st(uint32_t szp, uint32_t qp, const DnCtx<N
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) c[r][nt][i] = d[r][nt][i] = 0.f;
+            // one token: h hi and lo into one accumulator (fewer live registers; the four row
+            // blocks still run in parallel)
+            float (&dd)[4] = ONE ? c[r][nt] : d[r][nt];
             mma16816(c[r][nt], a0, a1, a2, a3, dc.hb[nt][0], dc.hb[nt][1]);
-            mma16816(d[r][nt], a0, a1, a2, a3, dc.lb[nt][0], dc.lb[nt][1]);
+            mma16816(dd, a0, a1, a2, a3, dc.lb[nt][0], dc.lb[nt][1]);
             if (BITS != 4) {
                 mma16816(c[r][nt], h0, h1, h2, h3, dc.hb16[nt][0], dc.hb16[nt][1]);
-                mma16816(d[r][nt], h0, h1, h2, h3, dc.lb16[nt][0], dc.lb16[nt][1]);
+                mma16816(dd, h0, h1, h2, h3, dc.lb16[nt][0], dc.lb16[nt][1]);
             }
         }
     }
@@ -819,9 +826,11 @@ __device__ __forceinline__ void down_st(uint32_t szp, uint32_t qp, const DnCtx<N
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             acc[r][nt][0] += (sA * dc.w0[nt]) * ((c[r][nt][0] + d[r][nt][0]) - oA * dc.X0[nt]);
-            acc[r][nt][1] += (sA * dc.w1[nt]) * ((c[r][nt][1] + d[r][nt][1]) - oA * dc.X1[nt]);
             acc[r][nt][2] += (sB * dc.w0[nt]) * ((c[r][nt][2] + d[r][nt][2]) - oB * dc.X0[nt]);
-            acc[r][nt][3] += (sB * dc.w1[nt]) * ((c[r][nt][3] + d[r][nt][3]) - oB * dc.X1[nt]);
+            if (!ONE) {
+                acc[r][nt][1] += (sA * dc.w1[nt]) * ((c[r][nt][1] + d[r][nt][1]) - oA * dc.X1[nt]);
+                acc[r][nt][3] += (sB * dc.w1[nt]) * ((c[r][nt][3] + d[r][nt][3]) - oB * dc.X1[nt]);
+            }
         }
     }
 }
@@ -867,7 +876,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     float *ycta = reinterpret_cast<float *>(dyn + L.ycta);
     const int NS = L.stages;
     const int T = a.T, H = a.H, E = a.E, K = a.k, P = T * K;
-    const int G = H / kGroup, KG = G, nst = H / 64;
+    const int G = H / kGroup, nst = H / 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nC = gridDim.x, c = blockIdx.x;
     uint32_t *status = &a.ctl->status;
@@ -1041,9 +1050,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 int b0, b1;
                 if (ch < w.ngc) {
                     chunk_items(w.gbase, w.grem, ch, b0, b1);
-                    const uint32_t bytes = (uint32_t)((b1 - b0) * w.tb);
+                    const uint32_t bytes = (uint32_t)((b1 - b0) * 2 * w.tb);
                     mbar_expect_tx(fb, bytes);
-                    bulk_g2s(dst, ug.gu + (size_t)b0 * w.tb, bytes, fb);
+                    bulk_g2s(dst, ug.gu + (size_t)b0 * 2 * w.tb, bytes, fb);
                 } else {
                     chunk_items(w.dbase, w.drem, ch - w.ngc, b0, b1);
                     const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * w.qb);
@@ -1072,8 +1081,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     // ---------------------------------------------------------------- consumers
     plan_ready_wait<CW>();
     const int g = lane >> 2, t = lane & 3;
+    // one token (STW = -1): only accumulator column 0 holds a pair, and the output rows are added
+    // into shared memory
+    constexpr bool ONE = STW < 0;
     constexpr int NL = STW > 0 ? STW : 1;
-    static_assert(STW >= 0 || NT == 1, "shared-memory output rows serve one token");
+    static_assert(!ONE || NT == 1, "one token takes one n-tile");
     float yacc[NL][4][NT][4];
     auto zero_y = [&]() {
 #pragma unroll
@@ -1149,12 +1161,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         for (int ch = 0; ch < ngc; ++ch) {
             wait_full();
             if (!bad) {
-                int t0, t1;
-                chunk_items(w.gbase, w.grem, ch, t0, t1);
+                int k0, k1;
+                chunk_items(w.gbase, w.grem, ch, k0, k1);
                 const uint8_t *stg = ring + (size_t)s * kStageBytes;
-                if (bits == 4) gu_chunk<4, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
-                else if (bits == 6) gu_chunk<6, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
-                else gu_chunk<8, NT, CW>(stg, t0, t1, KG, warp, jc, lane, gacc);
+                if (bits == 4) gu_chunk<4, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
+                else if (bits == 6) gu_chunk<6, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
+                else gu_chunk<8, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
             }
             release_stage();
         }
@@ -1240,17 +1252,17 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                         const int st = warp + l * kCW;
                         if (st >= s0 && st < s1) {
                             const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
-                            if (bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[l]);
-                            else if (bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[l]);
-                            else down_st<8, NT>(zp, qp, dc, lane, yacc[l]);
+                            if (bits == 4) down_st<4, NT, ONE>(zp, qp, dc, lane, yacc[l]);
+                            else if (bits == 6) down_st<6, NT, ONE>(zp, qp, dc, lane, yacc[l]);
+                            else down_st<8, NT, ONE>(zp, qp, dc, lane, yacc[l]);
                         }
                     }
                 } else {
                     for (int st = s0 + ((warp - s0) % kCW + kCW) % kCW; st < s1; st += kCW) {
                         const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
-                        if (bits == 4) down_st<4, NT>(zp, qp, dc, lane, yacc[0]);
-                        else if (bits == 6) down_st<6, NT>(zp, qp, dc, lane, yacc[0]);
-                        else down_st<8, NT>(zp, qp, dc, lane, yacc[0]);
+                        if (bits == 4) down_st<4, NT, ONE>(zp, qp, dc, lane, yacc[0]);
+                        else if (bits == 6) down_st<6, NT, ONE>(zp, qp, dc, lane, yacc[0]);
+                        else down_st<8, NT, ONE>(zp, qp, dc, lane, yacc[0]);
                         if (STW == 0) {
                             emit_st<NT>(a, S, cur_pf, cur_nj, st, yacc[0], lane);
                         } else if (t == 0) {

@@ -5,8 +5,10 @@
 //
 // Gate/up ("GU") tiles: 16 rows x 64 input columns (one quantisation group); rows 0-7 are gate
 // rows 8rb..8rb+7, rows 8-15 the up rows with the same indices, so one tile holds both
-// projections of eight intermediate rows; tile (rb, kg) for rb < I/8, kg < H/64, stored rb-major
-// (a row block's K sweep is contiguous). A tile is [lo nibble plane 512 B][hi plane: 0 B
+// projections of eight intermediate rows; tile (rb, kg) for rb < I/8, kg < H/64. Row blocks pair
+// up (2i, 2i + 1: the 16 intermediate rows 16i..16i+15) and a pair's tiles are stored K-major,
+// tile (rb, kg) at ((rb / 2) * (H/64) + kg) * 2 + rb % 2, so that the gate/up tiles of 16
+// intermediate rows are one contiguous run and the two tiles of each group column are adjacent. A tile is [lo nibble plane 512 B][hi plane: 0 B
 // (4-bit), 256 B (6-bit), 512 B (8-bit)][scale/zero 64 B]. Lane L of a warp (g = L/4, t = L%4)
 // owns bytes 16L..16L+15 of the lo plane: word j (j = 0..3) holds the eight codes that lane feeds
 // to MMA j as its A operand (rows g and g+8, group columns 16t+4j .. 16t+4j+3), arranged so that

@@ -86,7 +86,11 @@ __global__ void pack_expert_kernel(PackSrc src, int H, int I, uint8_t *dst, long
         sz = make_uint2(sA | (zA << 16), sB | (zB << 16));
     }
     if (tile < ngu) {
-        uint8_t *tp = dst + tile * tile_bytes(BITS);
+        // row blocks 2i and 2i + 1 (16 intermediate rows) interleaved along K: tile (rb, kg) at
+        // ((rb / 2) * KG + kg) * 2 + rb % 2
+        const int KG = H / kGroup, rb = (int)(tile / KG);
+        const long long pos = ((long long)(rb >> 1) * KG + kg) * 2 + (rb & 1);
+        uint8_t *tp = dst + pos * tile_bytes(BITS);
         *reinterpret_cast<uint4 *>(tp + 16 * lane) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         if (BITS == 8) *reinterpret_cast<uint4 *>(tp + kLoBytes + 16 * lane) = make_uint4(hi8[0], hi8[1], hi8[2], hi8[3]);
         if (BITS == 6) *reinterpret_cast<uint2 *>(tp + kLoBytes + 8 * lane) = make_uint2(hi6[0], hi6[1]);

@@ -364,7 +364,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                 // entries of the unit's super-tiles and its four quarters
                 auto frag = [&](int b, const uint8_t *&lo16, const uint8_t *&hip, const uint8_t *&szp) {
                     if (GU) {
-                        const uint8_t *rawt = raw + (size_t)rs * slot_bytes + (size_t)(b * KC + jk) * tb;
+                        // slot: per row-block pair, its KC group columns x 2 tiles
+                        const uint8_t *rawt =
+                            raw + (size_t)rs * slot_bytes + (size_t)(((b >> 1) * KC + jk) * 2 + (b & 1)) * tb;
                         lo16 = rawt + 16 * lane;
                         hip = rawt + kLoBytes + (bits == 8 ? 16 : 8) * lane;
                         szp = rawt + kLoBytes + hi_bytes(bits) + 8 * (lane >> 2);
@@ -517,9 +519,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     mbar_expect_tx(fb, (uint32_t)(nb * KC * tb));
                     uint8_t *slot = raw + (size_t)rs * slot_bytes;
                     if (GU) {
-                        for (int b = 0; b < nb; ++b)
-                            bulk_g2s(smem_u32(slot + (size_t)b * KC * tb),
-                                     mat + ((size_t)(8 * U.mt + b) * G.KG + k0) * tb, (uint32_t)(KC * tb), fb);
+                        // one copy per row-block pair: its tiles of group columns k0 .. k0 + KC - 1
+                        for (int pp = 0; pp < nb / 2; ++pp)
+                            bulk_g2s(smem_u32(slot + (size_t)pp * 2 * KC * tb),
+                                     mat + ((size_t)(4 * U.mt + pp) * G.KG + k0) * 2 * tb, (uint32_t)(2 * KC * tb), fb);
                     } else {
                         // per K step: the scale/zero entries of the unit's super-tiles, then its
                         // piece of each quarter (nb / 4 super-tiles from super-tile 2 * mt)
