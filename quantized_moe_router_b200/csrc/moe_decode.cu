@@ -105,6 +105,8 @@ struct __align__(16) DecodeSmem {
     int sel_idx[kMaxP];
     float sel_w[kMaxP];
     float lpart[4 * kMaxWarps];         // slice sums of the router dot products
+    unsigned long long cand[kMaxWarps * 32];   // one token's top-k candidates, k per warp
+    unsigned long long selk[kMaxK];     // the selection in order
     float bias[kBiasRows];              // router bias of the CTA's rows c, c + nCTA, ...
 };
 
@@ -544,6 +546,92 @@ __device__ bool token_topk_merge(const DecodeArgs &a, DecodeSmem &S, int t, uint
     }
     __syncwarp();
     return true;
+}
+
+// One token's top-k by the whole CTA (E <= 32 x warps, k <= 32). Warp w polls the logits of
+// experts 32w .. 32w + 31 (one per lane) and sorts them by a bitonic network across the lanes;
+// its k largest become candidates. After a CTA barrier every warp ranks some candidates against
+// all of them (ballots); candidate of rank r < k is the r-th selection. Keys are 64-bit {order
+// key of the logit, 2^32 - 1 - expert}: equal logits put the lower expert first, exactly.
+// Phase 1 (warps w < ceil(E / 32)); returns false (warp-uniformly) when the wait expires.
+__device__ __forceinline__ bool topk_one_candidates(const DecodeArgs &a, DecodeSmem &S, uint32_t tag, int warp,
+                                                    int lane) {
+    const int e = 32 * warp + lane;
+    const unsigned long long *row = a.logits + (size_t)(blockIdx.x & (unsigned)(a.lrep - 1)) * a.lstride;
+    unsigned long long v = 0ull;
+    uint64_t t0 = 0;
+    for (int it = 0;; ++it) {
+        bool ok = true;
+        uint32_t kk = 0;
+        if (e < a.E) {
+            const unsigned long long w = ld_relaxed_u64(row + e);
+            ok = (uint32_t)(w >> 32) == tag;
+            float x = __uint_as_float((uint32_t)w);
+            if (x != x) x = -INFINITY;
+            kk = order_key(x);   // never 0 for a non-NaN value
+        }
+        if (__all_sync(0xffffffffu, ok)) {
+            v = e < a.E ? ((unsigned long long)kk << 32) | (0xFFFFFFFFu - (uint32_t)e) : 0ull;
+            break;
+        }
+        int expired = 0;
+        if (lane == 0) {
+            const uint64_t now = global_timer();
+            if (it == 0) t0 = now;
+            expired = (now - t0 > a.wait_ns) ? 1 : 0;
+            if (expired) atomicOr(&a.ctl->status, kStatusTimeout);
+        }
+        if (__shfl_sync(0xffffffffu, expired, 0)) return false;
+        __nanosleep(32);
+    }
+    // bitonic sort across the lanes, descending (lane 0 the largest)
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
+            const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+            v = keep_max ? (v > o ? v : o) : (v > o ? o : v);
+        }
+    if (lane < a.k) S.cand[warp * a.k + lane] = v;
+    return true;
+}
+// Phase 2 (all warps, after a barrier): candidate i's rank among the C = nw * k candidates.
+template <int kWarps>
+__device__ __forceinline__ void topk_one_rank(const DecodeArgs &a, DecodeSmem &S, int nw, int warp, int lane) {
+    const int C = nw * a.k;
+    unsigned long long mine[kMaxWarps];   // candidates lane + 32 m (C <= 32 * kWarps)
+#pragma unroll
+    for (int m = 0; m < kWarps; ++m) mine[m] = (lane + 32 * m < C) ? S.cand[lane + 32 * m] : 0ull;
+    for (int i = warp; i < C; i += kWarps) {
+        const unsigned long long x = S.cand[i];
+        int rank = 0;
+#pragma unroll
+        for (int m = 0; m < kWarps; ++m)
+            if (32 * m < C) rank += __popc(__ballot_sync(0xffffffffu, mine[m] > x));
+        if (lane == 0 && rank < a.k) S.selk[rank] = x;
+    }
+}
+// Phase 3 (one warp, after a barrier): indices and softmax weights of the selection.
+__device__ __forceinline__ void topk_one_finish(const DecodeArgs &a, DecodeSmem &S, int lane, int c) {
+    const int K = a.k;
+    const unsigned long long mine = lane < K ? S.selk[lane] : 0ull;
+    const float v0 = key_value((uint32_t)(S.selk[0] >> 32));
+    const float my_v = key_value((uint32_t)(mine >> 32));
+    float ex = 0.f;
+    if (lane < K) ex = (v0 == -INFINITY) ? 1.f : expf(my_v - v0);
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < K) {
+        const int e = (int)(0xFFFFFFFFu - (uint32_t)mine);
+        const float w = ex / sum;
+        S.sel_idx[lane] = e;
+        S.sel_w[lane] = w;
+        if (c == 0 && a.idx_out) a.idx_out[lane] = e;
+        if (c == 0 && a.w_out) a.w_out[lane] = w;
+    }
+    __syncwarp();
 }
 
 // floor(n / d) for n < 2^53 through the double quotient (within one of the result), corrected
@@ -1015,13 +1103,24 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                                               : token_topk_wide(a, S, t, tag, lane, c));
         if (!ok && lane == 0) S.abort = 1;
     };
-    // tokens go to warps from the control warp on, so that with one token the control warp routes
-    // it and makes the plan without a CTA barrier in between
-    for (int t = (warp + 1) % kWarps; t < T; t += kWarps) route_token(t);
-    if (warp != kPW || T > 1) group_sums(threadIdx.x, T > 1 ? kThreads : kCW * 32);
-    if (T > 1) __syncthreads();
+    const bool one = T == 1 && E <= 32 * kWarps;   // one token: the whole CTA routes it
+    if (one) {
+        const int nw = (E + 31) >> 5;
+        if (warp < nw && !S.abort && !topk_one_candidates(a, S, tag, warp, lane) && lane == 0) S.abort = 1;
+        __syncthreads();
+        if (!S.abort) topk_one_rank<kWarps>(a, S, nw, warp, lane);
+        __syncthreads();
+        if (warp != kPW) group_sums(threadIdx.x, kCW * 32);
+    } else {
+        // tokens go to warps from the control warp on, so that with one token the control warp
+        // routes it and makes the plan without a CTA barrier in between
+        for (int t = (warp + 1) % kWarps; t < T; t += kWarps) route_token(t);
+        if (warp != kPW || T > 1) group_sums(threadIdx.x, T > 1 ? kThreads : kCW * 32);
+        if (T > 1) __syncthreads();
+    }
     if (warp == kPW) {
         __syncwarp();
+        if (one && !S.abort) topk_one_finish(a, S, lane, c);
         const int Pp = S.abort ? 0 : P;
         if (T == 1) plan_single(S, Pp, lane);
         else plan_many(a, S, Pp, lane);
@@ -1192,12 +1291,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 const int nt = lane >> 3, pcol = lane & 7;
                 const int rb = k >> 3, src = ((k & 7) << 2) + (pcol >> 1), col = pcol & 1;
                 const float *gp = gred + ((rb * NT + nt) * 4 + col) * 32 + src;
-                float gt = 0.f, up = 0.f;
+                // the warps' partials, summed as a tree (all loads first)
+                float gv[kCW], uv[kCW];
 #pragma unroll
                 for (int w2 = 0; w2 < kCW; ++w2) {
-                    gt += gp[(size_t)w2 * 2 * NT * 4 * 32];
-                    up += gp[(size_t)w2 * 2 * NT * 4 * 32 + 2 * 32];
+                    gv[w2] = gp[(size_t)w2 * 2 * NT * 4 * 32];
+                    uv[w2] = gp[(size_t)w2 * 2 * NT * 4 * 32 + 2 * 32];
                 }
+#pragma unroll
+                for (int h = kCW / 2; h > 0; h >>= 1)
+#pragma unroll
+                    for (int w2 = 0; w2 < h; ++w2) {
+                        gv[w2] += gv[w2 + h];
+                        uv[w2] += uv[w2 + h];
+                    }
+                const float gt = gv[0], up = uv[0];
                 const float h = __fdividef(gt, 1.f + __expf(-gt)) * up;
                 const __nv_bfloat16 hi = __float2bfloat16_rn(h);
                 const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
@@ -1226,13 +1334,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 dc.hb16[nt][0] = dc.hb16[nt][1] = dc.lb16[nt][0] = dc.lb16[nt][1] = 0u;
             }
             // X of the lane's accumulator columns (pairs 2t, 2t + 1): the sums over the 16 rows
-            float x0 = 0.f, x1 = 0.f;
+            float xa[16], xb[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float2 v = *reinterpret_cast<const float2 *>(hrow + k * NT * 8 + nt * 8 + 2 * t);
-                x0 += v.x;
-                x1 += v.y;
+                xa[k] = v.x;
+                xb[k] = v.y;
             }
+#pragma unroll
+            for (int h = 8; h > 0; h >>= 1)
+#pragma unroll
+                for (int k = 0; k < h; ++k) {
+                    xa[k] += xa[k + h];
+                    xb[k] += xb[k + h];
+                }
+            const float x0 = xa[0], x1 = xb[0];
             dc.X0[nt] = x0;
             dc.X1[nt] = x1;
             const int q0 = nt * 8 + 2 * t, q1 = q0 + 1;
