@@ -596,21 +596,23 @@ __device__ __forceinline__ bool topk_one_candidates(const DecodeArgs &a, DecodeS
     if (lane < a.k) S.cand[warp * a.k + lane] = v;
     return true;
 }
-// Phase 2 (all warps, after a barrier): candidate i's rank among the C = nw * k candidates.
-template <int kWarps>
-__device__ __forceinline__ void topk_one_rank(const DecodeArgs &a, DecodeSmem &S, int nw, int warp, int lane) {
-    const int C = nw * a.k;
-    unsigned long long mine[kMaxWarps];   // candidates lane + 32 m (C <= 32 * kWarps)
-#pragma unroll
-    for (int m = 0; m < kWarps; ++m) mine[m] = (lane + 32 * m < C) ? S.cand[lane + 32 * m] : 0ull;
-    for (int i = warp; i < C; i += kWarps) {
-        const unsigned long long x = S.cand[i];
-        int rank = 0;
-#pragma unroll
-        for (int m = 0; m < kWarps; ++m)
-            if (32 * m < C) rank += __popc(__ballot_sync(0xffffffffu, mine[m] > x));
-        if (lane == 0 && rank < a.k) S.selk[rank] = x;
+// Phase 2 (all threads, after a barrier): thread i ranks candidate i among the C = nw * k
+// candidates, four independent counts over all of them.
+__device__ __forceinline__ void topk_one_rank(const DecodeArgs &a, DecodeSmem &S, int nw) {
+    const int C = nw * a.k, i = threadIdx.x;
+    if (i >= C) return;
+    const unsigned long long x = S.cand[i];
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+    int j = 0;
+    for (; j + 4 <= C; j += 4) {
+        r0 += S.cand[j] > x;
+        r1 += S.cand[j + 1] > x;
+        r2 += S.cand[j + 2] > x;
+        r3 += S.cand[j + 3] > x;
     }
+    for (; j < C; ++j) r0 += S.cand[j] > x;
+    const int rank = (r0 + r1) + (r2 + r3);
+    if (rank < a.k) S.selk[rank] = x;
 }
 // Phase 3 (one warp, after a barrier): indices and softmax weights of the selection.
 __device__ __forceinline__ void topk_one_finish(const DecodeArgs &a, DecodeSmem &S, int lane, int c) {
@@ -1108,7 +1110,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         const int nw = (E + 31) >> 5;
         if (warp < nw && !S.abort && !topk_one_candidates(a, S, tag, warp, lane) && lane == 0) S.abort = 1;
         __syncthreads();
-        if (!S.abort) topk_one_rank<kWarps>(a, S, nw, warp, lane);
+        if (!S.abort) topk_one_rank(a, S, nw);
         __syncthreads();
         if (warp != kPW) group_sums(threadIdx.x, kCW * 32);
     } else {
@@ -1127,49 +1129,63 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         plan_units(a, S, lane, c, nC);
         // hand the plan to the consumer warps and start streaming without waiting for them
         plan_ready_arrive<CW>();
-        // ------------------------------------------------------------ producer (one thread)
-        if (lane != 0) return;
+        // ------------------------------------------------------------ producer
+        // The copies of chunk cc (in unit order) go to stage cc % NS. The first NS chunks find
+        // every stage free: lane cc issues chunk cc, all at once; lane 0 then issues the rest,
+        // each after its stage is released.
         uint32_t cc = 0;
-        int s = 0;
-        uint32_t use = 0;
         bool ok = true;
         const int sp = a.I / kSlice;
-        int j = S.u0 / sp, i = S.u0 - (S.u0 / sp) * sp;   // slot and slice of the current unit
-        for (int u = S.u0; u < S.u1 && ok; ++u) {
-            const WidthPlan w = S.wplan[width_index(S.ubits[j])];
-            const UnitGeo ug = unit_geo(a, S, w, j, i);
-            for (int ch = 0; ch < w.ngc + w.ndc; ++ch) {
-                if (use > 0 && (S.abort || !mbar_wait_idle(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
-                    S.abort = 1;
-                    ok = false;
-                    break;
+        auto walk = [&](bool fill) {
+            int s = 0;
+            uint32_t use = 0;
+            int j = S.u0 / sp, i = S.u0 - (S.u0 / sp) * sp;   // slot and slice of the current unit
+            for (int u = S.u0; u < S.u1 && ok; ++u) {
+                const WidthPlan w = S.wplan[width_index(S.ubits[j])];
+                const UnitGeo ug = unit_geo(a, S, w, j, i);
+                for (int ch = 0; ch < w.ngc + w.ndc; ++ch) {
+                    if (fill ? (use > 0) : false) return;
+                    const bool mine = fill ? (int)cc == lane : use > 0;
+                    if (!fill && use > 0 &&
+                        (S.abort || !mbar_wait_idle(smem_u32(&S.empty[s]), (use - 1) & 1u, a.wait_ns, status))) {
+                        S.abort = 1;
+                        ok = false;
+                        return;
+                    }
+                    if (mine) {
+                        const uint32_t fb = smem_u32(&S.full[s]);
+                        const uint32_t dst = smem_u32(ring + (size_t)s * kStageBytes);
+                        int b0, b1;
+                        if (ch < w.ngc) {
+                            chunk_items(w.gbase, w.grem, ch, b0, b1);
+                            const uint32_t bytes = (uint32_t)((b1 - b0) * 2 * w.tb);
+                            mbar_expect_tx(fb, bytes);
+                            bulk_g2s(dst, ug.gu + (size_t)b0 * 2 * w.tb, bytes, fb);
+                        } else {
+                            chunk_items(w.dbase, w.drem, ch - w.ngc, b0, b1);
+                            const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * w.qb);
+                            mbar_expect_tx(fb, zb + qbytes);
+                            bulk_g2s(dst, ug.sz + (size_t)b0 * 256, zb, fb);
+                            bulk_g2s(dst + zb, ug.q + (size_t)b0 * w.qb, qbytes, fb);
+                        }
+                    }
+                    ++cc;
+                    if (++s == NS) {
+                        s = 0;
+                        ++use;
+                    }
                 }
-                const uint32_t fb = smem_u32(&S.full[s]);
-                const uint32_t dst = smem_u32(ring + (size_t)s * kStageBytes);
-                int b0, b1;
-                if (ch < w.ngc) {
-                    chunk_items(w.gbase, w.grem, ch, b0, b1);
-                    const uint32_t bytes = (uint32_t)((b1 - b0) * 2 * w.tb);
-                    mbar_expect_tx(fb, bytes);
-                    bulk_g2s(dst, ug.gu + (size_t)b0 * 2 * w.tb, bytes, fb);
-                } else {
-                    chunk_items(w.dbase, w.drem, ch - w.ngc, b0, b1);
-                    const uint32_t zb = (uint32_t)((b1 - b0) * 256), qbytes = (uint32_t)((b1 - b0) * w.qb);
-                    mbar_expect_tx(fb, zb + qbytes);
-                    bulk_g2s(dst, ug.sz + (size_t)b0 * 256, zb, fb);
-                    bulk_g2s(dst + zb, ug.q + (size_t)b0 * w.qb, qbytes, fb);
-                }
-                ++cc;
-                if (++s == NS) {
-                    s = 0;
-                    ++use;
+                if (++i == sp) {
+                    i = 0;
+                    ++j;
                 }
             }
-            if (++i == sp) {
-                i = 0;
-                ++j;
-            }
-        }
+        };
+        walk(true);
+        __syncwarp();
+        if (lane != 0) return;
+        cc = 0;
+        walk(false);
         // copies still in flight land before the CTA may exit (bounded by at least 1 ms, also when
         // the wait limit is 0)
         for (uint32_t q = cc > (uint32_t)NS ? cc - NS : 0; q < cc; ++q)
