@@ -130,12 +130,13 @@ inline DecodeWs decode_ws_layout(int T, int H, int I, int E, int k) {
 
 // Prefill workspace. x16: the hidden states of every (token, expert) pair in bucket order as fp16
 // scaled by 2^-xexp[t] per token; h: fp16 h of
-// every (token, expert) pair in bucket order, scaled by 2^-hexp per 16-column block; fexp: the
-// largest hexp of each pair; nt_start: N-tile prefix of the experts ([E] = total, [E+1] = the
-// largest N tile, rows rounded to 16).
+// every (token, expert) pair in bucket order, scaled by 2^-hexp per 16-column block; nt_start: N-tile prefix of the experts ([E] = total, [E+1] = the
+// largest N tile, rows rounded to 16); ntab: one entry per N tile {expert | bits << 16, first
+// bucket row, rows, expert's bucket offset}; pscale: a per-pair column scale in bucket order
+// (gate/up: 2^xexp of the pair's token; down: routing weight * 2^fexp).
 struct PrefillWs {
-    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, x16, xexp, h, hexp, fexp, out_acc, planes, lg,
-        total;
+    size_t idx, w, counts, offsets, blockhist, pair_tok, pair_w, nt_start, ntab, pscale, x16, xexp, h, hexp, out_acc,
+        planes, lg, total;
     int nblk;  // token blocks of the stable scatter
 };
 constexpr int kScatterTokens = 64;
@@ -152,12 +153,13 @@ inline PrefillWs prefill_ws_layout(int T, int H, int I, int E, int k) {
     w.blockhist = take((size_t)w.nblk * E * 4);
     w.pair_tok = take(P * 4);
     w.pair_w = take(P * 4);
-    w.nt_start = take((size_t)(E + 2) * 4);
+    w.nt_start = take((size_t)(E + 3) * 4);
+    w.ntab = take((P / 256 + (size_t)E + 1) * 16);   // sum over experts of ceil(n_e / 256)
+    w.pscale = take(P * 4);
     w.x16 = take(P * H * 2);
     w.xexp = take((size_t)T * 4);
     w.h = take(P * I * 2);
     w.hexp = take(P * (I / 16));
-    w.fexp = take(P * 4);
     w.out_acc = take((size_t)T * H * 4);
     w.planes = take((size_t)3 * E * H * 2);   // router rows as three bf16 planes
     w.lg = take((size_t)T * E * 4);           // fp32 router logits
@@ -259,6 +261,11 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
 }
 __device__ __forceinline__ void red_add_f32(float *p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+// the same reduction without a compiler memory barrier, for accumulators that the issuing kernel
+// never reads: loads around it may be scheduled freely
+__device__ __forceinline__ void red_add_f32_free(float *p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v));
 }
 // bf16x2 operand from a code word: (word >> shift) & mask | bf16(128) in both halves, i.e.
 // the bf16 pair {128 + field_lo, 128 + field_hi}; exact for fields < 128.

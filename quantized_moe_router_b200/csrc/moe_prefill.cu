@@ -18,9 +18,9 @@ moe_status_t launch_route_tc(const uint16_t *x, const float *wr, const float *bi
                              int32_t *idx_out, float *w_out, uint16_t *planes, float *lg, uint32_t *status,
                              cudaStream_t st);
 moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I, int E, int k, const int32_t *counts,
-                                     const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
-                                     const float *pair_w, const uint16_t *x, uint16_t *x16, int32_t *xexp,
-                                     uint16_t *h16, int8_t *hexp, int32_t *fexp, float *out_acc, uint32_t *status,
+                                     const int32_t *offsets, int32_t *nt_start, int4 *ntab, const int32_t *pair_tok,
+                                     const float *pair_w, float *pscale, const uint16_t *x, uint16_t *x16,
+                                     int32_t *xexp, uint16_t *h16, int8_t *hexp, float *out_acc, uint32_t *status,
                                      cudaStream_t st);
 
 namespace {
@@ -148,10 +148,11 @@ moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T
     moe_status_t s = launch_tc_prefill_gemms(
         static_cast<const uint8_t *>(packed), T, H, I, E, k, reinterpret_cast<const int32_t *>(w8 + L.counts),
         reinterpret_cast<const int32_t *>(w8 + L.offsets), reinterpret_cast<int32_t *>(w8 + L.nt_start),
-        reinterpret_cast<const int32_t *>(w8 + L.pair_tok), reinterpret_cast<const float *>(w8 + L.pair_w), x,
+        reinterpret_cast<int4 *>(w8 + L.ntab), reinterpret_cast<const int32_t *>(w8 + L.pair_tok),
+        reinterpret_cast<const float *>(w8 + L.pair_w), reinterpret_cast<float *>(w8 + L.pscale), x,
         reinterpret_cast<uint16_t *>(w8 + L.x16), reinterpret_cast<int32_t *>(w8 + L.xexp),
-        reinterpret_cast<uint16_t *>(w8 + L.h), reinterpret_cast<int8_t *>(w8 + L.hexp),
-        reinterpret_cast<int32_t *>(w8 + L.fexp), oacc, &reinterpret_cast<Control *>(w8)->status, st);
+        reinterpret_cast<uint16_t *>(w8 + L.h), reinterpret_cast<int8_t *>(w8 + L.hexp), oacc,
+        &reinterpret_cast<Control *>(w8)->status, st);
     if (s != MOE_OK) return s;
     const size_t n = (size_t)T * H;
     convert_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 256, 0, st>>>(oacc, out, n);

@@ -19,14 +19,19 @@
 //   * 1 warp issues tcgen05.mma (kind::f16, fp16 x fp16 -> fp32, M = 128, N = tokens rounded up
 //     to 16) into one of two TMEM accumulators, 4 MMAs (K = 16) per 64-wide K step, and frees
 //     each ring stage with tcgen05.commit;
-//   * 4 epilogue warps read the other accumulator with tcgen05.ld while the next unit runs:
-//     gate/up undoes the token scale, pairs each gate row with its up row (8 TMEM lanes apart),
-//     applies SiLU-GLU and stores h as fp16 with one power-of-two exponent per 16 columns (a small
-//     kernel between the GEMMs brings each pair's h to one common exponent); down undoes the
-//     pair's exponent and adds w * y into the fp32 output accumulator with red.add.
+//   * 8 epilogue warps (two per TMEM lane quarter, taking alternate 32-column chunks) read the
+//     other accumulator with tcgen05.ld while the next unit runs: gate/up undoes the token scale,
+//     pairs each gate row with its up row (8 TMEM lanes apart), applies SiLU-GLU and stores h as
+//     fp16 with one power-of-two exponent per 16 columns (a small kernel between the GEMMs brings
+//     each pair's h to one common exponent); down undoes the pair's exponent and adds w * y into
+//     the fp32 output accumulator with red.add. The per-column tables of the next unit (token,
+//     scale) are loaded while the current unit is processed.
 // fp16 operands (11-bit significands) keep the block within its error bound where bf16
 // operands (8-bit) would not; every scaling is by a power of two and exact.
 // Every mbarrier wait is bounded; the CTA frees its TMEM before it exits.
+#include <atomic>
+#include <mutex>
+
 #include "moe_tc.cuh"
 
 namespace moe {
@@ -38,25 +43,30 @@ constexpr int kMaxN = 256;                        // tokens per unit (UMMA N lim
 constexpr int kABStages = 3;
 constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
 constexpr int kMaxRaw = 8;                        // raw ring slots (K chunks) at most
-constexpr int kDqWarps = 4, kLdWarps = 1;
+#ifndef MOE_TC_DQ_WARPS
+#define MOE_TC_DQ_WARPS 4
+#endif
+constexpr int kDqWarps = MOE_TC_DQ_WARPS, kLdWarps = 1;
+constexpr int kBPW = 8 / kDqWarps;                // 16-row blocks of the A tile per dequantiser warp
 constexpr int kRowBox = 64;                       // token rows per tensor copy
 constexpr int kMmaWarp = kDqWarps + kLdWarps;
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quarter
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kEpiWarp0 = kMmaWarp + 1;
-constexpr int kProdWarp = kEpiWarp0 + 4;
+constexpr int kProdWarp = kEpiWarp0 + kEpiWarps;
 constexpr int kTcWarps = kProdWarp + 1;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr uint32_t kTmemCols = 2 * kMaxN;         // two accumulators of 256 fp32 columns
 constexpr int kBarEpi = 1;                        // named barrier of the epilogue warps (0 is __syncthreads)
 constexpr int kMaxSub = 64;                       // 16-column blocks of a down row (I <= 1024)
+static_assert(kEpiThreads == kMaxN, "one epilogue thread per column of a unit");
 
 struct TcArgs {
     const uint8_t *packed;
     int H, I, E;
-    const int32_t *counts, *offsets, *nt_start, *pair_tok;
-    const float *pair_w;
-    const uint16_t *act;   // gate/up: x16 [pairs x H]; down: h16 [pairs x I], both in bucket order
-    const int32_t *xexp;   // gate/up: per-token exponent of x16
-    const int32_t *fexp;   // down: per-pair exponent of h16
+    const int32_t *nt_start, *pair_tok;
+    const int4 *ntab;      // N tiles: {expert | bits << 16, first row in the bucket, rows, bucket offset}
+    const float *pscale;   // per pair in bucket order: gate/up 2^xexp of its token, down w * 2^fexp
     uint16_t *h;           // gate/up output: h16
     int8_t *hexp_out;      // gate/up output: exponents of h16
     float *out_acc;        // down output: [T x H] fp32
@@ -89,28 +99,21 @@ __host__ __device__ inline int ntile_count(int n) {
 }
 
 struct Unit {
-    int e, mt, n0, nn, nr, base;
+    int e, bits, mt, n0, nn, nr, base;
 };
 
-// Unit u = (N tile u / mtiles, M tile u % mtiles); the expert owning an N tile is found by a
-// binary search of nt_start (exclusive prefix of the experts' N-tile counts).
+// Unit u = (N tile u / mtiles, M tile u % mtiles), read from the N-tile table.
 __device__ __forceinline__ Unit unit_at(const TcArgs &a, int u, int mtiles) {
     Unit U;
     const int ti = u / mtiles;
     U.mt = u - ti * mtiles;
-    int lo = 0, hi = a.E;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(a.nt_start + mid) <= ti) lo = mid;
-        else hi = mid;
-    }
-    U.e = lo;
-    const int n_e = __ldg(a.counts + lo);
-    const int sz = ntile_size(n_e);
-    U.n0 = (ti - __ldg(a.nt_start + lo)) * sz;
-    U.nn = min(sz, n_e - U.n0);
-    U.nr = (U.nn + 15) & ~15;
-    U.base = __ldg(a.offsets + lo);
+    const int4 v = __ldg(a.ntab + ti);
+    U.e = v.x & 0xFFFF;
+    U.bits = v.x >> 16;
+    U.n0 = v.y;
+    U.nn = v.z;
+    U.nr = (v.z + 15) & ~15;
+    U.base = v.w;
     return U;
 }
 
@@ -145,7 +148,8 @@ __device__ __forceinline__ int scale_exp(float vmax) {
 //   low nibble q of byte x  -> 0x3F0q0000 = 0.5 + q/256   (row g of the lane fragment)
 //   high nibble q of byte x -> 0x3F80(q<<4)00 = 1 + q/2048 (row g+8)
 // so w = (q - z) * s = f * S + C with S = 256 s (2048 s) and C = -(128 + z) s (-(2048 + z) s).
-// C is rounded once to fp32 (|error| <= 2^-24 |C|, far below the fp16 rounding of w).
+// C is rounded once to fp32 (|error| <= 2^-24 |C|, far below the fp16 rounding of w). (Measured
+// on B200: this fp32 form beats an fp16x2 s*q form with the zero point folded into extra K steps.)
 __device__ __forceinline__ float nib_float(uint32_t m, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(m), "r"(0x3F800000u), "r"(sel));
@@ -274,8 +278,8 @@ template <bool GU>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t tc_dyn[];
     __shared__ TcShared S;
-    __shared__ int ep_i[kMaxN];     // epilogue: token of each column (down) / unused (gate/up)
-    __shared__ float ep_f[kMaxN];   // epilogue: 2^xexp of each column (gate/up) / w * 2^fexp (down)
+    __shared__ __align__(16) int ep_i[2][kMaxN];     // epilogue: token of each column (down)
+    __shared__ __align__(16) float ep_f[2][kMaxN];   // epilogue: scale of each column
     const uint32_t pad = (1024u - (smem_u32(tc_dyn) & 1023u)) & 1023u;
     uint8_t *base = tc_dyn + pad;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -292,16 +296,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     const uint32_t side_bytes = GU ? (uint32_t)align_up((size_t)nr_max * 128, 1024) : 0u;
     uint8_t *raw = side + side_bytes;
     // K chunks of KC tiles per row block (KC divides the unit's K steps, so chunks never straddle
-    // units); a raw slot holds one chunk of the 8 row blocks at the layer's widest tile
-    const int KC = (G.KG % 4 == 0) ? 4 : ((G.KG % 2 == 0) ? 2 : 1);
-    int tb_max = 0;
-    {
-        const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
-        for (int e = 0; e < a.E; ++e) tb_max = max(tb_max, tile_bytes(pe[e].bits));
+    // units); a raw slot holds one chunk of the 8 row blocks at the layer's widest tile. The
+    // largest KC that leaves room for 3 slots (at least 2).
+    const int tb_max = __ldg(a.nt_start + a.E + 2);
+    const long long raw_room = (long long)a.smem_bytes - (long long)pad - (long long)(raw - base);
+    int KC = 1, R = 0;
+    for (int kc = 4; kc >= 1; kc >>= 1) {
+        if (G.KG % kc) continue;
+        const int r = (int)(raw_room / (8LL * kc * tb_max));
+        if (r >= 3 || kc == 1) {
+            KC = kc;
+            R = r;
+            break;
+        }
     }
-    const uint32_t slot_bytes = (uint32_t)(8 * KC * tb_max);
-    int R = (int)(((long long)a.smem_bytes - (long long)pad - (long long)(raw - base)) / slot_bytes);
     R = R > kMaxRaw ? kMaxRaw : R;
+    const uint32_t slot_bytes = (uint32_t)(8 * KC * tb_max);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kABStages; ++s) {
@@ -310,7 +320,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&S.acc_full[s]), 1);
-            mbar_init(smem_u32(&S.acc_empty[s]), 4);
+            mbar_init(smem_u32(&S.acc_empty[s]), kEpiWarps);
         }
         mbar_init(smem_u32(&S.fin), 1);
         for (int s = 0; s < kMaxRaw; ++s) {
@@ -335,9 +345,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
 
     if (warp < kDqWarps) {
         // ------------------------------------------------------------ dequantisers
-        const int b0 = warp, b1 = warp + 4;
         bool ok = run;
-        const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(a.packed + sizeof(PackedHeader));
         // step counters kept incrementally (no division in the loop): position jk in the K
         // chunk, raw slot rs and its phase, A/B stage slot and its phase
         int jk = 0, rs = 0, slot = 0;
@@ -346,9 +354,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
             const Unit U = unit_at(a, u, G.mtiles);
             // per unit: the expert's width and whether this warp's row block exists
-            const int bits = __ldg(&pe[U.e].bits);
+            const int bits = U.bits;
             const int tb = tile_bytes(bits);
-            const bool have0 = 8 * U.mt + b0 < G.nrb, have1 = 8 * U.mt + b1 < G.nrb;
+            // this warp's row blocks warp + kDqWarps * i, and whether they exist in this M tile
+            bool have_all = true;
+#pragma unroll
+            for (int i = 0; i < kBPW; ++i) have_all &= 8 * U.mt + warp + kDqWarps * i < G.nrb;
             for (int kg = 0; kg < G.KG; ++kg) {
                 if (jk == 0 && !tc_wait(S, a, &S.raw_full[rs], rpar)) {
                     ok = false;
@@ -379,19 +390,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                         szp = base + (b >> 2) * 256 + (b & 3) * 64 + 8 * g;
                     }
                 };
-                const uint8_t *l0, *h0, *z0, *l1, *h1, *z1;
-                frag(b0, l0, h0, z0);
-                frag(b1, l1, h1, z1);
-                if (have0 && have1 && bits == 4) {
-                    dequant_fragment<4, !GU>(l0, h0, z0, lane, As, b0);
-                    dequant_fragment<4, !GU>(l1, h1, z1, lane, As, b1);
+                if (have_all && bits == 4) {
+#pragma unroll
+                    for (int i = 0; i < kBPW; ++i) {
+                        const uint8_t *lo16, *hip, *szp;
+                        frag(warp + kDqWarps * i, lo16, hip, szp);
+                        dequant_fragment<4, !GU>(lo16, hip, szp, lane, As, warp + kDqWarps * i);
+                    }
                 } else {
 #pragma unroll 1
-                    for (int bb = 0; bb < 2; ++bb) {
-                        const int b = bb ? b1 : b0;
-                        const bool have = bb ? have1 : have0;
-                        const uint8_t *lo16 = bb ? l1 : l0, *hip = bb ? h1 : h0, *szp = bb ? z1 : z0;
-                        if (!have) {
+                    for (int i = 0; i < kBPW; ++i) {
+                        const int b = warp + kDqWarps * i;
+                        const uint8_t *lo16, *hip, *szp;
+                        frag(b, lo16, hip, szp);
+                        if (8 * U.mt + b >= G.nrb) {
                             const uint4 z = make_uint4(0, 0, 0, 0);
                             const int g = lane >> 2, t = lane & 3;
                             *reinterpret_cast<uint4 *>(As + sw128_off(16 * b + g, 2 * t)) = z;
@@ -478,11 +490,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                     break;
                 }
                 tc_fence_after();
-                const uint32_t As = smem_u32(ring + (size_t)slot * stage_bytes);
+                const uint32_t As = smem_u32(ring + (size_t)slot * stage_bytes), Bs = As + kABytes;
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(d_tmem, sw128_desc(As + 32 * kk), sw128_desc(As + kABytes + 32 * kk), idesc,
+                        umma_f16(d_tmem, sw128_desc(As + 32 * kk), sw128_desc(Bs + 32 * kk), idesc,
                                  (kg > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(smem_u32(&S.ab_empty[slot]));
                 }
@@ -545,86 +557,135 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;          // this warp may read TMEM lanes 32q .. 32q+31
-        const int row = 32 * q + lane;   // accumulator row
-        const int et = threadIdx.x - kEpiWarp0 * 32;
+        const int q = warp & 3;                         // this warp may read TMEM lanes 32q .. 32q+31
+        const int half = (warp - kEpiWarp0) >> 2;       // it takes the 32-column chunks 2c + half
+        const int row = 32 * q + lane;                  // accumulator row
+        const int et = threadIdx.x - kEpiWarp0 * 32;    // 0 .. kEpiThreads - 1 (= kMaxN - 1)
         uint32_t i = 0;
         bool ok = run;
+        // column tables (token, scale) of unit i in buffer i & 1; those of unit i + 1 are loaded
+        // into registers while unit i is processed and stored after it
+        int nt_tok = 0;
+        float nt_sc = 0.f;
+        auto load_table = [&](const Unit &V) {
+            nt_tok = 0;
+            nt_sc = 0.f;
+            if (et < V.nn) {
+                nt_tok = __ldg(a.pair_tok + V.base + V.n0 + et);
+                nt_sc = __ldg(a.pscale + V.base + V.n0 + et);
+            }
+        };
+        Unit U{};
+        if ((int)blockIdx.x < nunits) {
+            U = unit_at(a, blockIdx.x, G.mtiles);
+            load_table(U);
+            ep_i[0][et] = nt_tok;
+            ep_f[0][et] = nt_sc;
+        }
         // every epilogue warp walks all units through the same named barriers; after an expired
         // wait it only skips the work
         for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
-            const Unit U = unit_at(a, u, G.mtiles);
             const uint32_t buf = i & 1u;
-            // per-column tables of this unit (filled while its MMAs run)
-            named_sync(kBarEpi, 128);
-            for (int r = et; ok && r < U.nn; r += 128) {
-                const int pos = U.base + U.n0 + r;
-                if (GU) {
-                    ep_f[r] = exp2i(__ldg(a.xexp + __ldg(a.pair_tok + pos)));
-                } else {
-                    ep_i[r] = __ldg(a.pair_tok + pos);
-                    ep_f[r] = __ldg(a.pair_w + pos) * exp2i(__ldg(a.fexp + pos));
-                }
+            named_sync(kBarEpi, kEpiThreads);   // tables of unit i stored; the staging tile is free
+            const int un = u + (int)gridDim.x;
+            Unit Un{};
+            if (un < nunits) {
+                Un = unit_at(a, un, G.mtiles);
+                load_table(Un);
             }
-            named_sync(kBarEpi, 128);
             if (ok && !tc_wait(S, a, &S.acc_full[buf], (i >> 1) & 1u)) ok = false;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kMaxN;
+            const int *tk = ep_i[buf];
+            const float *tf = ep_f[buf];
             if (GU) {
                 // row 16b + g: gate (g < 8) or up (g >= 8) of intermediate column 8b + (g & 7)
                 const bool gate = (row & 8) == 0;
                 const int col = 8 * (row >> 4) + (row & 7);
                 uint16_t *stg = reinterpret_cast<uint16_t *>(side);
-                for (int c0 = 0; ok && c0 < U.nr; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + c0, v);
+                // 16 columns from cb: the gate lane finishes token cb+2p, its up partner cb+2p+1
+                auto glu16 = [&](const uint32_t(&v)[16], int cb) {
+                    float recv[8], hv[8];
 #pragma unroll
-                    for (int jj = 0; jj < 16; jj += 2) {
-                        // the gate lane finishes token c0+jj, its up partner token c0+jj+1
-                        const float send = __uint_as_float(gate ? v[jj + 1] : v[jj]);
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-                        const int tok = c0 + jj + (gate ? 0 : 1);
-                        const float xs = ep_f[tok < U.nn ? tok : 0];
-                        const float gv = (gate ? __uint_as_float(v[jj]) : recv) * xs;
-                        const float uv = (gate ? recv : __uint_as_float(v[jj + 1])) * xs;
-                        const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                    for (int p = 0; p < 8; ++p)
+                        recv[p] = __shfl_xor_sync(0xffffffffu, __uint_as_float(gate ? v[2 * p + 1] : v[2 * p]), 8);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const float xs = tf[cb + 2 * p + (gate ? 0 : 1)];
+                        const float gv = (gate ? __uint_as_float(v[2 * p]) : recv[p]) * xs;
+                        const float uv = (gate ? recv[p] : __uint_as_float(v[2 * p + 1])) * xs;
+                        hv[p] = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                    }
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const int tok = cb + 2 * p + (gate ? 0 : 1);
                         // one exponent per 16 columns of this token: the max over the 16 lanes
                         // that hold the token (gate lanes 0-7, 16-23 or up lanes 8-15, 24-31)
-                        const uint32_t hb = (tok < U.nn) ? (__float_as_uint(hv) & 0x7FFFFFFFu) : 0u;
-                        const uint32_t mx = gate ? __reduce_max_sync(0x00FF00FFu, hb) : __reduce_max_sync(0xFF00FF00u, hb);
+                        const uint32_t hb = (tok < U.nn) ? (__float_as_uint(hv[p]) & 0x7FFFFFFFu) : 0u;
+                        const uint32_t mx =
+                            gate ? __reduce_max_sync(0x00FF00FFu, hb) : __reduce_max_sync(0xFF00FF00u, hb);
                         const int f = scale_exp(__uint_as_float(mx));
-                        stg[tok * 64 + col] = __half_as_ushort(__float2half_rn(hv * exp2i(-f)));
+                        stg[tok * 64 + col] = __half_as_ushort(__float2half_rn(hv[p] * exp2i(-f)));
                         if ((lane & 23) == 0 && tok < U.nn)   // lane 0 (gate group) or lane 8 (up group)
                             a.hexp_out[(size_t)(U.base + U.n0 + tok) * SUB + 4 * U.mt + q] = (int8_t)f;
                     }
+                };
+                for (int c0 = 32 * half; ok && c0 < U.nr; c0 += 64) {
+                    uint32_t v0[16], v1[16];
+                    const bool two = c0 + 16 < U.nr;
+                    tmem_ld16_nowait(taddr + c0, v0);
+                    if (two) tmem_ld16_nowait(taddr + c0 + 16, v1);
+                    tmem_wait_ld();
+                    glu16(v0, c0);
+                    if (two) glu16(v1, c0 + 16);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
-                named_sync(kBarEpi, 128);
+                named_sync(kBarEpi, kEpiThreads);
                 // coalesced copy-out: 8 threads per 128-byte token row
                 const int cc = et & 7;
-                for (int tok = et >> 3; ok && tok < U.nn; tok += 16) {
+                for (int tok = et >> 3; ok && tok < U.nn; tok += kEpiThreads / 8) {
                     const uint4 val = *reinterpret_cast<const uint4 *>(side + tok * 128 + cc * 16);
                     *reinterpret_cast<uint4 *>(a.h + (size_t)(U.base + U.n0 + tok) * a.I + 64 * U.mt + cc * 8) = val;
                 }
             } else {
                 const int orow = kTM * U.mt + row;
                 const bool valid = orow < a.H;
-                for (int c0 = 0; ok && c0 < U.nr; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + c0, v);
+                float *ob = a.out_acc + orow;
+                auto down16 = [&](const uint32_t(&v)[16], int cb) {
+                    int t16[16];
+                    float s16[16];
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int tok = c0 + jj;
-                        if (valid && tok < U.nn)
-                            red_add_f32(a.out_acc + (size_t)ep_i[tok] * a.H + orow, ep_f[tok] * __uint_as_float(v[jj]));
+                    for (int j = 0; j < 4; ++j) {
+                        const int4 ti4 = *reinterpret_cast<const int4 *>(tk + cb + 4 * j);
+                        const float4 tf4 = *reinterpret_cast<const float4 *>(tf + cb + 4 * j);
+                        t16[4 * j] = ti4.x, t16[4 * j + 1] = ti4.y, t16[4 * j + 2] = ti4.z, t16[4 * j + 3] = ti4.w;
+                        s16[4 * j] = tf4.x, s16[4 * j + 1] = tf4.y, s16[4 * j + 2] = tf4.z, s16[4 * j + 3] = tf4.w;
                     }
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        if (valid && cb + jj < U.nn)
+                            red_add_f32_free(ob + (size_t)t16[jj] * a.H, s16[jj] * __uint_as_float(v[jj]));
+                };
+                for (int c0 = 32 * half; ok && c0 < U.nr; c0 += 64) {
+                    uint32_t v0[16], v1[16];
+                    const bool two = c0 + 16 < U.nr;
+                    tmem_ld16_nowait(taddr + c0, v0);
+                    if (two) tmem_ld16_nowait(taddr + c0 + 16, v1);
+                    tmem_wait_ld();
+                    down16(v0, c0);
+                    if (two) down16(v1, c0 + 16);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(smem_u32(&S.acc_empty[buf]));
             }
+            if (un < nunits) {
+                ep_i[buf ^ 1u][et] = nt_tok;
+                ep_f[buf ^ 1u][et] = nt_sc;
+            }
+            U = Un;
         }
     }
     tc_fence_before();
@@ -636,12 +697,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     }
 }
 
-// Exclusive prefix of the experts' N-tile counts (nt_start[E] = total) and the largest N tile in
-// rows (nt_start[E + 1]); one CTA of 1024 threads.
-__global__ void ntile_scan_kernel(const int32_t *counts, int E, int32_t *nt_start) {
+// Exclusive prefix of the experts' N-tile counts (nt_start[E] = total), the largest N tile in
+// rows (nt_start[E + 1]), the largest tile in bytes (nt_start[E + 2]) and the N-tile table; one
+// CTA of 1024 threads.
+__global__ void ntile_scan_kernel(const int32_t *counts, const int32_t *offsets, const uint8_t *packed, int E,
+                                  int32_t *nt_start, int4 *ntab) {
     __shared__ int warp_tot[32];
     __shared__ int warp_max[32];
+    __shared__ int tb_max;
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    const PackedExpert *pe = reinterpret_cast<const PackedExpert *>(packed + sizeof(PackedHeader));
+    if (e == 0) tb_max = 0;
+    __syncthreads();
+    if (e < E) atomicMax(&tb_max, tile_bytes(pe[e].bits));
     const int n = e < E ? counts[e] : 0;
     const int c = ntile_count(n);
     const int sz = (ntile_size(n) + 15) & ~15;
@@ -673,7 +741,10 @@ __global__ void ntile_scan_kernel(const int32_t *counts, int E, int32_t *nt_star
             nt_start[E] = excl + c;
             nt_start[E + 1] = warp_max[0];
         }
+        const int bits = pe[e].bits, s = ntile_size(n), off = offsets[e];
+        for (int j = 0; j < c; ++j) ntab[excl + j] = make_int4(e | (bits << 16), j * s, min(s, n - j * s), off);
     }
+    if (e == 0) nt_start[E + 2] = tb_max;
 }
 
 // xexp[t]: the exponent that keeps every |x[t] * 2^-xexp[t]| below 2^15 (0 unless some |x| >= 2^15);
@@ -695,13 +766,16 @@ __global__ void xexp_kernel(const uint16_t *x, int T, int H, int32_t *xexp) {
     }
 }
 
-// x16[p] = fp16(x[pair_tok[p]] * 2^-xexp[token]) for every pair p in bucket order; one warp per pair.
+// x16[p] = fp16(x[pair_tok[p]] * 2^-xexp[token]) for every pair p in bucket order, and the
+// pair's column scale 2^xexp[token]; one warp per pair.
 __global__ void x16_gather_kernel(const uint16_t *x, const int32_t *pair_tok, const int32_t *xexp, int P, int H,
-                                  uint16_t *x16) {
+                                  uint16_t *x16, float *pscale) {
     const int lane = threadIdx.x & 31;
     for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
         const int t = __ldg(pair_tok + p);
-        const float sc = exp2i(-__ldg(xexp + t));
+        const int xe = __ldg(xexp + t);
+        const float sc = exp2i(-xe);
+        if (lane == 0) pscale[p] = exp2i(xe);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)p * H);
         for (int i = lane; i < H / 8; i += 32) {
@@ -718,17 +792,19 @@ __global__ void x16_gather_kernel(const uint16_t *x, const int32_t *pair_tok, co
     }
 }
 
-// Brings each pair's h16 to one exponent: fexp[p] = max over its 16-column exponents hexp[p][*],
-// and every block is multiplied by 2^(hexp - fexp) in place (exact unless the block falls into
-// fp16's subnormal range, where its contribution is negligible). One warp per pair.
-__global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, int P, int I, int32_t *fexp) {
+// Brings each pair's h16 to one exponent: f = max over its 16-column exponents hexp[p][*], every
+// block is multiplied by 2^(hexp - f) in place (exact unless the block falls into fp16's
+// subnormal range, where its contribution is negligible), and the pair's column scale for the
+// down GEMM is w_p * 2^f. One warp per pair.
+__global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, const float *pair_w, int P, int I,
+                                   float *pscale) {
     const int lane = threadIdx.x & 31;
     const int SUB = I / 16;
     for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
         int m = -128;
         for (int sb = lane; sb < SUB; sb += 32) m = max(m, (int)hexp[(size_t)p * SUB + sb]);
         m = __reduce_max_sync(0xffffffffu, m);
-        if (lane == 0) fexp[p] = m;
+        if (lane == 0) pscale[p] = __ldg(pair_w + p) * exp2i(m);
         // 8 fp16 per 16-byte chunk, two chunks per 16-column block
         uint4 *row = reinterpret_cast<uint4 *>(h16 + (size_t)p * I);
         for (int ch = lane; ch < I / 8; ch += 32) {
@@ -753,16 +829,17 @@ bool make_row_map(CUtensorMap *map, const void *base, int rows, int cols) {
 template <bool GU>
 moe_status_t launch_tc(const TcArgs &a0, const CUtensorMap &map, const DeviceInfo *dev, cudaStream_t st) {
     TcArgs a = a0;
-    a.smem_bytes = dev->max_smem_optin - (int)sizeof(TcShared) - 2 * kMaxN * 4 - 256;
-    static bool attr_set[64] = {};
+    a.smem_bytes = dev->max_smem_optin - (int)sizeof(TcShared) - 4 * kMaxN * 4 - 256;
+    // the attribute is per device: set once per device, race-free across host threads
+    static std::once_flag once[64];
+    static std::atomic<int> attr_err[64];
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return MOE_ERR_CUDA;
-    if (!attr_set[d]) {
-        if (cudaFuncSetAttribute(tc_grouped_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 a.smem_bytes) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_set[d] = true;
-    }
+    std::call_once(once[d], [&]() {
+        attr_err[d] = cudaFuncSetAttribute(tc_grouped_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           a.smem_bytes) != cudaSuccess;
+    });
+    if (attr_err[d]) return MOE_ERR_CUDA;
     tc_grouped_kernel<GU><<<(unsigned)dev->sms, kTcThreads, a.smem_bytes, st>>>(a, map);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -770,9 +847,9 @@ moe_status_t launch_tc(const TcArgs &a0, const CUtensorMap &map, const DeviceInf
 }  // namespace
 
 moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I, int E, int k, const int32_t *counts,
-                                     const int32_t *offsets, int32_t *nt_start, const int32_t *pair_tok,
-                                     const float *pair_w, const uint16_t *x, uint16_t *x16, int32_t *xexp,
-                                     uint16_t *h16, int8_t *hexp, int32_t *fexp, float *out_acc, uint32_t *status,
+                                     const int32_t *offsets, int32_t *nt_start, int4 *ntab, const int32_t *pair_tok,
+                                     const float *pair_w, float *pscale, const uint16_t *x, uint16_t *x16,
+                                     int32_t *xexp, uint16_t *h16, int8_t *hexp, float *out_acc, uint32_t *status,
                                      cudaStream_t st) {
     const DeviceInfo *dev = device_info();
     if (dev == nullptr) return MOE_ERR_CUDA;
@@ -780,32 +857,28 @@ moe_status_t launch_tc_prefill_gemms(const uint8_t *packed, int T, int H, int I,
     const size_t P = (size_t)T * k;
     CUtensorMap xmap, hmap;
     if (!make_row_map(&xmap, x16, (int)P, H) || !make_row_map(&hmap, h16, (int)P, I)) return MOE_ERR_CUDA;
-    ntile_scan_kernel<<<1, 1024, 0, st>>>(counts, E, nt_start);
+    ntile_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, packed, E, nt_start, ntab);
     xexp_kernel<<<(unsigned)((T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096), 256, 0, st>>>(x, T, H, xexp);
     x16_gather_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(x, pair_tok, xexp, (int)P,
-                                                                                           H, x16);
+                                                                                           H, x16, pscale);
     TcArgs a{};
     a.packed = packed;
     a.H = H;
     a.I = I;
     a.E = E;
-    a.counts = counts;
-    a.offsets = offsets;
     a.nt_start = nt_start;
+    a.ntab = ntab;
     a.pair_tok = pair_tok;
-    a.pair_w = pair_w;
-    a.xexp = xexp;
+    a.pscale = pscale;
     a.h = h16;
     a.hexp_out = hexp;
-    a.fexp = fexp;
     a.out_acc = out_acc;
     a.wait_ns = wait_limit_ns();
     a.status = status;
-    a.act = x16;
     moe_status_t s = launch_tc<true>(a, xmap, dev, st);
     if (s != MOE_OK) return s;
-    h16_rescale_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(h16, hexp, (int)P, I, fexp);
-    a.act = h16;
+    h16_rescale_kernel<<<(unsigned)((P + 7) / 8 < 8192 ? (P + 7) / 8 : 8192), 256, 0, st>>>(h16, hexp, pair_w, (int)P,
+                                                                                            I, pscale);
     s = launch_tc<false>(a, hmap, dev, st);
     if (s != MOE_OK) return s;
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
