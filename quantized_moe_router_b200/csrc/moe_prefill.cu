@@ -78,36 +78,57 @@ __global__ void bucket_scan_kernel(int32_t *blockhist, int nblk, int E, int32_t 
     }
 }
 
-// One warp per token block: pairs in ascending (token, slot) order, so the order inside each
-// expert's bucket is ascending token.
-__global__ void bucket_scatter_kernel(const int32_t *idx, const float *w, int T, int k, int E,
-                                      const int32_t *blockbase, int32_t *pair_tok, float *pair_w) {
-    extern __shared__ int cur[];
-    const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32) cur[e] = blockbase[(size_t)blockIdx.x * E + e];
-    __syncwarp();
+// One CTA of 256 threads per token block: its pairs in rounds of 256 (warp w of a round takes
+// pairs 32w .. 32w+31 of it), ranked inside the warp by match_any and across the round's warps by
+// a per-expert prefix in shared memory, so the order inside each expert's bucket is ascending
+// (token, slot). Shared memory: cur[E] (next free position of each expert), cnt[8][E].
+constexpr int kScatterThreads = 256;
+__global__ void __launch_bounds__(kScatterThreads) bucket_scatter_kernel(const int32_t *idx, const float *w, int T,
+                                                                         int k, int E, const int32_t *blockbase,
+                                                                         int32_t *pair_tok, float *pair_w) {
+    extern __shared__ int sm[];
+    int *cur = sm;
+    int *cnt = sm + E;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < E; e += kScatterThreads) cur[e] = blockbase[(size_t)blockIdx.x * E + e];
     const int t0 = blockIdx.x * kScatterTokens;
-    const int t1 = min(T, t0 + kScatterTokens);
-    for (int base = t0 * k; base < t1 * k; base += 32) {
-        const int p = base + lane;
-        const bool ok = p < t1 * k;
+    const int p0 = t0 * k, p1 = min(T, t0 + kScatterTokens) * k;
+    for (int base = p0; base < p1; base += kScatterThreads) {
+        for (int i = threadIdx.x; i < 8 * E; i += kScatterThreads) cnt[i] = 0;
+        __syncthreads();
+        const int p = base + threadIdx.x;
+        const bool ok = p < p1;
         const int e = ok ? idx[p] : -1 - lane;
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         const int rank = __popc(peers & ((1u << lane) - 1u));
+        if (ok && rank == 0) cnt[wp * E + e] = __popc(peers);
+        __syncthreads();
+        for (int ee = threadIdx.x; ee < E; ee += kScatterThreads) {
+            int run = cur[ee];
+            for (int j = 0; j < 8; ++j) {
+                const int c = cnt[j * E + ee];
+                cnt[j * E + ee] = run;
+                run += c;
+            }
+            cur[ee] = run;
+        }
+        __syncthreads();
         if (ok) {
-            const int pos = cur[e] + rank;
+            const int pos = cnt[wp * E + e] + rank;
             pair_tok[pos] = p / k;
             pair_w[pos] = w[p];
         }
-        __syncwarp();
-        if (ok && rank == 0) cur[e] += __popc(peers);
-        __syncwarp();
+        __syncthreads();
     }
 }
 
-__global__ void convert_kernel(const float *acc, uint16_t *out, size_t n) {
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-        out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i]));
+// out = bf16(acc), four elements per thread and step (n a multiple of 4)
+__global__ void convert_kernel(const float4 *acc, uint2 *out, size_t n4) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = acc[i];
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        out[i] = make_uint2(*reinterpret_cast<const uint32_t *>(&a), *reinterpret_cast<const uint32_t *>(&b));
+    }
 }
 
 }  // namespace
@@ -133,7 +154,7 @@ moe_status_t launch_prefill_route(const uint16_t *x, const float *wr, const floa
     if (w_out && cudaMemcpyAsync(w_out, wt, P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
     bucket_hist_kernel<<<L.nblk, 256, E * sizeof(int), st>>>(idx, T, k, E, bh);
     bucket_scan_kernel<<<1, 1024, 0, st>>>(bh, L.nblk, E, counts, offsets);
-    bucket_scatter_kernel<<<L.nblk, 32, E * sizeof(int), st>>>(idx, wt, T, k, E, bh, ptok, pw);
+    bucket_scatter_kernel<<<L.nblk, kScatterThreads, 9 * E * sizeof(int), st>>>(idx, wt, T, k, E, bh, ptok, pw);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -154,8 +175,11 @@ moe_status_t launch_prefill_experts(const uint16_t *x, const void *packed, int T
         reinterpret_cast<uint16_t *>(w8 + L.h), reinterpret_cast<int8_t *>(w8 + L.hexp), oacc,
         &reinterpret_cast<Control *>(w8)->status, st);
     if (s != MOE_OK) return s;
-    const size_t n = (size_t)T * H;
-    convert_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 256, 0, st>>>(oacc, out, n);
+    const size_t n4 = (size_t)T * H / 4;
+    const DeviceInfo *dev = device_info();
+    if (dev == nullptr) return MOE_ERR_CUDA;
+    const size_t nb = (n4 + 255) / 256 < (size_t)dev->sms * 8 ? (n4 + 255) / 256 : (size_t)dev->sms * 8;
+    convert_kernel<<<(unsigned)nb, 256, 0, st>>>(reinterpret_cast<const float4 *>(oacc), reinterpret_cast<uint2 *>(out), n4);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

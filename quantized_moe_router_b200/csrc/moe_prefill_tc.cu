@@ -8,9 +8,9 @@
 //   * 1 producer warp streams the unit's packed tiles from HBM into a ring of raw slots with 1-D
 //     bulk copies (one per row block and K chunk of up to 4 tiles; the copy engine, not the
 //     load/store path, so the token-row loads below do not queue behind the weight stream);
-//   * 4 dequantiser warps, each taking two of the unit's 8 row blocks per K step (the two tiles'
-//     work interleaves; measured faster than 8 warps of one tile, which compete for issue slots
-//     with the rest of the SM), read their packed 16x64 tiles from the raw slot and write
+//   * 8 dequantiser warps, one of the unit's 8 row blocks each per K step (measured slightly
+//     faster than 4 warps of two row blocks; the dequantisation runs at the SMs' issue rate, so
+//     more warps add little), read their packed 16x64 tiles from the raw slot and write
 //     w = (q - z) * s as fp16 into a 128-byte-swizzled K-major tile A [128 x 64];
 //   * 1 loader thread brings the unit's token rows into a swizzled tile B [N x 64] with 2-D tensor
 //     copies (TMA, 64 rows each, the 128-byte swizzle applied by the copy engine): gate/up reads
@@ -43,8 +43,9 @@ constexpr int kMaxN = 256;                        // tokens per unit (UMMA N lim
 constexpr int kABStages = 3;
 constexpr int kABytes = kTM * 128;                // 128 rows x 64 fp16
 constexpr int kMaxRaw = 8;                        // raw ring slots (K chunks) at most
+constexpr int kDnSkew = 128;                      // extra bytes per down K step in a raw slot (3 x 32 used)
 #ifndef MOE_TC_DQ_WARPS
-#define MOE_TC_DQ_WARPS 4
+#define MOE_TC_DQ_WARPS 8
 #endif
 constexpr int kDqWarps = MOE_TC_DQ_WARPS, kLdWarps = 1;
 constexpr int kBPW = 8 / kDqWarps;                // 16-row blocks of the A tile per dequantiser warp
@@ -300,10 +301,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
     // largest KC that leaves room for 3 slots (at least 2).
     const int tb_max = __ldg(a.nt_start + a.E + 2);
     const long long raw_room = (long long)a.smem_bytes - (long long)pad - (long long)(raw - base);
+    // a down K step in a slot: scale/zero entries, then the four quarters, quarter q shifted by
+    // 32 q bytes so that the lanes (g, t) reading quarter t fall into distinct shared-memory banks
+    const int kstep = GU ? 8 * tb_max : 8 * tb_max + kDnSkew;
     int KC = 1, R = 0;
     for (int kc = 4; kc >= 1; kc >>= 1) {
         if (G.KG % kc) continue;
-        const int r = (int)(raw_room / (8LL * kc * tb_max));
+        const int r = (int)(raw_room / ((long long)kc * kstep));
         if (r >= 3 || kc == 1) {
             KC = kc;
             R = r;
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
         }
     }
     R = R > kMaxRaw ? kMaxRaw : R;
-    const uint32_t slot_bytes = (uint32_t)(8 * KC * tb_max);
+    const uint32_t slot_bytes = (uint32_t)(KC * kstep);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kABStages; ++s) {
@@ -383,8 +387,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                         szp = rawt + kLoBytes + hi_bytes(bits) + 8 * (lane >> 2);
                     } else {
                         const int qb = d_quarter_bytes(bits), g = lane >> 2, t = lane & 3;
-                        const uint8_t *base = raw + (size_t)rs * slot_bytes + (size_t)jk * 8 * tb;
-                        const uint8_t *qp = base + 512 + (size_t)t * 2 * qb + (size_t)(b >> 2) * qb;
+                        const uint8_t *base = raw + (size_t)rs * slot_bytes + (size_t)jk * (8 * tb + kDnSkew);
+                        const uint8_t *qp = base + 512 + (size_t)t * (2 * qb + 32) + (size_t)(b >> 2) * qb;
                         lo16 = qp + (b & 3) * 128 + 16 * g;
                         hip = qp + kLoBytes + (b & 3) * (bits == 8 ? 128 : 64) + (bits == 8 ? 16 : 8) * g;
                         szp = base + (b >> 2) * 256 + (b & 3) * 64 + 8 * g;
@@ -541,10 +545,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(const TcArgs 
                         const int nst = nb / 4, qb = d_quarter_bytes(ex.bits);
                         for (int kk = 0; kk < KC; ++kk) {
                             const uint8_t *blk = mat + (size_t)(k0 + kk) * d_block_bytes(a.H, ex.bits);
-                            uint8_t *dstk = slot + (size_t)kk * 8 * tb;
+                            uint8_t *dstk = slot + (size_t)kk * (8 * tb + kDnSkew);
                             bulk_g2s(smem_u32(dstk), blk + (size_t)2 * U.mt * 256, (uint32_t)(nst * 256), fb);
                             for (int q = 0; q < 4; ++q)
-                                bulk_g2s(smem_u32(dstk + 512 + (size_t)q * 2 * qb),
+                                bulk_g2s(smem_u32(dstk + 512 + (size_t)q * (2 * qb + 32)),
                                          blk + d_quarter_offset(a.H, ex.bits, q) + (size_t)2 * U.mt * qb,
                                          (uint32_t)(nst * qb), fb);
                         }
