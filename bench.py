@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-ties", action="store_true", help="skip the near-tie count against the oracle")
     ap.add_argument("--layers", type=int, default=0,
                     help="stack only this many layers of the workload (smaller case for profiling)")
+    ap.add_argument("--next", action="store_true",
+                    help="with --only: also time the next rows (quantiser, streamed decode, mixed prefill)")
     ap.add_argument("--seq", type=int, default=0,
                     help="decode steps per bench step (default: the workload's own count)")
     return ap.parse_args()
@@ -711,6 +713,180 @@ def prefill_leg(args, w, world, rank):
     return res
 
 
+
+# ------------------------------------------------------------------------------ next rows
+
+# fp64 issue rate of the part: 148 SMs x 64 fp64 lanes x 1.965 GHz, one operation per lane and clock
+FP64_OPS_PEAK = 148 * 64 * 1.965e9
+
+
+def quantizer_leg():
+    """moe_quantize_hqq on whole expert matrices (published defaults p = 0.7, beta = 10,
+    kappa = 1.01, 20 steps): weights per second, and the fp64 operations of its definition per
+    second against the fp64 issue rate. Per weight, an error pass is 10 operations (3 of them a
+    division, rint and clamps counted as one each) and a zero pass 15 (2 divisions); a group
+    that ran n steps did n error passes and at least n - 1 zero passes (counted: n - 1)."""
+    import torch
+    import oracle
+    import synth
+    import quantized_moe_router_b200 as qm
+    res = {}
+    gen = torch.Generator(device="cuda")
+    for label, rows, cols, bits in (("gate_up_I512xH2048_64experts_int4", 64 * 512, 2048, 4),
+                                    ("down_H2048xI512_64experts_int8", 64 * 2048, 512, 8),
+                                    ("gate_up_I1024xH4096_16experts_int4", 16 * 1024, 4096, 4)):
+        gen.manual_seed(rows + cols + bits)
+        wt = (torch.randn((rows, cols), generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        qm.quantize_hqq(wt, bits, with_iters=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record()
+        for _ in range(reps):
+            codes, sc, zr, it = qm.quantize_hqq(wt, bits, with_iters=True)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3 / reps
+        steps = it.to(torch.int64)
+        ops = 64.0 * float((10 * steps + 15 * (steps - 1).clamp(min=0)).sum())
+        ent = {"weights": rows * cols, "bits": bits, "ms": t * 1e3, "weights_per_s": rows * cols / t,
+               "mean_steps": float(steps.float().mean()),
+               "roofline": {"bound": "alu", "achieved": ops / t / 1e12, "peak": FP64_OPS_PEAK / 1e12,
+                            "unit": "T fp64 op/s", "frac": ops / t / FP64_OPS_PEAK, "traffic": None,
+                            "peak_source": "148 SMs x 64 fp64 lanes x 1.965 GHz (nominal issue rate)"}}
+        if label.startswith("gate_up_I512"):
+            # stored zeros against the oracle on the first 512 rows (one expert's gate matrix)
+            wb = wt[:512].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+            _, rs, rz, rit = oracle.get().hqq_quantize(wb, bits)
+            z16 = zr[:512].cpu().numpy().view(np.uint16)
+            zsame = synth.f16_bits_to_f64(z16) == synth.f16_bits_to_f64(rz)
+            ent["oracle_check"] = {"groups": int(zsame.size), "zero_mismatch": int((~zsame).sum()),
+                                   "scale_equal": bool(np.array_equal(sc[:512].cpu().numpy().view(np.uint16), rs)),
+                                   "steps_equal": bool(np.array_equal(it[:512].cpu().numpy(), rit))}
+        res[label] = ent
+        del wt, codes, sc, zr, it
+    torch.cuda.empty_cache()
+    return res
+
+
+def streamed_leg(slot_counts=(96, 256, 640), L=4, S=4):
+    """Decode through an ExpertCache: the layers of the mixed 4/6/8-bit Zipf workload stay in
+    pinned host memory, a device pool of `slots` experts serves the calls. Per call the routing
+    names the experts (moe_route_topk), the missing ones are copied (moe_cache_commit) and the
+    fused decode kernel reads them through the layer's cache header. Two schedules: serial
+    (route, copy, compute per layer) and overlapped (the next layer's copies on a second stream
+    while this layer computes; the benchmark's inputs are independent per layer, so the next
+    layer's routing is known a layer ahead -- a model would need a predictor for it)."""
+    import torch
+    import synth
+    import synth.device as sd
+    import quantized_moe_router_b200 as qm
+    w = synth.WORKLOADS["decode_t16_l24_h2048_e256_k8_i768_mixed468_zipf1.1"]
+    host, wrs, biases, bits = [], [], [], []
+    for l in range(L):
+        b = synth.expert_bits(w, l)
+        experts = [sd.expert_tensors(w, l, e, int(b[e])) for e in range(w.E)]
+        host.append(qm.pack_layer(experts, w.H, w.I).cpu().pin_memory())
+        del experts
+        wrs.append(sd.router_weights(w, l))
+        bb = synth.router_bias(w, l)
+        biases.append(None if bb is None else torch.from_numpy(bb).cuda())
+        bits.append(b)
+    torch.cuda.empty_cache()
+    xs = [[sd.hidden(w, s, l) for l in range(L)] for s in range(S + 1)]
+    nbytes = [[expert_bytes(w.H, w.I, int(bits[l][e])) for e in range(w.E)] for l in range(L)]
+    ws = qm.workspace(w.T, w.H, w.I, w.E, w.k, qm.MODE_DECODE)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((w.T, w.k), dtype=torch.float32, device="cuda")
+    # every call's routing, for the requests (the fused kernel routes again; the two must agree)
+    routes = [[None] * L for _ in range(S + 1)]
+    for s in range(S + 1):
+        for l in range(L):
+            qm.route_topk(xs[s][l], wrs[l], biases[l], w.k, idx_out=idx, w_out=wts)
+            routes[s][l] = sorted(set(idx.cpu().flatten().tolist()))
+    comp = torch.cuda.current_stream()
+    cst = torch.cuda.Stream()
+    res = {}
+    for slots in slot_counts:
+        ent = {}
+        for sched in ("serial", "overlapped"):
+            cache = qm.ExpertCache(host, slots, keep_recent=2)
+            outside = 0
+
+            def run(s, count):
+                nonlocal outside
+                loaded = 0
+                pk = [None] * L
+                ev = [None] * L
+
+                def fetch(l, stream):
+                    nonlocal loaded
+                    le, _ = cache.request(l, routes[s][l])
+                    loaded += sum(nbytes[l][e] for e in le)
+                    pk[l] = cache.commit(stream)
+                    ev[l] = torch.cuda.Event()
+                    ev[l].record(stream)
+                done = [None] * L
+                if sched == "overlapped":
+                    cst.wait_stream(comp)
+                    fetch(0, cst)
+                for l in range(L):
+                    if sched == "serial":
+                        fetch(l, comp)
+                    comp.wait_event(ev[l])
+                    qm.forward_decode(xs[s][l], wrs[l], biases[l], pk[l], w.I, w.E, w.k, ws, out=out,
+                                      idx_out=idx, w_out=wts, stream=comp)
+                    done[l] = torch.cuda.Event()
+                    done[l].record(comp)
+                    if sched == "overlapped" and l + 1 < L:
+                        # keep_recent = 2 protects this layer's experts and the next one's; the
+                        # copies wait until the call before this one has read its experts
+                        if l >= 1:
+                            cst.wait_event(done[l - 1])
+                        fetch(l + 1, cst)
+                    if count and not set(idx.cpu().flatten().tolist()) <= set(routes[s][l]):
+                        outside += 1
+                return loaded
+            run(S, False)   # warm: the first pass fills the pool
+            torch.cuda.synchronize()
+            h0 = cache.stats()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0 = time.perf_counter()
+            e0.record(comp)
+            loaded = sum(run(s, False) for s in range(S))
+            e1.record(comp)
+            torch.cuda.synchronize()
+            wall = time.perf_counter() - t0
+            dev = e0.elapsed_time(e1) * 1e-3
+            h1 = cache.stats()
+            hits, miss = h1["hits"] - h0["hits"], h1["misses"] - h0["misses"]
+            # the fused kernel's own routing against the requests, outside the timed region
+            run(S, True)
+            torch.cuda.synchronize()
+            assert qm.device_status(ws) == qm.MOE_OK
+            ent[sched] = {"tokens_per_s": w.T * S / dev, "ms_per_token_step": dev / S * 1e3,
+                          "host_GBps": loaded / dev / 1e9, "hit_rate": hits / max(1, hits + miss),
+                          "expert_misses": miss, "wall_s": wall, "calls_outside_request": outside}
+            cache.close()
+        res[f"slots_{slots}"] = ent
+    return {"workload": f"{w.name} (first {L} layers in pinned host memory, {w.T} tokens per call, {S} steps)",
+            "experts_in_play": L * w.E, "schedules": res}
+
+
+def next_rows_leg(args, world, rank):
+    import dataclasses
+    import synth
+    pw = synth.WORKLOADS[PREFILL_WORKLOAD]
+    mixed = dataclasses.replace(pw, name="prefill_t4096_l2_h2048_e256_k8_i512_mixed468", mixed_bits=True, layers=2)
+    a2 = argparse.Namespace(**vars(args))
+    a2.no_cpu_baseline = True
+    a2.steps = min(args.steps, 5)
+    return {"quantizer": quantizer_leg(),
+            "streamed_decode": streamed_leg(),
+            "mixed_prefill": prefill_leg(a2, mixed, world, rank)}
+
+
 def leg(args, w, world, rank):
     if w.mode == "prefill":
         return prefill_leg(args, w, world, rank)
@@ -737,6 +913,8 @@ def run_ours(args, w):
     line.update(head)
     if others:
         line["configs"] = others
+    if args.next or not args.only:
+        line["next_rows"] = next_rows_leg(args, world, rank)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

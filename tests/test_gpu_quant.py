@@ -70,11 +70,13 @@ def check_quantizer(w_bits, bits, exact=False, **prm):
     same_cols = np.repeat(zsame, G, 1)
     assert np.array_equal(q[same_cols], rq[same_cols].astype(np.int64)), "codes differ where zeros agree"
     nbad = int((~zsame).sum())
+    print(f"stored zeros differing from the oracle: {nbad} of {zsame.size} groups")
     if exact:
         assert nbad == 0, nbad
     # a CPU model of this kind of difference moved about 1 zero in 2000 groups (fp16 midpoints);
-    # the cap only catches a systematic divergence, each differing group is checked below
-    assert nbad <= max(4, zsame.size // 200), f"{nbad} of {zsame.size} stored zeros differ"
+    # on a B200 none of the ~120,000 groups of these tests differed. The cap catches anything
+    # above that model's rate; each differing group is checked below
+    assert nbad <= max(2, zsame.size // 2000), f"{nbad} of {zsame.size} stored zeros differ"
     if nbad:
         w = synth.bf16_bits_to_f32(w_bits).astype(np.float64)
         for r, g in zip(*np.nonzero(~zsame)):
