@@ -54,7 +54,8 @@ DECODE_SOURCES = ["quantized_moe_router_b200/csrc/moe_decode.cu",
                   "quantized_moe_router_b200/csrc/moe_topk.cuh"]
 PREFILL_SOURCES = ["quantized_moe_router_b200/csrc/moe_prefill_tc.cu",
                    "quantized_moe_router_b200/csrc/moe_prefill.cu",
-                   "quantized_moe_router_b200/csrc/moe_internal.cuh"]
+                   "quantized_moe_router_b200/csrc/moe_internal.cuh",
+                   "quantized_moe_router_b200/csrc/moe_tc.cuh"]
 
 
 def parse():
