@@ -4,7 +4,7 @@
 // This is the "MoE megakernel" of the page "Raon-1-mini ... RTX 5070 Ti" (table row: one
 // persistent kernel for each layer's expert block) with the "pipelined megakernel" row's
 // overlap (the next weights are in flight while the current ones are multiplied), laid out for
-// sm_100a. One CTA per SM: 16 consumer warps and one control warp.
+// sm_100a. One CTA per SM: 16 consumer warps (8 above 16 tokens) and one control warp.
 //   * Prologue, before the programmatic-dependent-launch wait (it overlaps the previous
 //     layer): mbarrier set-up, this CTA's router rows copied into shared memory, the packed
 //     layer's expert table read. Both are weights, never produced by the previous launch.
@@ -26,9 +26,10 @@
 //     mma.sync on bf16 operands made from the codes by one LOP3 per register (exact integers
 //     128 + q), the group's scale and zero applied in fp32; the warps' partial sums meet in shared
 //     memory, and one warp per 8 tokens forms h = silu(g) * u as a bf16 hi + lo pair.
-//   * Down: super-tile st (64 output rows) of the unit's quarter goes to warp st % 16; w * y is
-//     accumulated in registers across the CTA's units (one token: all of them; several tokens: the
-//     units of one expert) and added into the fp32 output accumulator once.
+//   * Down: super-tile st (64 output rows) of the unit's quarter goes to warp st % 16. One token:
+//     w * y is accumulated in shared memory across all of the CTA's units and added into the fp32
+//     output accumulator once, four rows per vector reduction. Several tokens: each super-tile's
+//     w * y is added into the accumulator as soon as it is computed.
 //   * Completion: one counter per 256 output rows; the CTA that completes a row group converts it
 //     to bf16 and clears it for the next call.
 // Every wait is bounded; on expiry the kernel records MOE_ERR_TIMEOUT in the workspace, the
