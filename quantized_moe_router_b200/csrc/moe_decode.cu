@@ -42,6 +42,9 @@
 namespace moe {
 namespace {
 
+#ifndef MOE_DECODE_GROUPS
+#define MOE_DECODE_GROUPS 2                 // consumer groups up to 16 tokens
+#endif
 constexpr int kMaxCW = 16;                  // consumer warps at most (+ one control warp)
 constexpr int kMaxWarps = kMaxCW + 1;
 constexpr int kSlice = 16;                  // intermediate rows per work unit
@@ -116,7 +119,7 @@ struct DecodeLayout {
     size_t xs, xsum, gred, hbuf, hcol, ycta, ring, total;
     int stages;
 };
-template <int NT, int CW>
+template <int NT, int CW, int NG>
 DecodeLayout decode_layout(int T, int H, int smem_limit) {
     DecodeLayout L;
     size_t o = align_up(sizeof(DecodeSmem), 128);
@@ -126,12 +129,12 @@ DecodeLayout decode_layout(int T, int H, int smem_limit) {
     o += align_up((size_t)T * (H / kGroup) * 4, 128);
     L.gred = o;                                   // gate/up partial sums of each warp [CW][2][NT][4][32] fp32
     o += (size_t)CW * 2 * NT * 4 * 32 * 4;
-    L.hbuf = o;                                   // h hi / lo [2][NT][8 pairs][16] bf16
-    o += (size_t)2 * NT * 8 * 16 * 2;
-    L.hcol = o;                                   // h of each of the 16 rows and pair columns [16][NT x 8] fp32
-    o += (size_t)16 * NT * 8 * 4;
-    L.ycta = o;                                   // one token: the CTA's output rows [H] fp32
-    if (T == 1) o += align_up((size_t)H * 4, 128);
+    L.hbuf = o;                                   // per consumer group: h hi / lo [2][NT][8 pairs][16] bf16
+    o += (size_t)NG * 2 * NT * 8 * 16 * 2;
+    L.hcol = o;                                   // per group: h of each of the 16 rows and pair columns [16][NT x 8] fp32
+    o += (size_t)NG * 16 * NT * 8 * 4;
+    L.ycta = o;                                   // one token, per group: the CTA's output rows [H] fp32
+    if (T == 1) o += (size_t)NG * align_up((size_t)H * 4, 128);
     L.ring = align_up(o, 128);
     const long long room = (long long)min(smem_limit, kSmemBudget) - (long long)L.ring;
     L.stages = room > 0 ? (int)(room / kStageBytes) : 0;
@@ -152,6 +155,24 @@ __device__ __forceinline__ bool consumer_sync_or(bool flag) {
         "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)flag), "n"(CW * 32)
+        : "memory");
+    return r != 0;
+}
+// Named barriers 3 and 4: the two consumer groups (NG = 2, CW / 2 warps each); with one group the
+// consumer barrier 1.
+template <int NG, int CW>
+__device__ __forceinline__ void group_sync(int gi) {
+    if (NG == 1) consumer_sync<CW>();
+    else asm volatile("bar.sync %0, %1;" ::"r"(3 + gi), "n"(CW / NG * 32) : "memory");
+}
+template <int NG, int CW>
+__device__ __forceinline__ bool group_sync_or(int gi, bool flag) {
+    if (NG == 1) return consumer_sync_or<CW>(flag);
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)flag), "r"(3 + gi), "n"(CW / NG * 32)
         : "memory");
     return r != 0;
 }
@@ -952,19 +973,20 @@ __device__ __forceinline__ void emit_st(const DecodeArgs &a, const DecodeSmem &S
 // NT: MMA n-tiles (8 tokens each) per unit; CW: consumer warps; STW: how a warp keeps the output
 // rows of its super-tiles across units: > 0, in registers, STW super-tiles per warp (several
 // tokens: the units of one expert slot); 0, not at all (each super-tile's rows are added out at
-// once); -1, in shared memory (one token: all units of the CTA).
-template <int NT, int STW, int CW>
+// once); -1, in shared memory (one token: all units of the CTA). NG: consumer groups; with two,
+// group i (CW / 2 warps) runs the CTA's units i, i + 2, ... with its own barriers and h buffers,
+// so that one group's barriers and SiLU-GLU overlap the other group's multiplications.
+template <int NT, int STW, int CW, int NG>
 __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeArgs a, const DecodeLayout L) {
     constexpr int kCW = CW, kPW = CW, kWarps = CW + 1, kThreads = kWarps * 32;
+    constexpr int GW = CW / NG;   // warps per consumer group
+    static_assert(NG == 1 || (NG == 2 && STW <= 0), "two groups: no register carry of output rows");
     extern __shared__ __align__(128) uint8_t dyn[];
     DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(dyn);
     uint8_t *ring = dyn + L.ring;
     float *Xs = reinterpret_cast<float *>(dyn + L.xsum);
     float *gred = reinterpret_cast<float *>(dyn + L.gred);
-    uint16_t *hhi = reinterpret_cast<uint16_t *>(dyn + L.hbuf);
-    uint16_t *hlo = hhi + NT * 8 * 16;
-    float *hrow = reinterpret_cast<float *>(dyn + L.hcol);
-    float *ycta = reinterpret_cast<float *>(dyn + L.ycta);
+    float *ycta_all = reinterpret_cast<float *>(dyn + L.ycta);
     const int NS = L.stages;
     const int T = a.T, H = a.H, E = a.E, K = a.k, P = T * K;
     const int G = H / kGroup, nst = H / 64;
@@ -1007,7 +1029,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     }
     if (threadIdx.x < 3) S.wplan[threadIdx.x] = make_width_plan(H, a.I, 4 + 2 * threadIdx.x);
     if (STW < 0)
-        for (int i = threadIdx.x; i < H; i += kThreads) ycta[i] = 0.f;
+        for (int i = threadIdx.x; i < NG * H; i += kThreads) ycta_all[i] = 0.f;
     // the router bias of this CTA's rows (a weight), off the logits' critical path
     if (threadIdx.x < ne && threadIdx.x < kBiasRows) S.bias[threadIdx.x] = a.bias ? a.bias[c + threadIdx.x * nC] : 0.f;
     __syncthreads();
@@ -1197,6 +1219,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     // ---------------------------------------------------------------- consumers
     plan_ready_wait<CW>();
     const int g = lane >> 2, t = lane & 3;
+    const int cg = NG == 1 ? 0 : warp / GW;    // this warp's consumer group
+    const int gw = warp - cg * GW;             // and its warp within the group
+    uint16_t *hhi = reinterpret_cast<uint16_t *>(dyn + L.hbuf) + (size_t)cg * 2 * NT * 8 * 16;
+    uint16_t *hlo = hhi + NT * 8 * 16;
+    float *hrow = reinterpret_cast<float *>(dyn + L.hcol) + (size_t)cg * 16 * NT * 8;
+    float *ycta = ycta_all + (size_t)cg * H;
     // one token (STW = -1): only accumulator column 0 holds a pair, and the output rows are added
     // into shared memory
     constexpr bool ONE = STW < 0;
@@ -1235,8 +1263,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             par ^= 1u;
         }
     };
+    // the lanes leave the bounded poll at different iterations: the vote makes the outcome
+    // warp-uniform and reconverges the warp before its next aligned instruction (mma.sync, bar)
     auto wait_full = [&]() {
         if (!bad && (S.abort || !mbar_wait_idle(smem_u32(&S.full[s]), par, a.wait_ns, status))) bad = true;
+        bad = __any_sync(0xffffffffu, bad);
     };
     auto release_stage = [&]() {
         __syncwarp();
@@ -1248,6 +1279,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     for (int u = S.u0; u < S.u1; ++u) {
         const int bits = S.ubits[uj];
         const WidthPlan w = S.wplan[width_index(bits)];
+        if (NG > 1 && ((u - S.u0) & (NG - 1)) != cg) {
+            // the other group's unit: every consumer warp still waits for each chunk and releases
+            // it (without reading it), so that both groups pass the ring's stages in order: a
+            // stage's phase parity only tells consecutive phases apart, and a group more than one
+            // phase ahead of or behind a stage would misread it
+            for (int ch = 0; ch < w.ngc + w.ndc; ++ch) {
+                wait_full();
+                release_stage();
+            }
+            if (++ui == sp) {
+                ui = 0;
+                ++uj;
+            }
+            continue;
+        }
         if (uj != cur) {
             if (T > 1 && cur >= 0 && !bad) flush_slot();
             cur = uj;
@@ -1280,9 +1326,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 int k0, k1;
                 chunk_items(w.gbase, w.grem, ch, k0, k1);
                 const uint8_t *stg = ring + (size_t)s * kStageBytes;
-                if (bits == 4) gu_chunk<4, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
-                else if (bits == 6) gu_chunk<6, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
-                else gu_chunk<8, NT, CW, ONE>(stg, k0, k1, warp, jc, lane, gacc);
+                if (bits == 4) gu_chunk<4, NT, GW, ONE>(stg, k0, k1, gw, jc, lane, gacc);
+                else if (bits == 6) gu_chunk<6, NT, GW, ONE>(stg, k0, k1, gw, jc, lane, gacc);
+                else gu_chunk<8, NT, GW, ONE>(stg, k0, k1, gw, jc, lane, gacc);
             }
             release_stage();
         }
@@ -1296,27 +1342,27 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
 #pragma unroll
                     for (int i = 0; i < 4; ++i) gw[((rb * NT + nt) * 4 + i) * 32] = gacc[rb][nt][i];
         }
-        if (consumer_sync_or<CW>(bad || S.abort)) {
+        if (group_sync_or<NG, CW>(cg, bad || S.abort)) {
             aborted = true;
             break;
         }
-        // SiLU-GLU, one intermediate row k of the unit per warp (warps k, k + CW), one pair column
-        // per lane: the gate and up sums over the warps' partials, h as a bf16 hi + lo pair, and
-        // hi + lo of every (row, column) for the down step's correction sums.
-        for (int k = warp; k < 16; k += kCW) {
+        // SiLU-GLU, one intermediate row k of the unit per warp of the group (warps k, k + GW),
+        // one pair column per lane: the gate and up sums over the group's partials, h as a bf16
+        // hi + lo pair, and hi + lo of every (row, column) for the down step's correction sums.
+        for (int k = gw; k < 16; k += GW) {
             if (lane < 8 * NT) {
                 const int nt = lane >> 3, pcol = lane & 7;
                 const int rb = k >> 3, src = ((k & 7) << 2) + (pcol >> 1), col = pcol & 1;
-                const float *gp = gred + ((rb * NT + nt) * 4 + col) * 32 + src;
+                const float *gp = gred + (size_t)cg * GW * 2 * NT * 4 * 32 + ((rb * NT + nt) * 4 + col) * 32 + src;
                 // the warps' partials, summed as a tree (all loads first)
-                float gv[kCW], uv[kCW];
+                float gv[GW], uv[GW];
 #pragma unroll
-                for (int w2 = 0; w2 < kCW; ++w2) {
+                for (int w2 = 0; w2 < GW; ++w2) {
                     gv[w2] = gp[(size_t)w2 * 2 * NT * 4 * 32];
                     uv[w2] = gp[(size_t)w2 * 2 * NT * 4 * 32 + 2 * 32];
                 }
 #pragma unroll
-                for (int h = kCW / 2; h > 0; h >>= 1)
+                for (int h = GW / 2; h > 0; h >>= 1)
 #pragma unroll
                     for (int w2 = 0; w2 < h; ++w2) {
                         gv[w2] += gv[w2 + h];
@@ -1332,7 +1378,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                 hrow[k * NT * 8 + lane] = __bfloat162float(hi) + __bfloat162float(lo);
             }
         }
-        consumer_sync<CW>();
+        group_sync<NG, CW>(cg);
         DnCtx<NT> dc;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -1372,7 +1418,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
             dc.w0[nt] = q0 < cur_nj ? S.pw[cur_pf + q0] : 0.f;
             dc.w1[nt] = q1 < cur_nj ? S.pw[cur_pf + q1] : 0.f;
         }
-        // down: super-tile st of the unit's quarter goes to warp st % kCW
+        // down: super-tile st of the unit's quarter goes to warp st % GW of the group
         for (int ch = 0; ch < ndc; ++ch) {
             wait_full();
             if (!bad) {
@@ -1391,7 +1437,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
                         }
                     }
                 } else {
-                    for (int st = s0 + ((warp - s0) % kCW + kCW) % kCW; st < s1; st += kCW) {
+                    for (int st = s0 + ((gw - s0) % GW + GW) % GW; st < s1; st += GW) {
                         const uint32_t zp = zb + (uint32_t)((st - s0) * 256), qp = qbase + (uint32_t)((st - s0) * qb);
                         if (bits == 4) down_st<4, NT, ONE>(zp, qp, dc, lane, yacc[0]);
                         else if (bits == 6) down_st<6, NT, ONE>(zp, qp, dc, lane, yacc[0]);
@@ -1419,8 +1465,17 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         if (STW < 0) {
             // one token: the CTA's rows, one vector addition per 4 rows
             consumer_sync<CW>();
-            for (int i = threadIdx.x; i < H / 4; i += kCW * 32)
-                red_add_v4_f32(a.out_acc + 4 * i, *reinterpret_cast<const float4 *>(ycta + 4 * i));
+            for (int i = threadIdx.x; i < H / 4; i += kCW * 32) {
+                float4 v = reinterpret_cast<const float4 *>(ycta_all)[i];
+                if (NG > 1) {
+                    const float4 v2 = reinterpret_cast<const float4 *>(ycta_all + H)[i];
+                    v.x += v2.x;
+                    v.y += v2.y;
+                    v.z += v2.z;
+                    v.w += v2.w;
+                }
+                red_add_v4_f32(a.out_acc + 4 * i, v);
+            }
         } else if (STW > 0) {
             flush_slot();
         }
@@ -1469,9 +1524,9 @@ void logit_copies(int T, int E, int &rep, int &stride) {
     while (rep < 32 && (size_t)(rep * 2) * stride <= (size_t)kMaxT * kMaxE) rep *= 2;
 }
 
-template <int NT, int STW, int CW>
+template <int NT, int STW, int CW, int NG>
 moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t st) {
-    const DecodeLayout L = decode_layout<NT, CW>(a.T, a.H, dev->max_smem_optin);
+    const DecodeLayout L = decode_layout<NT, CW, NG>(a.T, a.H, dev->max_smem_optin);
     if (L.stages < 2) return MOE_ERR_UNSUPPORTED;
     // the kernel attribute, once per device (concurrent first calls from several host threads
     // set the same value; the flag is atomic)
@@ -1479,7 +1534,7 @@ moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t 
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return MOE_ERR_CUDA;
     if (!attr_set[d].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(decode_kernel<NT, STW, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(decode_kernel<NT, STW, CW, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dev->max_smem_optin) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_set[d].store(true, std::memory_order_release);
@@ -1494,7 +1549,7 @@ moe_status_t launch_nt(const DecodeArgs &a, const DeviceInfo *dev, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_kernel<NT, STW, CW>, a, L) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<NT, STW, CW, NG>, a, L) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
@@ -1532,10 +1587,10 @@ moe_status_t launch_decode(const uint16_t *x, const float *wr, const float *bias
     }
     // One token: 16 consumer warps, the CTA's output rows in shared memory. Several tokens: every
     // super-tile's rows are added into the output at once.
-    if (T == 1) return launch_nt<1, -1, 16>(a, dev, st);
-    if (T <= 8) return launch_nt<1, 0, 16>(a, dev, st);
-    if (T <= 16) return launch_nt<2, 0, 16>(a, dev, st);
-    return launch_nt<4, 0, 8>(a, dev, st);
+    if (T == 1) return launch_nt<1, -1, 16, MOE_DECODE_GROUPS>(a, dev, st);
+    if (T <= 8) return launch_nt<1, 0, 16, MOE_DECODE_GROUPS>(a, dev, st);
+    if (T <= 16) return launch_nt<2, 0, 16, MOE_DECODE_GROUPS>(a, dev, st);
+    return launch_nt<4, 0, 8, 1>(a, dev, st);
 }
 
 }  // namespace moe
