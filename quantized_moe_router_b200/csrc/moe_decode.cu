@@ -4,7 +4,10 @@
 // This is the "MoE megakernel" of the page "Raon-1-mini ... RTX 5070 Ti" (table row: one
 // persistent kernel for each layer's expert block) with the "pipelined megakernel" row's
 // overlap (the next weights are in flight while the current ones are multiplied), laid out for
-// sm_100a. One CTA per SM: 16 consumer warps (8 above 16 tokens) and one control warp.
+// sm_100a. One CTA per SM: 16 consumer warps (8 above 16 tokens) and one control warp. Up to 16
+// tokens the consumers form two groups of eight warps that take alternate work units, each with
+// its own barriers and h buffers, so that one group's barriers and SiLU-GLU overlap the other
+// group's multiplications.
 //   * Prologue, before the programmatic-dependent-launch wait (it overlaps the previous
 //     layer): mbarrier set-up, this CTA's router rows copied into shared memory, the packed
 //     layer's expert table read. Both are weights, never produced by the previous launch.
@@ -21,7 +24,7 @@
 //     one contiguous range per CTA with equal bytes.
 //   * Streaming. The control warp issues the bulk copies of its range's weights (a unit is three
 //     contiguous pieces: gate/up tiles, the down quarter, the down scale/zero entries) into a ring
-//     of 32 KB stages as soon as the selection is known; consumers free stages as they go.
+//     of 48 KB stages as soon as the selection is known; consumers free stages as they go.
 //   * Gate/up: tile kg of the unit goes to consumer warp kg % 16 (split K), multiplied with
 //     mma.sync on bf16 operands made from the codes by one LOP3 per register (exact integers
 //     128 + q), the group's scale and zero applied in fp32; the warps' partial sums meet in shared
@@ -48,7 +51,7 @@ namespace {
 constexpr int kMaxCW = 16;                  // consumer warps at most (+ one control warp)
 constexpr int kMaxWarps = kMaxCW + 1;
 constexpr int kSlice = 16;                  // intermediate rows per work unit
-constexpr int kStageBytes = 32768;          // bytes per ring stage
+constexpr int kStageBytes = 49152;          // bytes per ring stage (measured: 24 KB and 32 KB slower)
 constexpr int kMaxStages = 8;
 constexpr int kActBytes = 65536;            // x of all tokens in shared memory (more: read through L2)
 constexpr int kMaxP = kDecodeMaxP;
