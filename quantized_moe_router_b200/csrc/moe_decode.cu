@@ -417,14 +417,14 @@ __device__ __forceinline__ int slot_of(const DecodeSmem &S, int e) {
 }
 
 // Expert slots of one token (P = k <= 32 pairs, distinct experts): slot j is selection j.
-__device__ __forceinline__ void plan_single(DecodeSmem &S, int P, int lane) {
+__device__ __forceinline__ void plan_single(DecodeSmem &S, int P, int lane, bool weights) {
     if (lane < P) {
         const int e = S.sel_idx[lane];
         S.ubits[lane] = S.ebits[e];
         S.uoff[lane] = S.eoff[e];
         S.pfirst[lane] = lane;
         S.ptok[lane] = 0;
-        S.pw[lane] = S.sel_w[lane];
+        if (weights) S.pw[lane] = S.sel_w[lane];
     }
     if (lane == 0) {
         S.U = P;
@@ -640,6 +640,12 @@ __device__ __forceinline__ void topk_one_rank(const DecodeArgs &a, DecodeSmem &S
     if (rank < a.k) S.selk[rank] = x;
 }
 // Phase 3 (one warp, after a barrier): indices and softmax weights of the selection.
+// The selection in order from the ranked keys (the control warp), before the weights.
+__device__ __forceinline__ void topk_one_select(const DecodeArgs &a, DecodeSmem &S, int lane) {
+    if (lane < a.k) S.sel_idx[lane] = (int)(0xFFFFFFFFu - (uint32_t)S.selk[lane]);
+    __syncwarp();
+}
+// The softmax weights of the selection (also the slots' pair weights; idx_out / w_out from CTA 0).
 __device__ __forceinline__ void topk_one_finish(const DecodeArgs &a, DecodeSmem &S, int lane, int c) {
     const int K = a.k;
     const unsigned long long mine = lane < K ? S.selk[lane] : 0ull;
@@ -653,8 +659,8 @@ __device__ __forceinline__ void topk_one_finish(const DecodeArgs &a, DecodeSmem 
     if (lane < K) {
         const int e = (int)(0xFFFFFFFFu - (uint32_t)mine);
         const float w = ex / sum;
-        S.sel_idx[lane] = e;
         S.sel_w[lane] = w;
+        S.pw[lane] = w;
         if (c == 0 && a.idx_out) a.idx_out[lane] = e;
         if (c == 0 && a.w_out) a.w_out[lane] = w;
     }
@@ -1148,13 +1154,15 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
     }
     if (warp == kPW) {
         __syncwarp();
-        if (one && !S.abort) topk_one_finish(a, S, lane, c);
-        const int Pp = S.abort ? 0 : P;
-        if (T == 1) plan_single(S, Pp, lane);
+        // one token: the slots and the unit cut from the ranked selection, the first copies, and
+        // only then the softmax weights (the consumers need them for the down step, the copies
+        // do not)
+        const bool sel_ok = !S.abort;
+        if (one && sel_ok) topk_one_select(a, S, lane);
+        const int Pp = sel_ok ? P : 0;
+        if (T == 1) plan_single(S, Pp, lane, !one);
         else plan_many(a, S, Pp, lane);
         plan_units(a, S, lane, c, nC);
-        // hand the plan to the consumer warps and start streaming without waiting for them
-        plan_ready_arrive<CW>();
         // ------------------------------------------------------------ producer
         // The copies of chunk cc (in unit order) go to stage cc % NS. The first NS chunks find
         // every stage free: lane cc issues chunk cc, all at once; lane 0 then issues the rest,
@@ -1209,6 +1217,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, 1) decode_kernel(const __grid_c
         };
         walk(true);
         __syncwarp();
+        if (one && sel_ok) topk_one_finish(a, S, lane, c);
+        // hand the plan to the consumer warps and stream the rest without waiting for them
+        plan_ready_arrive<CW>();
         if (lane != 0) return;
         cc = 0;
         walk(false);
