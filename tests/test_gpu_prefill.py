@@ -28,7 +28,8 @@ def prefill_call(layer, x_bits, I, E, k):
 @pytest.mark.parametrize("T,E,H,I,k,widths", [
     (1, 8, 128, 64, 2, [4]), (7, 6, 192, 128, 2, [6]), (64, 5, 64, 64, 3, [8]), (300, 9, 256, 192, 4, [4, 6, 8]),
     (129, 33, 128, 64, 8, [4, 8]), (40, 16, 320, 128, 16, [6, 4]),
-    (700, 4, 192, 128, 2, [4, 8]), (1200, 3, 128, 64, 1, [6])])
+    (700, 4, 192, 128, 2, [4, 8]), (1200, 3, 128, 64, 1, [6]),
+    (64, 1024, 128, 64, 32, [4, 8])])   # the largest E and k
 def test_prefill_hand_layers(T, E, H, I, k, widths):
     rng = np.random.default_rng(T * 10 + E)
     exs = [pins.make_expert(rng, H, I, widths[e % len(widths)])[0] for e in range(E)]
