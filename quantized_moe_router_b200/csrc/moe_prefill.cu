@@ -38,15 +38,27 @@ __global__ void bucket_hist_kernel(const int32_t *idx, int T, int k, int E, int3
 }
 
 // counts[e], offsets[e] (exclusive scan, offsets[E] = T*k) and, in place, blockhist[b][e] ->
-// first output position of block b's pairs of expert e.
+// first output position of block b's pairs of expert e. One CTA of 1024 threads; each expert's
+// token blocks are split over tpe = 1024 / E threads (rounded down to a power of two), so that
+// the per-expert walks over the blocks are tpe times shorter.
 __global__ void bucket_scan_kernel(int32_t *blockhist, int nblk, int E, int32_t *counts, int32_t *offsets) {
     __shared__ int warp_tot[32];
-    const int e = threadIdx.x;  // blockDim.x = 1024 >= E
+    __shared__ int part[1024];      // part[e * tpe + q]: pairs of expert e in thread q's blocks
+    __shared__ int excl_e[kMaxE];
+    int tpe = 1;
+    while (tpe * 2 * E <= 1024) tpe *= 2;
+    const int tid = threadIdx.x, ex = tid / tpe, q = tid - ex * tpe;
+    const int b0 = (int)((long long)nblk * q / tpe), b1 = (int)((long long)nblk * (q + 1) / tpe);
+    int mine = 0;
+    if (ex < E)
+        for (int b = b0; b < b1; ++b) mine += blockhist[(size_t)b * E + ex];
+    part[tid] = mine;
+    __syncthreads();
+    // block-wide exclusive scan of the experts' totals (thread e holds expert e's)
+    const int e = tid, lane = tid & 31, w = tid >> 5;
     int c = 0;
     if (e < E)
-        for (int b = 0; b < nblk; ++b) c += blockhist[(size_t)b * E + e];
-    // block-wide exclusive scan of c
-    const int lane = e & 31, w = e >> 5;
+        for (int j = 0; j < tpe; ++j) c += part[e * tpe + j];
     int incl = c;
     for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
@@ -64,15 +76,20 @@ __global__ void bucket_scan_kernel(int32_t *blockhist, int nblk, int E, int32_t 
         warp_tot[lane] = iv - v;
     }
     __syncthreads();
-    const int excl = warp_tot[w] + incl - c;
     if (e < E) {
+        const int excl = warp_tot[w] + incl - c;
         counts[e] = c;
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = excl + c;
-        int run = excl;
-        for (int b = 0; b < nblk; ++b) {
-            const int h = blockhist[(size_t)b * E + e];
-            blockhist[(size_t)b * E + e] = run;
+        excl_e[e] = excl;
+    }
+    __syncthreads();
+    if (ex < E) {
+        int run = excl_e[ex];
+        for (int j = 0; j < q; ++j) run += part[ex * tpe + j];
+        for (int b = b0; b < b1; ++b) {
+            const int h = blockhist[(size_t)b * E + ex];
+            blockhist[(size_t)b * E + ex] = run;
             run += h;
         }
     }

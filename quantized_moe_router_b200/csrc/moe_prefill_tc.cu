@@ -805,22 +805,36 @@ __global__ void h16_rescale_kernel(uint16_t *h16, const int8_t *hexp, const floa
     const int lane = threadIdx.x & 31;
     const int SUB = I / 16;
     for (int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += gridDim.x * (blockDim.x / 32)) {
-        int m = -128;
-        for (int sb = lane; sb < SUB; sb += 32) m = max(m, (int)hexp[(size_t)p * SUB + sb]);
+        // the row's chunks are loaded before the exponents are reduced, so the two loads overlap
+        // (8 fp16 per 16-byte chunk, two chunks per 16-column block; I <= 1024: 4 per lane)
+        uint4 *row = reinterpret_cast<uint4 *>(h16 + (size_t)p * I);
+        uint4 v[4];
+        int eb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int ch = lane + 32 * i;
+            if (ch < I / 8) {
+                v[i] = row[ch];
+                eb[i] = (int)hexp[(size_t)p * SUB + ch / 2];
+            } else {
+                eb[i] = -128;
+            }
+        }
+        int m = max(max(eb[0], eb[1]), max(eb[2], eb[3]));
         m = __reduce_max_sync(0xffffffffu, m);
         if (lane == 0) pscale[p] = __ldg(pair_w + p) * exp2i(m);
-        // 8 fp16 per 16-byte chunk, two chunks per 16-column block
-        uint4 *row = reinterpret_cast<uint4 *>(h16 + (size_t)p * I);
-        for (int ch = lane; ch < I / 8; ch += 32) {
-            const int d = (int)hexp[(size_t)p * SUB + ch / 2] - m;
-            if (d == 0) continue;
-            const uint32_t f = h2_pow2(d);
-            uint4 v = row[ch];
-            v.x = hmul2_bits(v.x, f);
-            v.y = hmul2_bits(v.y, f);
-            v.z = hmul2_bits(v.z, f);
-            v.w = hmul2_bits(v.w, f);
-            row[ch] = v;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int ch = lane + 32 * i;
+            const int d = eb[i] - m;
+            if (ch < I / 8 && d != 0) {
+                const uint32_t f = h2_pow2(d);
+                v[i].x = hmul2_bits(v[i].x, f);
+                v[i].y = hmul2_bits(v[i].y, f);
+                v[i].z = hmul2_bits(v[i].z, f);
+                v[i].w = hmul2_bits(v[i].w, f);
+                row[ch] = v[i];
+            }
         }
     }
 }
