@@ -741,12 +741,13 @@ def quantizer_leg():
         qm.quantize_hqq(wt, bits, with_iters=True)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 3
-        e0.record()
-        for _ in range(reps):
-            codes, sc, zr, it = qm.quantize_hqq(wt, bits, with_iters=True)
-        e1.record()
-        torch.cuda.synchronize()
+        reps = 20
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            e0.record()
+            for _ in range(reps):
+                codes, sc, zr, it = qm.quantize_hqq(wt, bits, with_iters=True)
+            e1.record()
+            torch.cuda.synchronize()
         t = e0.elapsed_time(e1) * 1e-3 / reps
         steps = it.to(torch.int64)
         ops = 64.0 * float((10 * steps + 15 * (steps - 1).clamp(min=0)).sum())
@@ -754,7 +755,8 @@ def quantizer_leg():
                "mean_steps": float(steps.float().mean()),
                "roofline": {"bound": "alu", "achieved": ops / t / 1e12, "peak": FP64_OPS_PEAK / 1e12,
                             "unit": "T fp64 op/s", "frac": ops / t / FP64_OPS_PEAK, "traffic": None,
-                            "peak_source": "148 SMs x 64 fp64 lanes x 1.965 GHz (nominal issue rate)"}}
+                            "peak_source": "148 SMs x 64 fp64 lanes x 1.965 GHz (nominal issue rate)"},
+               "clocks": clk.summary()}
         if label.startswith("gate_up_I512"):
             # stored zeros against the oracle on the first 512 rows (one expert's gate matrix)
             wb = wt[:512].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
@@ -853,12 +855,13 @@ def streamed_leg(slot_counts=(96, 256, 640), L=4, S=4):
             torch.cuda.synchronize()
             h0 = cache.stats()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            t0 = time.perf_counter()
-            e0.record(comp)
-            loaded = sum(run(s, False) for s in range(S))
-            e1.record(comp)
-            torch.cuda.synchronize()
-            wall = time.perf_counter() - t0
+            with ClockSampler(torch.cuda.current_device()) as clk:
+                t0 = time.perf_counter()
+                e0.record(comp)
+                loaded = sum(run(s, False) for s in range(S))
+                e1.record(comp)
+                torch.cuda.synchronize()
+                wall = time.perf_counter() - t0
             dev = e0.elapsed_time(e1) * 1e-3
             h1 = cache.stats()
             hits, miss = h1["hits"] - h0["hits"], h1["misses"] - h0["misses"]
@@ -868,7 +871,8 @@ def streamed_leg(slot_counts=(96, 256, 640), L=4, S=4):
             assert qm.device_status(ws) == qm.MOE_OK
             ent[sched] = {"tokens_per_s": w.T * S / dev, "ms_per_token_step": dev / S * 1e3,
                           "host_GBps": loaded / dev / 1e9, "hit_rate": hits / max(1, hits + miss),
-                          "expert_misses": miss, "wall_s": wall, "calls_outside_request": outside}
+                          "expert_misses": miss, "wall_s": wall, "calls_outside_request": outside,
+                          "clocks": clk.summary()}
             cache.close()
         res[f"slots_{slots}"] = ent
     return {"workload": f"{w.name} (first {L} layers in pinned host memory, {w.T} tokens per call, {S} steps)",
@@ -882,10 +886,17 @@ def next_rows_leg(args, world, rank):
     mixed = dataclasses.replace(pw, name="prefill_t4096_l2_h2048_e256_k8_i512_mixed468", mixed_bits=True, layers=2)
     a2 = argparse.Namespace(**vars(args))
     a2.no_cpu_baseline = True
-    a2.steps = min(args.steps, 5)
-    return {"quantizer": quantizer_leg(),
-            "streamed_decode": streamed_leg(),
-            "mixed_prefill": prefill_leg(a2, mixed, world, rank)}
+    a2.steps = 40   # ~50 ms timed: enough clock samples
+
+    def guarded(fn, *fa):
+        # a failing next row is reported in its entry and does not take the benchmark line down
+        try:
+            return fn(*fa)
+        except Exception as ex:  # noqa: BLE001
+            return {"error": f"{type(ex).__name__}: {ex}"[:300]}
+    return {"quantizer": guarded(quantizer_leg),
+            "streamed_decode": guarded(streamed_leg),
+            "mixed_prefill": guarded(prefill_leg, a2, mixed, world, rank)}
 
 
 def leg(args, w, world, rank):
